@@ -1,0 +1,117 @@
+"""Pins for the oracle's QLoRA linear and gated-MLP forward/backward.
+
+The matmul library routine is cross-checked by explicit loops; gradients are
+checked by central finite differences of <dY, Y> in float64; invariants that
+follow from the algebra on the pages (B = 0, alpha = 0) and the page's
+adapter-count example are checked directly.
+"""
+import numpy as np
+import pytest
+
+from oracle import lora, nf4
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+def test_forward_matches_triple_loop():
+    rng = np.random.default_rng(0)
+    M, N, K, r, s = 3, 5, 4, 2, 1.5
+    X, W, A, B = _rand(rng, M, K), _rand(rng, N, K), _rand(rng, r, K), _rand(rng, N, r)
+    Y, U = lora.forward(X, W, A, B, s, materialize=False)
+    for m in range(M):
+        for n in range(N):
+            u = [sum(X[m, k] * A[j, k] for k in range(K)) for j in range(r)]
+            y = sum(X[m, k] * W[n, k] for k in range(K)) + s * sum(u[j] * B[n, j] for j in range(r))
+            assert Y[m, n] == pytest.approx(y, rel=1e-12, abs=1e-12)
+
+
+def _fd(f, P, eps=1e-6):
+    g = np.zeros_like(P)
+    it = np.nditer(P, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = P[i]
+        P[i] = old + eps
+        fp = f()
+        P[i] = old - eps
+        fm = f()
+        P[i] = old
+        g[i] = (fp - fm) / (2 * eps)
+    return g
+
+
+def test_backward_matches_finite_differences():
+    rng = np.random.default_rng(1)
+    M, N, K, r, s = 4, 6, 5, 3, 0.75
+    X, W, A, B, dY = (_rand(rng, M, K), _rand(rng, N, K), _rand(rng, r, K),
+                      _rand(rng, N, r), _rand(rng, M, N))
+    loss = lambda: float(np.sum(dY * lora.forward(X, W, A, B, s, materialize=False)[0]))
+    g = lora.backward(X, W, A, B, s, dY, materialize=False)
+    for name, P in (("dX", X), ("dA", A), ("dB", B)):
+        num = _fd(loss, P)
+        assert np.allclose(g[name], num, rtol=1e-8, atol=1e-8), name
+
+
+def test_invariants_B_zero_and_alpha_zero():
+    rng = np.random.default_rng(2)
+    M, N, K, r = 4, 6, 5, 3
+    X, W, A, dY = _rand(rng, M, K), _rand(rng, N, K), _rand(rng, r, K), _rand(rng, M, N)
+    B0 = np.zeros((N, r))
+    Y, _ = lora.forward(X, W, A, B0, 2.0)
+    assert np.array_equal(Y, X @ W.T)
+    g = lora.backward(X, W, A, B0, 2.0, dY)
+    assert np.all(g["dA"] == 0)
+    B = _rand(rng, N, r)
+    g0 = lora.backward(X, W, A, B, 0.0, dY)
+    assert np.all(g0["dA"] == 0) and np.all(g0["dB"] == 0)
+    assert np.array_equal(g0["dX"], dY @ W)
+
+
+def test_adapter_count_from_page(golden):
+    g = golden["adapter_params_4096_r16"]
+    assert lora.adapter_param_count(g["d"], g["k"], g["r"]) == g["value"]
+
+
+def test_materialized_U_V_are_bf16():
+    rng = np.random.default_rng(3)
+    X, W, A, B, dY = (_rand(rng, 4, 8), _rand(rng, 6, 8), _rand(rng, 2, 8),
+                      _rand(rng, 6, 2), _rand(rng, 4, 6))
+    from oracle.formats import bf16
+    _, U = lora.forward(X, W, A, B, 1.0)
+    g = lora.backward(X, W, A, B, 1.0, dY)
+    assert np.array_equal(U, bf16(X @ A.T)) and np.array_equal(g["V"], bf16(dY @ B))
+
+
+def test_mlp_backward_matches_finite_differences():
+    rng = np.random.default_rng(4)
+    M, D, H, r, s = 3, 4, 5, 2, 0.5
+    Wg, Wu, Wd = _rand(rng, H, D), _rand(rng, H, D), _rand(rng, D, H)
+    Ag, Au, Ad = _rand(rng, r, D), _rand(rng, r, D), _rand(rng, r, H)
+    Bg, Bu, Bd = _rand(rng, H, r), _rand(rng, H, r), _rand(rng, D, r)
+    X, dy = _rand(rng, M, D), _rand(rng, M, D)
+    args = lambda: (X, Wg, Ag, Bg, Wu, Au, Bu, Wd, Ad, Bd, s)
+    loss = lambda: float(np.sum(dy * lora.mlp_forward(*args(), materialize=False)["y"]))
+    fwd = lora.mlp_forward(*args(), materialize=False)
+    g = lora.mlp_backward(*args(), dy, fwd, materialize=False)
+    for name, P in (("dX", X), ("dAg", Ag), ("dBg", Bg), ("dAu", Au), ("dBu", Bu),
+                    ("dAd", Ad), ("dBd", Bd)):
+        assert np.allclose(g[name], _fd(loss, P), rtol=1e-7, atol=1e-8), name
+
+
+def test_silu_special_values():
+    assert lora.silu(np.array([0.0]))[0] == 0.0
+    x = np.array([-3.0, 1.0, 20.0])
+    assert np.allclose(lora.silu(x), x / (1 + np.exp(-x)), rtol=0, atol=0)
+
+
+def test_dequant_then_linear_uses_table_values():
+    """A weight that is exactly c * q_j quantizes to code j and comes back exact."""
+    q = nf4.codebook()
+    c = 0.5
+    w = np.tile(q * c, 4)[: 64]              # one block: absmax c, every level present
+    packed, cb, _ = nf4.quantize(w)
+    assert cb[0] == c
+    what = nf4.dequant(packed, 64, cb, out="f32")
+    assert np.array_equal(what, w)
