@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  nf4_quantize (fp32 W -> NF4 codes + fp32 absmax)
+  nf4_double_quant (absmax -> E4M3 codes + group scales + mean)
+  qlora_linear_fwd (U = X A^T, Y = X dequant(W)^T + s U B^T; dequant fused)
+  qlora_linear_bwd (V, dB, dX = dY dequant(W) + s V A, dA)
+On the 4096 x 4096 projection with 4096 tokens, r = 16, alpha = 32 (the
+metric's workload).  Throughput counts the GEMM work 4 M N K + 6 M r (K + N)
+per step (dequantization and quantization are not counted as FLOPs).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun (N > 1) every rank runs its own batch (weak scaling) and the
+adapter gradients dA, dB are all-reduced over NCCL each step (the data-parallel
+exchange).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s & small-M weight GB/s vs B200 roofline"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-secondary", action="store_true", help="skip the small-M and codec side measurements")
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ the workload
+class Projection:
+    """The 4096 x 4096 projection workload, resident on one device."""
+
+    def __init__(self, q, dev, rank=0):
+        import torch
+        from synthetic import inputs as S
+        self.q, self.dev = q, dev
+        w = S.WORKLOADS["c2"]
+        self.w = w
+        lin = w.linears[0]
+        self.N, self.K, self.M, self.r, self.s = lin.N, lin.K, w.M, w.r, w.s
+        d = S.linear_inputs(w, 0, device=dev)
+        self.W, self.X, self.A, self.B, self.dY = d["W"], d["X"], d["A"], d["B"], d["dY"]
+        if rank:   # a different batch per rank, same weights
+            self.X = S.normal((self.M, self.K), 1.0, 100000 + rank, device=dev, dtype=torch.bfloat16)
+            self.dY = S.normal((self.M, self.N), 1.0, 200000 + rank, device=dev, dtype=torch.bfloat16)
+        self.wq = q.NF4Weight.allocate(self.N, self.K, dev, dq=True)
+        n = self.N * self.K
+        self.absmax = torch.empty(-(-n // 64), dtype=torch.float32, device=dev)
+        self.ws_dq = torch.empty(q.qlora_workspace_size(q.QL_OP_DOUBLE_QUANT, self.absmax.numel()),
+                                 dtype=torch.uint8, device=dev)
+        self.Y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=dev)
+        self.U = torch.empty(self.M, self.r, dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty(self.M, self.K, dtype=torch.bfloat16, device=dev)
+        self.dA = torch.empty(self.r, self.K, dtype=torch.float32, device=dev)
+        self.dB = torch.empty(self.N, self.r, dtype=torch.float32, device=dev)
+        self.ws = torch.empty(q.qlora_workspace_size(q.QL_OP_BWD, self.M, self.N, self.K, self.r),
+                              dtype=torch.uint8, device=dev)
+
+    @property
+    def flops(self) -> float:
+        M, N, K, r = self.M, self.N, self.K, self.r
+        return 4.0 * M * N * K + 6.0 * M * r * (K + N)
+
+    def gemm_flops(self) -> tuple[float, float]:
+        M, N, K, r = self.M, self.N, self.K, self.r
+        return 2.0 * M * N * K + 2.0 * M * r * N, 2.0 * M * N * K + 2.0 * M * r * K
+
+    def step(self, allreduce=None):
+        q = self.q
+        q.nf4_quantize(self.W, self.wq.codes, self.absmax)
+        q.nf4_double_quant(self.absmax, self.wq.absmax_q, self.wq.scale2, self.wq.offset, self.ws_dq)
+        q.qlora_linear_fwd(self.wq, self.X, self.A, self.B, self.r, self.s, self.Y, U_out=self.U, ws=self.ws)
+        q.qlora_linear_bwd(self.wq, self.X, self.dY, self.A, self.B, self.r, self.s, self.U, self.dX, self.dA,
+                           self.dB, ws=self.ws)
+        if allreduce:
+            allreduce(self.dA)
+            allreduce(self.dB)
+
+
+def trace_read(q):
+    import ctypes
+    L = q._lib.LIB
+    L.qlora_trace_read.restype = ctypes.c_int
+    L.qlora_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+    L.qlora_trace_kind_name.restype = ctypes.c_char_p
+    L.qlora_trace_kind_name.argtypes = [ctypes.c_int]
+    ms = (ctypes.c_double * 32)()
+    cnt = (ctypes.c_int * 32)()
+    n = L.qlora_trace_read(ms, cnt, 32)
+    return {L.qlora_trace_kind_name(k).decode(): (ms[k], cnt[k]) for k in range(n) if cnt[k]}
+
+
+def trace_enable(q, on):
+    import ctypes
+    L = q._lib.LIB
+    L.qlora_trace_enable.argtypes = [ctypes.c_int]
+    L.qlora_trace_enable.restype = None
+    L.qlora_trace_enable(1 if on else 0)
+
+
+# --------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(rows: int = 256, tokens: int = 256):
+    """The oracle on a bounded sample of the projection step: quantize + double
+    quant + dequant of `rows` weight rows, fwd + bwd for `tokens` tokens."""
+    import numpy as np
+    from oracle import lora, nf4
+    from synthetic import inputs as S
+    w = S.WORKLOADS["c2"]
+    d = S.linear_inputs(w, 0)
+    W = d["W"][:rows]
+    X, dY = d["X"][:tokens], d["dY"][:tokens, :rows]
+    A, B = d["A"], d["B"][:rows]
+    K = W.shape[1]
+    t0 = time.perf_counter()
+    packed, c, _ = nf4.quantize(W)
+    e, s2, mu = nf4.double_quant(c)
+    What = nf4.dequant(packed, rows * K, nf4.dq_constants(e, s2, mu)).reshape(rows, K)
+    Y, U = lora.forward(X, What, A, B, w.s)
+    lora.backward(X, What, A, B, w.s, dY, U=U)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * tokens * rows * K + 6.0 * tokens * w.r * (K + rows)
+    return flops, dt, f"weight rows {rows} of 4096 (quantize, double quant, dequant), fwd+bwd on {tokens} of 4096 tokens"
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------- secondary lines
+def small_m_and_codec(q, dev, hbm_peak):
+    """Small-token forward on the 28672 x 8192 weight (HBM-bound on the packed
+    weight) and the standalone quantize + double quant over 4 Gi bf16 elements."""
+    import torch
+    from synthetic import inputs as S
+    out = {}
+    w5 = S.WORKLOADS["c5"]
+    lin = w5.linears[0]
+    N, K, r, s = lin.N, lin.K, w5.r, w5.s
+    W = S.normal((N, K), w5.wstd, S.seed_of(5, 0, "W"), device=dev)
+    wq = q.quantize_weight(W, dq=True)
+    del W
+    A = S.uniform((r, K), 1.0 / K ** 0.5, S.seed_of(5, 0, "A"), device=dev)
+    B = S.normal((N, r), 0.01, S.seed_of(5, 0, "B"), device=dev, dtype=torch.bfloat16)
+    wbytes = q.nf4_storage_bytes(N * K, True)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for M in w5.Ms:
+        X = S.normal((M, K), 1.0, S.seed_of(5, 0, "X") + M, device=dev, dtype=torch.bfloat16)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, q.qlora_workspace_size(q.QL_OP_FWD, M, N, K, r)), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            q.qlora_linear_fwd(wq, X, A, B, r, s, Y, ws=ws)
+        times = []
+        for _ in range(20):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            q.qlora_linear_fwd(wq, X, A, B, r, s, Y, ws=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        t = statistics.median(times) / 1e3
+        gbs = wbytes / t / 1e9
+        out[f"M{M}"] = {"us": round(t * 1e6, 2), "weight_GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 3)}
+    del wq
+    torch.cuda.empty_cache()
+    # codec over 4 Gi bf16 elements
+    n = w5.codec_n
+    x = S.codec_tensor(n, 0.02, S.seed_of(5, 9, "W"), device=dev)
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+    aq = torch.empty(n // 64, dtype=torch.uint8, device=dev)
+    s2 = torch.empty(-(-n // 64 // 256), dtype=torch.float32, device=dev)
+    mu = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(q.qlora_workspace_size(q.QL_OP_DOUBLE_QUANT, n // 64), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        q.nf4_quantize(x, codes, absmax)
+        q.nf4_double_quant(absmax, aq, s2, mu, ws)
+    times = []
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        q.nf4_quantize(x, codes, absmax)
+        q.nf4_double_quant(absmax, aq, s2, mu, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    t = statistics.median(times) / 1e3
+    # bytes that must move: read x, write codes + absmax, read absmax twice (mean, encode), write E4M3 + scales
+    nb = n // 64
+    moved = 2 * n + n // 2 + 4 * nb + 2 * 4 * nb + nb + 4 * (nb // 256)
+    out["codec_4Gi_bf16"] = {"ms": round(t * 1e3, 3), "GBps": round(moved / t / 1e9, 1),
+                             "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3), "bytes": moved}
+    del x, codes, absmax, aq
+    torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------------- arms
+def run_reference(args, rank):
+    """The oracle (CPU, float64 numpy) as the reference arm, rank 0 only."""
+    if rank != 0:
+        return
+    for _ in range(max(0, min(args.warmup, 1))):
+        cpu_oracle_sample(64, 64)
+    total_f, total_t = 0.0, 0.0
+    desc = ""
+    for _ in range(args.steps):
+        f, t, desc = cpu_oracle_sample(128, 128)
+        total_f += f
+        total_t += t
+    v = total_f / total_t / 1e12
+    line = {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": "projection 4096x4096, 4096 tokens, r=16, alpha=32, NF4+DQ, fwd+bwd",
+                       "global_batch": 4096, "parallelism": "cpu oracle"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import bit_nf4_quantized_10_b200 as q
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hbm_peak, bf16_peak, bf16_sus, peak_src = peaks()
+    wl = Projection(q, dev, rank)
+    allreduce = None
+    if world > 1:
+        allreduce = lambda t: dist.all_reduce(t)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2 (126 MB)
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    t_warm = time.time()
+    for _ in range(args.warmup):
+        wl.step(allreduce)
+    torch.cuda.synchronize()
+    while time.time() - t_warm < 0.5:          # give the clock sampler samples under load
+        wl.step(allreduce)
+        torch.cuda.synchronize()
+    st = q.qlora_get_status()
+    if st != q.QL_OK:
+        raise RuntimeError(f"device status after warm-up: {q.status_string(st)}")
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    trace_enable(q, True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record()
+        wl.step(allreduce)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    kern = trace_read(q)
+    trace_enable(q, False)
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_s = sum(step_ms) / 1e3
+    if world > 1:
+        tt = torch.tensor([total_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_s = float(tt.item())
+    st = q.qlora_get_status()
+    if st != q.QL_OK:
+        raise RuntimeError(f"device status after timing: {q.status_string(st)}")
+    value = world * args.steps * wl.flops / total_s / 1e12
+
+    # dominant kernel: the fused dequant GEMM (forward and backward launches)
+    f_fwd, f_bwd = wl.gemm_flops()
+    ms_f, n_f = kern.get("qlora_gemm_fwd", (0.0, 0))
+    ms_b, n_b = kern.get("qlora_gemm_bwd", (0.0, 0))
+    gemm_ms = ms_f + ms_b
+    gemm_launches = n_f + n_b
+    achieved = (n_f * f_fwd + n_b * f_bwd) / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
+    gpu_launches = sum(c for _, c in kern.values())
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if rank == 0 or world > 1:
+        hW = torch.empty_like(wl.W, device="cpu").pin_memory().copy_(wl.W)
+        hX = torch.empty_like(wl.X, device="cpu").pin_memory().copy_(wl.X)
+        hA = torch.empty_like(wl.A, device="cpu").pin_memory().copy_(wl.A)
+        hB = torch.empty_like(wl.B, device="cpu").pin_memory().copy_(wl.B)
+        hdY = torch.empty_like(wl.dY, device="cpu").pin_memory().copy_(wl.dY)
+        oY = torch.empty_like(wl.Y, device="cpu").pin_memory()
+        odX = torch.empty_like(wl.dX, device="cpu").pin_memory()
+        odA = torch.empty_like(wl.dA, device="cpu").pin_memory()
+        odB = torch.empty_like(wl.dB, device="cpu").pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hW, hX, hA, hB, hdY))
+        d2h = sum(t.numel() * t.element_size() for t in (oY, odX, odA, odB))
+
+        def e2e_step():
+            wl.W.copy_(hW, non_blocking=True)
+            wl.X.copy_(hX, non_blocking=True)
+            wl.A.copy_(hA, non_blocking=True)
+            wl.B.copy_(hB, non_blocking=True)
+            wl.dY.copy_(hdY, non_blocking=True)
+            wl.step(allreduce)
+            oY.copy_(wl.Y, non_blocking=True)
+            odX.copy_(wl.dX, non_blocking=True)
+            odA.copy_(wl.dA, non_blocking=True)
+            odB.copy_(wl.dB, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(5, args.steps // 2)
+        e0.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        t_e2e = e0.elapsed_time(e1) / 1e3
+        if world > 1:
+            tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            t_e2e = float(tt.item())
+        e2e = {"value": world * n_e2e * wl.flops / t_e2e / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    secondary = None
+    if rank == 0 and not args.no_secondary:
+        del flush
+        torch.cuda.empty_cache()
+        secondary = small_m_and_codec(q, dev, hbm_peak)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        f, t, desc = cpu_oracle_sample(1024, 512)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc + f" ({t:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "projection 4096x4096 NF4+DQ, 4096 tokens/GPU, r=16, alpha=32: quantize + "
+                                   "double quant + fwd + bwd (dX, dA, dB)",
+                       "global_batch": 4096 * world, "N": 4096, "K": 4096, "r": 16,
+                       "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, untimed)",
+                       "outputs": "Y, dX bf16; dA, dB fp32"},
+            "roofline": {"bound": "tensor", "kernel": "qlora_gemm (fused NF4 dequant + tcgen05 GEMM + LoRA)",
+                         "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                         "frac": achieved / bf16_peak, "peak_source": f"{peak_src} bf16 burst",
+                         "traffic": None, "launches": gemm_launches,
+                         "avg_launch_us": gemm_ms / max(gemm_launches, 1) * 1e3},
+            "kernels": {k: {"ms_total": round(v[0], 4), "launches": v[1]} for k, v in kern.items()},
+            "gpu_launches": gpu_launches,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clk,
+            "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,222 @@
+// C ABI of the library: argument checks, workspace carving and the launch
+// sequences of each call.  Argument errors return before anything is launched.
+#include <cstring>
+
+#include "common.cuh"
+
+namespace ql {
+// codec.cu
+ql_status launch_quantize(const void* x, ql_dtype dt, int64_t n, uint8_t* codes, float* absmax, cudaStream_t st);
+size_t dq_workspace_bytes(int64_t nb);
+ql_status launch_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q, float* scale2, float* offset,
+                              void* ws, cudaStream_t st);
+ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStream_t st);
+unsigned status_word_codec(cudaStream_t st);
+// gemm.cu
+ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
+                          float s, void* Y, ql_dtype y_dt, cudaStream_t st);
+ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* V, const void* A, int r,
+                          float s, void* dX, ql_dtype dx_dt, int accumulate, cudaStream_t st);
+unsigned status_word_gemm(cudaStream_t st);
+// lora_side.cu
+ql_status launch_proj_xa(const void* X, int64_t M, int K, const void* A, int r, void* U, cudaStream_t st);
+ql_status launch_proj_dyb(const void* dY, int64_t M, int N, const void* B, int r, void* V, cudaStream_t st);
+size_t colacc_partial_bytes(int64_t M, int64_t ncols, int r);
+ql_status launch_colacc(const void* act, int64_t M, int ncols, const void* G, int r, float s, int transpose,
+                        void* out, ql_dtype out_dt, float* partial, cudaStream_t st);
+// mlp.cu
+ql_status launch_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, cudaStream_t st);
+ql_status launch_silu_gate_bwd(const void* dh, const void* g, const void* u, void* dg, void* du, int64_t n,
+                               cudaStream_t st);
+}  // namespace ql
+
+namespace {
+
+inline bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool dtype_ok(ql_dtype d) { return d == QL_F32 || d == QL_BF16; }
+inline size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Weight descriptor checks shared by dequant and the GEMM calls.
+ql_status check_weight(const ql_nf4_weight* w) {
+  if (!w || w->rows <= 0 || w->cols <= 0) return QL_ERR_INVALID_ARG;
+  if (!aligned16(w->codes)) return QL_ERR_INVALID_ARG;
+  if (w->absmax) {
+    if (!aligned16(w->absmax)) return QL_ERR_INVALID_ARG;
+  } else {
+    if (!aligned16(w->absmax_q) || !aligned16(w->scale2) || !aligned16(w->offset)) return QL_ERR_INVALID_ARG;
+  }
+  return QL_OK;
+}
+
+ql_status check_gemm_shape(const ql_nf4_weight* w, int64_t M, int r) {
+  ql_status st = check_weight(w);
+  if (st != QL_OK) return st;
+  if (M < 0) return QL_ERR_INVALID_ARG;
+  if (w->cols % 64 != 0 || w->rows % 8 != 0) return QL_ERR_INVALID_ARG;
+  if (M >= (1ll << 31) || w->rows >= (1ll << 31) || w->cols >= (1ll << 31)) return QL_ERR_UNSUPPORTED;
+  if (r < 0 || r % 8 != 0) return QL_ERR_INVALID_ARG;
+  if (r > QL_MAX_RANK) return QL_ERR_UNSUPPORTED;
+  return QL_OK;
+}
+
+size_t ws_fwd(int64_t M, int r) { return r > 0 ? align256((size_t)M * r * 2) : 0; }
+
+size_t ws_bwd(int64_t M, int64_t N, int64_t K, int r) {
+  if (r == 0) return 0;
+  size_t part = ql::colacc_partial_bytes(M, N, r);
+  size_t part2 = ql::colacc_partial_bytes(M, K, r);
+  if (part2 > part) part = part2;
+  return 2 * align256((size_t)M * r * 2) + align256(part);
+}
+
+}  // namespace
+
+extern "C" {
+
+ql_status nf4_quantize(const void* x, ql_dtype x_dt, int64_t n, uint8_t* codes, float* absmax, void* stream) {
+  if (n <= 0 || !dtype_ok(x_dt)) return QL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(absmax)) return QL_ERR_INVALID_ARG;
+  return ql::launch_quantize(x, x_dt, n, codes, absmax, as_stream(stream));
+}
+
+ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q, float* scale2, float* offset,
+                           void* ws, size_t ws_bytes, void* stream) {
+  if (nb <= 0) return QL_ERR_INVALID_ARG;
+  if (!aligned16(absmax) || !aligned16(absmax_q) || !aligned16(scale2) || !aligned16(offset) || !aligned16(ws))
+    return QL_ERR_INVALID_ARG;
+  if (ws_bytes < ql::dq_workspace_bytes(nb)) return QL_ERR_WORKSPACE;
+  return ql::launch_double_quant(absmax, nb, absmax_q, scale2, offset, ws, as_stream(stream));
+}
+
+ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* stream) {
+  ql_status st = check_weight(w);
+  if (st != QL_OK) return st;
+  if (!dtype_ok(out_dt) || !aligned16(out)) return QL_ERR_INVALID_ARG;
+  return ql::launch_dequant(w, out, out_dt, as_stream(stream));
+}
+
+ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* A, const void* B, int r,
+                           float s, void* Y, ql_dtype y_dt, void* U_out, void* ws, size_t ws_bytes, void* stream) {
+  ql_status st = check_gemm_shape(w, M, r);
+  if (st != QL_OK) return st;
+  if (!dtype_ok(y_dt) || !aligned16(X) || !aligned16(Y)) return QL_ERR_INVALID_ARG;
+  if (r > 0 && (!aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
+  if (U_out && !aligned16(U_out)) return QL_ERR_INVALID_ARG;
+  if (M == 0) return QL_OK;
+  void* U = U_out;
+  if (r > 0 && !U) {
+    if (ws_bytes < ws_fwd(M, r)) return QL_ERR_WORKSPACE;
+    if (!aligned16(ws)) return QL_ERR_INVALID_ARG;
+    U = ws;
+  }
+  cudaStream_t cs = as_stream(stream);
+  const int K = (int)w->cols;
+  if (r > 0) {
+    st = ql::launch_proj_xa(X, M, K, A, r, U, cs);
+    if (st != QL_OK) return st;
+  }
+  return ql::launch_gemm_fwd(w, X, M, U, B, r, s, Y, y_dt, cs);
+}
+
+ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
+                           const void* B, int r, float s, const void* U, void* dX, ql_dtype dx_dt, int accumulate_dx,
+                           void* dA, void* dB, ql_dtype grad_dt, void* ws, size_t ws_bytes, void* stream) {
+  ql_status st = check_gemm_shape(w, M, r);
+  if (st != QL_OK) return st;
+  if (!dtype_ok(dx_dt) || !dtype_ok(grad_dt) || !aligned16(dY) || !aligned16(dX)) return QL_ERR_INVALID_ARG;
+  if (r > 0 && (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(dA) || !aligned16(dB)))
+    return QL_ERR_INVALID_ARG;
+  if (U && !aligned16(U)) return QL_ERR_INVALID_ARG;
+  const int64_t N = w->rows, K = w->cols;
+  if (r > 0 && ws_bytes < ws_bwd(M, N, K, r)) return QL_ERR_WORKSPACE;
+  if (r > 0 && !aligned16(ws)) return QL_ERR_INVALID_ARG;
+  cudaStream_t cs = as_stream(stream);
+  if (M == 0) {
+    // no tokens: the adapter gradients are zero, dX is empty
+    if (r > 0) {
+      const size_t e = grad_dt == QL_F32 ? 4 : 2;
+      QL_CUDA_TRY(cudaMemsetAsync(dA, 0, (size_t)r * K * e, cs));
+      QL_CUDA_TRY(cudaMemsetAsync(dB, 0, (size_t)N * r * e, cs));
+    }
+    return QL_OK;
+  }
+  if (r == 0) return ql::launch_gemm_bwd(w, dY, M, nullptr, nullptr, 0, s, dX, dx_dt, accumulate_dx, cs);
+  uint8_t* wp = reinterpret_cast<uint8_t*>(ws);
+  void* Uw = wp;
+  wp += align256((size_t)M * r * 2);
+  void* V = wp;
+  wp += align256((size_t)M * r * 2);
+  float* partial = reinterpret_cast<float*>(wp);
+  if (!U) {
+    st = ql::launch_proj_xa(X, M, (int)K, A, r, Uw, cs);
+    if (st != QL_OK) return st;
+    U = Uw;
+  }
+  st = ql::launch_proj_dyb(dY, M, (int)N, B, r, V, cs);
+  if (st != QL_OK) return st;
+  st = ql::launch_colacc(dY, M, (int)N, U, r, s, 0, dB, grad_dt, partial, cs);       // dB = s dY^T U
+  if (st != QL_OK) return st;
+  st = ql::launch_gemm_bwd(w, dY, M, V, A, r, s, dX, dx_dt, accumulate_dx, cs);     // dX
+  if (st != QL_OK) return st;
+  return ql::launch_colacc(X, M, (int)K, V, r, s, 1, dA, grad_dt, partial, cs);      // dA = s V^T X
+}
+
+ql_status qlora_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, void* stream) {
+  if (n <= 0 || !aligned16(g) || !aligned16(u) || !aligned16(h)) return QL_ERR_INVALID_ARG;
+  return ql::launch_silu_gate_fwd(g, u, h, n, as_stream(stream));
+}
+
+ql_status qlora_silu_gate_bwd(const void* dh, const void* g, const void* u, void* dg, void* du, int64_t n,
+                              void* stream) {
+  if (n <= 0 || !aligned16(dh) || !aligned16(g) || !aligned16(u) || !aligned16(dg) || !aligned16(du))
+    return QL_ERR_INVALID_ARG;
+  return ql::launch_silu_gate_bwd(dh, g, u, dg, du, n, as_stream(stream));
+}
+
+size_t qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r) {
+  switch (op) {
+    case QL_OP_DOUBLE_QUANT: return M > 0 ? ql::dq_workspace_bytes(M) : 0;
+    case QL_OP_FWD: return ws_fwd(M, r);
+    case QL_OP_BWD: return ws_bwd(M, N, K, r);
+    default: return 0;
+  }
+}
+
+int64_t nf4_storage_bytes(int64_t n, int dq) {
+  if (n <= 0) return 0;
+  const int64_t nb = (n + 63) / 64;
+  const int64_t ng = (nb + 255) / 256;
+  return (n + 1) / 2 + (dq ? nb + 4 * ng + 4 : 4 * nb);
+}
+
+void nf4_codebook(float out[16]) {
+  if (out) std::memcpy(out, ql::nf4_table().q, sizeof(float) * 16);
+}
+
+ql_status qlora_get_status(void* stream) {
+  cudaStream_t cs = as_stream(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return QL_ERR_CUDA;
+  const unsigned a = ql::status_word_codec(cs);
+  const unsigned b = ql::status_word_gemm(cs);
+  if (a == ~0u || b == ~0u) return QL_ERR_CUDA;
+  const unsigned v = a | b;
+  if (v & ql::ST_NONFINITE) return QL_ERR_NONFINITE;
+  if (v & ql::ST_TIMEOUT) return QL_ERR_TIMEOUT;
+  return QL_OK;
+}
+
+const char* qlora_status_string(ql_status s) {
+  switch (s) {
+    case QL_OK: return "ok";
+    case QL_ERR_INVALID_ARG: return "invalid argument";
+    case QL_ERR_UNSUPPORTED: return "unsupported";
+    case QL_ERR_WORKSPACE: return "workspace too small";
+    case QL_ERR_CUDA: return "CUDA error";
+    case QL_ERR_NONFINITE: return "non-finite input";
+    case QL_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

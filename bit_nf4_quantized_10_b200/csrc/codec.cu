@@ -1,0 +1,353 @@
+// NF4 codec kernels: blockwise quantize + pack, double quantization of the
+// block constants, and standalone dequantization.
+//
+// "QLoRA — Fine-Tuning a 65B Model on One GPU", "Quantization in one
+// paragraph": c = max|x| per block of 64, store the index of the nearest
+// level, x_hat = c * q_index.  "QLoRA: Quantize Base Weights to 4-Bit", §2.2:
+// the fp32 constants are grouped by 256 and stored as 8-bit floats with one
+// fp32 second-level constant; "Double quantization: the constants are not
+// free" (same page 3): the mean is subtracted first.
+//
+// All kernels are HBM-bound streaming passes.  Loads and stores are 16 bytes
+// wide, grids are sized to a multiple of the SM count and loop grid-stride,
+// and every index is 64-bit so tensors above 2^32 elements work.
+#include "common.cuh"
+#include "trace.cuh"
+
+namespace ql {
+
+QL_DEFINE_STATUS_ACCESSOR(status_word_codec)
+
+// ---------------------------------------------------------------- quantize
+// Code of x: #{j : x > t_j} over the 15 sorted thresholds, found with a
+// branch-free 4-step binary search.  Ties (x == t_j) go to the lower level.
+__device__ __forceinline__ uint32_t nf4_code(float x, const float (&t)[15]) {
+  uint32_t k = (x > t[7]) ? 8u : 0u;
+  float t2 = k ? t[11] : t[3];
+  k += (x > t2) ? 4u : 0u;
+  float t1;
+  switch (k) {  // k in {0,4,8,12}; threshold index k + 1
+    case 0: t1 = t[1]; break;
+    case 4: t1 = t[5]; break;
+    case 8: t1 = t[9]; break;
+    default: t1 = t[13]; break;
+  }
+  k += (x > t1) ? 2u : 0u;
+  float t0;
+  switch (k) {  // k even; threshold index k
+    case 0: t0 = t[0]; break;
+    case 2: t0 = t[2]; break;
+    case 4: t0 = t[4]; break;
+    case 6: t0 = t[6]; break;
+    case 8: t0 = t[8]; break;
+    case 10: t0 = t[10]; break;
+    case 12: t0 = t[12]; break;
+    default: t0 = t[14]; break;
+  }
+  k += (x > t0) ? 1u : 0u;
+  return k;
+}
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* x, int64_t e0, int64_t n, float (&v)[8]);
+
+template <>
+__device__ __forceinline__ void load8<float>(const float* x, int64_t e0, int64_t n, float (&v)[8]) {
+  if (e0 + 8 <= n) {
+    float4 a = __ldcs(reinterpret_cast<const float4*>(x + e0));
+    float4 b = __ldcs(reinterpret_cast<const float4*>(x + e0) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = (e0 + i < n) ? x[e0 + i] : 0.0f;
+  }
+}
+
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* x, int64_t e0, int64_t n,
+                                                     float (&v)[8]) {
+  if (e0 + 8 <= n) {
+    uint4 a = __ldcs(reinterpret_cast<const uint4*>(x + e0));
+    uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = bf16_lo(w[i]);
+      v[2 * i + 1] = bf16_hi(w[i]);
+    }
+  } else {
+    const uint16_t* u = reinterpret_cast<const uint16_t*>(x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = (e0 + i < n) ? __uint_as_float(((uint32_t)u[e0 + i]) << 16) : 0.0f;
+  }
+}
+
+// 8 threads per 64-block, 8 consecutive elements per thread.  The loop runs
+// over blocks, so the 8 threads of a block always iterate together and can
+// reduce the absmax with shuffles.
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, int64_t n,
+                                                       uint8_t* __restrict__ codes,
+                                                       float* __restrict__ absmax, NF4Table tab) {
+  const int64_t nb = (n + 63) / 64;
+  const int lane8 = threadIdx.x & 7;
+  // the whole warp (4 blocks) iterates together so the shuffles see all lanes
+  const int64_t warps_per_grid = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t wb = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4; wb < nb;
+       wb += warps_per_grid * 4) {
+    const int64_t b = wb + ((threadIdx.x >> 3) & 3);
+    const int64_t e0 = b * 64 + lane8 * 8;   // >= n for a block past the end
+    float v[8];
+    load8<T>(x, e0, n, v);
+    float amax = 0.0f;
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float a = fabsf(v[i]);
+      bad |= !(a <= 3.402823466e38f);   // NaN or Inf
+      amax = fmaxf(amax, a);
+    }
+    unsigned anybad = bad ? 1u : 0u;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      anybad |= __shfl_xor_sync(0xffffffffu, anybad, o);
+    }
+    if (anybad && lane8 == 0) raise_status(ST_NONFINITE);
+    const float c = amax;
+    float t[15];
+#pragma unroll
+    for (int j = 0; j < 15; ++j) t[j] = __fmul_rn(tab.m[j], c);
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t code = (c == 0.0f) ? 8u : nf4_code(v[i], t);
+      word |= code << (4 * i);
+    }
+    if (e0 + 8 <= n) {
+      __stcs(reinterpret_cast<uint32_t*>(codes + (e0 >> 1)), word);
+    } else if (e0 < n) {
+      const int valid = (int)(n - e0);          // 1..7
+      for (int i = 0; i < valid; i += 2) {
+        uint32_t lo = (word >> (4 * i)) & 0xFu;
+        uint32_t hi = (i + 1 < valid) ? ((word >> (4 * (i + 1))) & 0xFu) : 8u;
+        codes[(e0 + i) >> 1] = (uint8_t)(lo | (hi << 4));
+      }
+    }
+    if (lane8 == 0 && b < nb) absmax[b] = c;
+  }
+}
+
+// --------------------------------------------------------- double quant: mean
+// Fixed adjacent-pair tree in float64.  One CTA sums 2048 consecutive inputs
+// (zero beyond `count`): 8 per thread as a 3-level tree, then the xor-shuffle
+// butterfly (offsets 1..16 combine adjacent subtrees), then the 8 warp sums as
+// a 3-level tree.  Every CTA's result is one node of the global tree, so
+// repeating the pass on the partials reproduces the whole tree.
+template <typename T>
+__global__ void __launch_bounds__(256) tree_sum_pass(const T* __restrict__ in, int64_t count,
+                                                     double* __restrict__ out, int64_t total_nb,
+                                                     float* __restrict__ mean_out) {
+  __shared__ double warp_sums[8];
+  const int64_t base = (int64_t)blockIdx.x * 2048 + threadIdx.x * 8;
+  double v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = (base + i < count) ? (double)in[base + i] : 0.0;
+  double s = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) s = s + __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const double* w = warp_sums;
+    double tot = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+    out[blockIdx.x] = tot;
+    if (mean_out) *mean_out = __double2float_rn(__ddiv_rn(tot, (double)total_nb));
+  }
+}
+
+// ------------------------------------------------------- double quant: codes
+// One warp per group of 256 constants, 8 per lane.
+__global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict__ absmax, int64_t nb,
+                                                        const float* __restrict__ mean,
+                                                        uint8_t* __restrict__ absmax_q,
+                                                        float* __restrict__ scale2) {
+  const int64_t ng = (nb + 255) / 256;
+  const int lane = threadIdx.x & 31;
+  const float mu = *mean;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < ng; g += warps) {
+    const int64_t b0 = g * 256 + lane * 8;
+    float d[8];
+    float dmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      d[i] = (b0 + i < nb) ? __fsub_rn(absmax[b0 + i], mu) : 0.0f;
+      dmax = fmaxf(dmax, fabsf(d[i]));
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+    const float s2 = __fdiv_rn(dmax, 448.0f);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t e = (s2 != 0.0f) ? f32_to_e4m3(__fdiv_rn(d[i], s2)) : 0u;
+      if (i < 4) lo |= e << (8 * i); else hi |= e << (8 * (i - 4));
+    }
+    if (b0 + 8 <= nb) {
+      *reinterpret_cast<uint2*>(absmax_q + b0) = make_uint2(lo, hi);
+    } else {
+      for (int i = 0; i < 8; ++i)
+        if (b0 + i < nb) absmax_q[b0 + i] = (uint8_t)(((i < 4 ? lo : hi) >> (8 * (i & 3))) & 0xFF);
+    }
+    if (lane == 0) scale2[g] = s2;
+  }
+}
+
+// --------------------------------------------------------------- dequantize
+// bf16 output: one thread per 64-block.  The block's 16 results
+// bf16(fl32(q_j * c)) are built once into a register byte-plane table and
+// looked up with prmt.
+__global__ void __launch_bounds__(256) dequant_bf16_kernel(const uint8_t* __restrict__ codes, WeightConsts wc,
+                                                           int64_t n, __nv_bfloat16* __restrict__ out,
+                                                           NF4Table tab) {
+  const int64_t nb = (n + 63) / 64;
+  const float mu = wc.absmax ? 0.0f : *wc.offset;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nb; b += stride) {
+    const float c = block_const(wc, b, mu);
+    const Lut16 L = make_lut(tab, c);
+    const int64_t e0 = b * 64;
+    if (e0 + 64 <= n) {
+      const uint4* src = reinterpret_cast<const uint4*>(codes + (e0 >> 1));
+      uint4 c0 = __ldcs(src), c1 = __ldcs(src + 1);
+      uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      uint4* dst = reinterpret_cast<uint4*>(out + e0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) __stcs(dst + i, lut_lookup8(L, w[i]));
+    } else {
+      for (int64_t e = e0; e < n; ++e) {
+        uint32_t byte = codes[e >> 1];
+        uint32_t code = (e & 1) ? (byte >> 4) : (byte & 0xF);
+        out[e] = __float2bfloat16_rn(__fmul_rn(tab.q[code], c));
+      }
+    }
+  }
+}
+
+// fp32 output: 8 elements per thread, the 16 levels read from shared memory.
+__global__ void __launch_bounds__(256) dequant_f32_kernel(const uint8_t* __restrict__ codes, WeightConsts wc,
+                                                          int64_t n, float* __restrict__ out, NF4Table tab) {
+  __shared__ float q[16];
+  if (threadIdx.x < 16) q[threadIdx.x] = tab.q[threadIdx.x];
+  __syncthreads();
+  const float mu = wc.absmax ? 0.0f : *wc.offset;
+  const int64_t nchunks = (n + 7) / 8;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < nchunks; k += stride) {
+    const int64_t e0 = k * 8;
+    const float c = block_const(wc, e0 >> 6, mu);
+    if (e0 + 8 <= n) {
+      uint32_t w = __ldcs(reinterpret_cast<const uint32_t*>(codes + (e0 >> 1)));
+      float r[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) r[i] = __fmul_rn(q[(w >> (4 * i)) & 0xF], c);
+      float4* dst = reinterpret_cast<float4*>(out + e0);
+      __stcs(dst, make_float4(r[0], r[1], r[2], r[3]));
+      __stcs(dst + 1, make_float4(r[4], r[5], r[6], r[7]));
+    } else {
+      for (int64_t e = e0; e < n; ++e) {
+        uint32_t byte = codes[e >> 1];
+        uint32_t code = (e & 1) ? (byte >> 4) : (byte & 0xF);
+        out[e] = __fmul_rn(q[code], c);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------- launch
+static int sm_count() {
+  static int count = 0;
+  if (!count) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+    if (count <= 0) count = 148;
+  }
+  return count;
+}
+
+static unsigned grid_for(int64_t work_items, int per_cta, int ctas_per_sm) {
+  int64_t need = (work_items + per_cta - 1) / per_cta;
+  int64_t cap = (int64_t)sm_count() * ctas_per_sm;
+  if (need < 1) need = 1;
+  return (unsigned)(need < cap ? need : cap);
+}
+
+ql_status launch_quantize(const void* x, ql_dtype dt, int64_t n, uint8_t* codes, float* absmax,
+                          cudaStream_t st) {
+  const int64_t nb = (n + 63) / 64;
+  const unsigned grid = grid_for(nb, 32, 8);   // 32 blocks (8 warps x 4) per CTA-iteration
+  TraceScope ts(TK_QUANTIZE, st);
+  if (dt == QL_F32)
+    quantize_kernel<float><<<grid, 256, 0, st>>>((const float*)x, n, codes, absmax, nf4_table());
+  else
+    quantize_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, n, codes, absmax,
+                                                         nf4_table());
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
+size_t dq_workspace_bytes(int64_t nb) {
+  // one double per node of each tree pass above the leaves
+  size_t total = 0;
+  int64_t cnt = nb;
+  do {
+    cnt = (cnt + 2047) / 2048;
+    total += (size_t)cnt * sizeof(double);
+  } while (cnt > 1);
+  return (total + 255) & ~(size_t)255;
+}
+
+ql_status launch_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q, float* scale2,
+                              float* offset, void* ws, cudaStream_t st) {
+  double* buf = reinterpret_cast<double*>(ws);
+  int64_t cnt = (nb + 2047) / 2048;
+  {
+  TraceScope ts(TK_DQ_MEAN, st);
+  tree_sum_pass<float><<<(unsigned)cnt, 256, 0, st>>>(absmax, nb, buf, nb, cnt == 1 ? offset : nullptr);
+  QL_LAUNCH_CHECK();
+  double* prev = buf;
+  while (cnt > 1) {
+    int64_t next = (cnt + 2047) / 2048;
+    double* dst = prev + cnt;
+    tree_sum_pass<double><<<(unsigned)next, 256, 0, st>>>(prev, cnt, dst, nb, next == 1 ? offset : nullptr);
+    QL_LAUNCH_CHECK();
+    prev = dst;
+    cnt = next;
+  }
+  }
+  const int64_t ng = (nb + 255) / 256;
+  TraceScope ts(TK_DQ_ENCODE, st);
+  dq_encode_kernel<<<grid_for(ng, 8, 8), 256, 0, st>>>(absmax, nb, offset, absmax_q, scale2);
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
+ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStream_t st) {
+  const int64_t n = w->rows * w->cols;
+  WeightConsts wc{w->absmax, w->absmax_q, w->scale2, w->offset};
+  TraceScope ts(TK_DEQUANT, st);
+  if (dt == QL_BF16) {
+    const int64_t nb = (n + 63) / 64;
+    dequant_bf16_kernel<<<grid_for(nb, 256, 4), 256, 0, st>>>(w->codes, wc, n, (__nv_bfloat16*)out,
+                                                             nf4_table());
+  } else {
+    dequant_f32_kernel<<<grid_for((n + 7) / 8, 256, 8), 256, 0, st>>>(w->codes, wc, n, (float*)out,
+                                                                     nf4_table());
+  }
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
+}  // namespace ql

@@ -1,0 +1,220 @@
+/*
+ * qlora_nf4.h — C ABI of the B200 (sm_100a) QLoRA NF4 library.
+ *
+ * The library implements the data-parallel hot path of QLoRA:
+ *   - blockwise NF4 quantization of a frozen weight (blocks of 64, a 16-level
+ *     normal-quantile table with an exact zero, two codes per byte);
+ *   - double quantization of the fp32 block constants to 8-bit floats in
+ *     groups of 256;
+ *   - the frozen-4-bit + LoRA linear  Y = X * dequant(W)^T + s * (X A^T) B^T,
+ *     s = alpha / r, forward and backward (dX, dA, dB; W is never written).
+ *
+ * Sources (the web pages this library restates):
+ *   [P2] "QLoRA: Quantize Base Weights to 4-Bit": §2.1 (NF4 quantile formula),
+ *        §2.2 (B_1 = 64 fp32 constants, double quantization to 8-bit floats with
+ *        B_2 = 256), §3 (dequantize to BF16 on chip, BF16 matmul, LoRA branch
+ *        (B @ (A @ x)) * (alpha / r), gradients only into the adapters).
+ *   [P3] "QLoRA — Fine-Tuning a 65B Model on One GPU": "Prerequisite: LoRA's
+ *        low-rank update" (B is d x r, A is r x k), "Quantization in one
+ *        paragraph" (absmax c = max|x|, nearest level of x/c, x_hat = c * q),
+ *        "NF4: sixteen levels shaped like the weights" (8 negative / 8
+ *        non-negative levels, exact 0, endpoints +-1), "Double quantization:
+ *        the constants are not free" (256 constants per group, 8-bit floats, one
+ *        fp32 second-level constant, mean subtracted first), "Where the
+ *        gradients actually go" (chain rule through dequant(W)^T; only A and B
+ *        get gradients).
+ *
+ * Conventions for every call:
+ *   - Pointers named as device pointers must point to memory of the current
+ *     CUDA device and be 16-byte aligned.  The library never allocates or frees
+ *     caller memory; the caller owns every buffer, including the workspace.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     is asynchronous on that stream.
+ *   - Argument errors return QL_ERR_INVALID_ARG / QL_ERR_UNSUPPORTED /
+ *     QL_ERR_WORKSPACE synchronously, before anything is launched.  A failed
+ *     launch returns QL_ERR_CUDA.  Conditions the device detects (a non-finite
+ *     input, a bounded wait that ran out) set bits in a per-device status word,
+ *     which qlora_get_status() reads and clears.
+ *   - Layouts are row-major.  A weight W in R^{N x K} (N = d_out, K = d_in) is
+ *     quantized as the flat array of its N*K elements.  Element i is in 64-block
+ *     i / 64, and that block is in double-quant group (i / 64) / 256.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or shape */
+  QL_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dtype, r > 64, ...) */
+  QL_ERR_WORKSPACE = 3,     /* workspace smaller than qlora_workspace_size() */
+  QL_ERR_CUDA = 4,          /* a CUDA runtime / launch error */
+  QL_ERR_NONFINITE = 5,     /* device: NaN or Inf met in a quantized block */
+  QL_ERR_TIMEOUT = 6        /* device: a bounded wait inside a kernel ran out */
+} ql_status;
+
+typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
+
+/* Block sizes fixed by the method ([P2] §2.2). */
+#define QL_BLOCK 64
+#define QL_DQ_GROUP 256
+#define QL_MAX_RANK 64
+
+/*
+ * An NF4 weight as stored on the device (all device pointers, caller-owned,
+ * only read by the library):
+ *   codes    uint8 [ceil(n/2)], n = rows*cols.  Byte k holds element 2k in its
+ *            low nibble and element 2k+1 in its high nibble.
+ *   absmax   fp32 [nb], nb = ceil(n/64): the block constants c_1.  NULL when
+ *            the double-quantized form below is used.
+ *   absmax_q uint8 [nb] E4M3 codes of (c_1 - mu) / s_2 (double quant).
+ *   scale2   fp32 [ng], ng = ceil(nb/256): second-level constants s_2.
+ *   offset   fp32 [1]: the mean mu subtracted before double quantization.
+ * Reconstructed constant ([P3] "Double quantization"):
+ *   c_hat = fl32(fl32(E4M3(absmax_q[b]) * scale2[b/256]) + offset[0]).
+ */
+typedef struct {
+  const uint8_t* codes;
+  const float* absmax;
+  const uint8_t* absmax_q;
+  const float* scale2;
+  const float* offset;
+  int64_t rows;   /* N */
+  int64_t cols;   /* K */
+} ql_nf4_weight;
+
+/*
+ * nf4_quantize — blockwise absmax NF4 quantization ([P3] "Quantization in one
+ * paragraph"; levels per [P2] §2.1 and [P3] "NF4").
+ *   x       device, n elements of type x_dt (QL_F32 or QL_BF16)
+ *   codes   device out, uint8 [ceil(n/2)] packed as in ql_nf4_weight
+ *   absmax  device out, fp32 [ceil(n/64)]: c_b = max|x| over the block (a
+ *           partial last block uses its valid elements)
+ * Code of element x in block b: with the fp32 decision thresholds
+ * t_j = fl32(m_j * c_b), m_j = fl32(fl32(q_j + q_{j+1}) / 2), the code is
+ * #{j : x > t_j} (ties go to the lower level).  A block with c_b == 0 codes
+ * every element as the zero level (8).  An odd n pads the last high nibble
+ * with 8.  NaN/Inf in a block sets QL_ERR_NONFINITE in the status word
+ * (that block's outputs are then unspecified).  n may exceed 2^32.
+ */
+ql_status nf4_quantize(const void* x, ql_dtype x_dt, int64_t n,
+                       uint8_t* codes, float* absmax, void* stream);
+
+/*
+ * nf4_double_quant — quantize the fp32 block constants ([P2] §2.2, [P3]
+ * "Double quantization: the constants are not free").
+ *   absmax    device, fp32 [nb] (c_1 from nf4_quantize)
+ *   absmax_q  device out, uint8 [nb] E4M3 codes
+ *   scale2    device out, fp32 [ceil(nb/256)]
+ *   offset    device out, fp32 [1]: mu
+ *   ws        device workspace, >= qlora_workspace_size(QL_OP_DOUBLE_QUANT, nb, 0, 0, 0)
+ * mu = fl32(S / nb) with S the float64 sum over a fixed adjacent-pair tree
+ * (zero padded to a power of two).  Per group of 256: d = fl32(c - mu),
+ * s_2 = fl32(max|d| / 448), code = E4M3_rne_satfinite(fl32(d / s_2)); a group
+ * with s_2 == 0 stores code 0x00.
+ */
+ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q,
+                           float* scale2, float* offset, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/*
+ * nf4_dequant — x_hat = bf16(fl32(q_code * c)) ([P3] "Quantization in one
+ * paragraph"; [P2] §3 dequantize to BF16), c = absmax[b] or the double-quant
+ * reconstruction when w->absmax is NULL.  out: device, rows*cols elements of
+ * out_dt (QL_F32 skips the bf16 rounding).
+ */
+ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* stream);
+
+/*
+ * qlora_linear_fwd — Y = X * W_hat^T + s * U * B^T, U = bf16(X * A^T)
+ * ([P3] "Where the gradients actually go", [P2] §3).
+ *   w      NF4 weight, rows = N, cols = K; K % 64 == 0
+ *   X      device bf16 [M, K]
+ *   A      device bf16 [r, K];  B device bf16 [N, r];  1 <= r <= 64, r % 8 == 0
+ *   s      alpha / r
+ *   Y      device out [M, N] of y_dt
+ *   U_out  device out bf16 [M, r] (the tensor the backward reuses) or NULL
+ *   ws     workspace >= qlora_workspace_size(QL_OP_FWD, M, N, K, r)
+ * The main product accumulates in fp32 on the tensor cores from the exact
+ * bf16 W_hat; the adapter term enters the same fp32 accumulator with B scaled
+ * by s and rounded to bf16 (exact when s is a power of two).
+ */
+ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M,
+                           const void* A, const void* B, int r, float s,
+                           void* Y, ql_dtype y_dt, void* U_out,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * qlora_linear_bwd — gradients of <dY, Y> for the forward above
+ * ([P3] "Where the gradients actually go": chain rule through W_hat^T, no
+ * gradient for W; [P2] §3 step 5):
+ *   V  = bf16(dY * B)                 [M, r]
+ *   dX = dY * W_hat + s * V * A       [M, K]   (+= when accumulate_dx != 0)
+ *   dA = s * V^T * X                  [r, K]
+ *   dB = s * dY^T * U                 [N, r]
+ *   X, dY, A, B: device bf16;  U: device bf16 [M, r] from the forward, or NULL
+ *   to recompute it.  dX of dx_dt; dA, dB of grad_dt (overwritten).
+ *   ws >= qlora_workspace_size(QL_OP_BWD, M, N, K, r).
+ */
+ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY, int64_t M,
+                           const void* A, const void* B, int r, float s, const void* U,
+                           void* dX, ql_dtype dx_dt, int accumulate_dx,
+                           void* dA, void* dB, ql_dtype grad_dt,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * SiLU-gated MLP glue between three QLoRA linears (the pages adapt every
+ * linear, [P3] "Seeing it in code": gate_proj, up_proj, down_proj).
+ *   qlora_silu_gate_fwd: h = bf16(silu(g) * u), silu(x) = x * sigmoid(x)
+ *   qlora_silu_gate_bwd: dg = bf16(dh * u * sig(g) * (1 + g (1 - sig(g)))),
+ *                        du = bf16(dh * silu(g))
+ * All device bf16 [n].
+ */
+ql_status qlora_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, void* stream);
+ql_status qlora_silu_gate_bwd(const void* dh, const void* g, const void* u,
+                              void* dg, void* du, int64_t n, void* stream);
+
+/* Workspace query.  op: one of the QL_OP_* values; unused sizes are ignored. */
+#define QL_OP_DOUBLE_QUANT 0   /* M = nb */
+#define QL_OP_FWD 1
+#define QL_OP_BWD 2
+size_t qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r);
+
+/* Bytes needed for n parameters: ceil(n/2) codes + (dq ? nb + 4*ng + 4 : 4*nb)
+ * ([P2] §2.2 and §4: 0.5 + 0.016 bytes per parameter with double quant). */
+int64_t nf4_storage_bytes(int64_t n, int dq);
+
+/* The 16 NF4 levels as fp32, increasing; index 8 is the exact zero
+ * ([P2] §2.1 formula, read per [P3] "NF4": see nf4_quantize).  Host memory. */
+void nf4_codebook(float out[16]);
+
+/* Synchronizes `stream`, then reads and clears the current device's status
+ * word.  Returns QL_OK, QL_ERR_NONFINITE or QL_ERR_TIMEOUT (the first set). */
+ql_status qlora_get_status(void* stream);
+
+/*
+ * Per-kernel device timing, for profiling.  qlora_trace_enable(1) starts
+ * recording a CUDA event pair around every kernel the library launches (on the
+ * caller's stream); qlora_trace_enable(0) stops; either call discards earlier
+ * records.  qlora_trace_read waits for the recorded events, writes for each
+ * kernel kind k < max_kinds the total device milliseconds and launch count,
+ * clears the records and returns the number of kinds written.  Kind names
+ * come from qlora_trace_kind_name.  Host-side only; the caller owns the arrays.
+ */
+void qlora_trace_enable(int on);
+int qlora_trace_read(double* total_ms, int* launches, int max_kinds);
+const char* qlora_trace_kind_name(int kind);
+
+/* Human-readable name of a status code (static string). */
+const char* qlora_status_string(ql_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_NF4_H */
