@@ -40,7 +40,13 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-secondary", action="store_true", help="skip the small-M and codec side measurements")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    return p.parse_args()
+    p.add_argument("--profile", action="store_true",
+                   help="fixed launch sequence for profilers: exactly --warmup then --steps steps, "
+                        "no clock-sampling warm-up, no e2e, secondary or CPU legs")
+    a = p.parse_args()
+    if a.profile:
+        a.no_secondary = a.no_cpu = True
+    return a
 
 
 def peaks():
@@ -324,7 +330,7 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.warmup):
         wl.step(allreduce)
     torch.cuda.synchronize()
-    while time.time() - t_warm < 0.5:          # give the clock sampler samples under load
+    while not args.profile and time.time() - t_warm < 0.5:   # clock samples under load
         wl.step(allreduce)
         torch.cuda.synchronize()
     st = q.qlora_get_status()
@@ -369,7 +375,7 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the public API with pinned host buffers
     e2e = None
-    if rank == 0 or world > 1:
+    if not args.profile:
         hW = torch.empty_like(wl.W, device="cpu").pin_memory().copy_(wl.W)
         hX = torch.empty_like(wl.X, device="cpu").pin_memory().copy_(wl.X)
         hA = torch.empty_like(wl.A, device="cpu").pin_memory().copy_(wl.A)

@@ -1,5 +1,6 @@
 // C ABI of the library: argument checks, workspace carving and the launch
 // sequences of each call.  Argument errors return before anything is launched.
+#include <algorithm>
 #include <cstring>
 
 #include "common.cuh"
@@ -13,17 +14,21 @@ ql_status launch_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q
 ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStream_t st);
 unsigned status_word_codec(cudaStream_t st);
 // gemm.cu
-ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
-                          float s, void* Y, ql_dtype y_dt, cudaStream_t st);
-ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* V, const void* A, int r,
-                          float s, void* dX, ql_dtype dx_dt, int accumulate, cudaStream_t st);
+ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* A, const void* B, int r,
+                          float s, void* U_out, void* Y, ql_dtype y_dt, cudaStream_t st);
+ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* Bt, const void* A, int r,
+                          float s, void* V, void* Vt, int ld_t, void* dX, ql_dtype dx_dt, int accumulate,
+                          cudaStream_t st);
 unsigned status_word_gemm(cudaStream_t st);
-// lora_side.cu
-ql_status launch_proj_xa(const void* X, int64_t M, int K, const void* A, int r, void* U, cudaStream_t st);
-ql_status launch_proj_dyb(const void* dY, int64_t M, int N, const void* B, int r, void* V, cudaStream_t st);
-size_t colacc_partial_bytes(int64_t M, int64_t ncols, int r);
-ql_status launch_colacc(const void* act, int64_t M, int ncols, const void* G, int r, float s, int transpose,
-                        void* out, ql_dtype out_dt, float* partial, cudaStream_t st);
+// lora_tc.cu
+size_t skinny_partial_bytes(int64_t rows, int64_t red, int r);
+ql_status launch_proj_u(const void* X, int64_t M, int K, const void* A, int r, void* U, float* partial,
+                        cudaStream_t st);
+ql_status launch_grad_b(const void* dY, int64_t M, int N, const void* Ut, int64_t ld_ut, int r, float s, void* dB,
+                        ql_dtype dt, float* partial, cudaStream_t st);
+ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t ld_vt, int r, float s, void* dA,
+                        ql_dtype dt, float* partial, cudaStream_t st);
+ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st);
 // mlp.cu
 ql_status launch_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, cudaStream_t st);
 ql_status launch_silu_gate_bwd(const void* dh, const void* g, const void* u, void* dg, void* du, int64_t n,
@@ -60,15 +65,34 @@ ql_status check_gemm_shape(const ql_nf4_weight* w, int64_t M, int r) {
   return QL_OK;
 }
 
-size_t ws_fwd(int64_t M, int r) { return r > 0 ? align256((size_t)M * r * 2) : 0; }
+size_t ws_fwd(int64_t, int) { return 0; }
 
-size_t ws_bwd(int64_t M, int64_t N, int64_t K, int r) {
-  if (r == 0) return 0;
-  size_t part = ql::colacc_partial_bytes(M, N, r);
-  size_t part2 = ql::colacc_partial_bytes(M, K, r);
-  if (part2 > part) part = part2;
-  return 2 * align256((size_t)M * r * 2) + align256(part);
+// Backward workspace, carved in this order (each piece 256-byte aligned):
+//   B^T [r, N], U^T [r, Mp], U [M, r] (recomputed only when not given),
+//   V [M, r], V^T [r, Mp], fp32 split-K partials.   Mp = M rounded up to 8.
+struct BwdWs {
+  size_t bt, ut, u, v, vt, part, total;
+};
+
+BwdWs ws_bwd_layout(int64_t M, int64_t N, int64_t K, int r) {
+  BwdWs w{};
+  if (r == 0) return w;
+  const int64_t Mp = (M + 7) / 8 * 8;
+  size_t off = 0;
+  w.bt = off; off += align256((size_t)r * N * 2);
+  w.ut = off; off += align256((size_t)r * Mp * 2);
+  w.u = off;  off += align256((size_t)M * r * 2);
+  w.v = off;  off += align256((size_t)M * r * 2);
+  w.vt = off; off += align256((size_t)r * Mp * 2);
+  size_t part = ql::skinny_partial_bytes(N, M, r);
+  part = std::max(part, ql::skinny_partial_bytes(K, M, r));
+  part = std::max(part, ql::skinny_partial_bytes(M, K, r));
+  w.part = off; off += align256(part);
+  w.total = off;
+  return w;
 }
+
+size_t ws_bwd(int64_t M, int64_t N, int64_t K, int r) { return ws_bwd_layout(M, N, K, r).total; }
 
 }  // namespace
 
@@ -104,19 +128,7 @@ ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, con
   if (r > 0 && (!aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
   if (U_out && !aligned16(U_out)) return QL_ERR_INVALID_ARG;
   if (M == 0) return QL_OK;
-  void* U = U_out;
-  if (r > 0 && !U) {
-    if (ws_bytes < ws_fwd(M, r)) return QL_ERR_WORKSPACE;
-    if (!aligned16(ws)) return QL_ERR_INVALID_ARG;
-    U = ws;
-  }
-  cudaStream_t cs = as_stream(stream);
-  const int K = (int)w->cols;
-  if (r > 0) {
-    st = ql::launch_proj_xa(X, M, K, A, r, U, cs);
-    if (st != QL_OK) return st;
-  }
-  return ql::launch_gemm_fwd(w, X, M, U, B, r, s, Y, y_dt, cs);
+  return ql::launch_gemm_fwd(w, X, M, A, B, r, s, U_out, Y, y_dt, as_stream(stream));
 }
 
 ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
@@ -141,25 +153,30 @@ ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY
     }
     return QL_OK;
   }
-  if (r == 0) return ql::launch_gemm_bwd(w, dY, M, nullptr, nullptr, 0, s, dX, dx_dt, accumulate_dx, cs);
+  if (r == 0)
+    return ql::launch_gemm_bwd(w, dY, M, nullptr, nullptr, 0, s, nullptr, nullptr, 0, dX, dx_dt, accumulate_dx, cs);
+  const BwdWs L = ws_bwd_layout(M, N, K, r);
   uint8_t* wp = reinterpret_cast<uint8_t*>(ws);
-  void* Uw = wp;
-  wp += align256((size_t)M * r * 2);
-  void* V = wp;
-  wp += align256((size_t)M * r * 2);
-  float* partial = reinterpret_cast<float*>(wp);
+  const int64_t Mp = (M + 7) / 8 * 8;
+  void* Bt = wp + L.bt;
+  void* Ut = wp + L.ut;
+  void* V = wp + L.v;
+  void* Vt = wp + L.vt;
+  float* partial = reinterpret_cast<float*>(wp + L.part);
+  st = ql::launch_transpose(B, N, r, Bt, N, cs);                                         // B^T [r, N]
+  if (st != QL_OK) return st;
   if (!U) {
-    st = ql::launch_proj_xa(X, M, (int)K, A, r, Uw, cs);
+    st = ql::launch_proj_u(X, M, (int)K, A, r, wp + L.u, partial, cs);                  // U = bf16(X A^T)
     if (st != QL_OK) return st;
-    U = Uw;
+    U = wp + L.u;
   }
-  st = ql::launch_proj_dyb(dY, M, (int)N, B, r, V, cs);
+  st = ql::launch_transpose(U, M, r, Ut, Mp, cs);                                       // U^T [r, Mp]
   if (st != QL_OK) return st;
-  st = ql::launch_colacc(dY, M, (int)N, U, r, s, 0, dB, grad_dt, partial, cs);       // dB = s dY^T U
+  st = ql::launch_gemm_bwd(w, dY, M, Bt, A, r, s, V, Vt, (int)Mp, dX, dx_dt, accumulate_dx, cs);  // dX, V, V^T
   if (st != QL_OK) return st;
-  st = ql::launch_gemm_bwd(w, dY, M, V, A, r, s, dX, dx_dt, accumulate_dx, cs);     // dX
+  st = ql::launch_grad_b(dY, M, (int)N, Ut, Mp, r, s, dB, grad_dt, partial, cs);         // dB = s dY^T U
   if (st != QL_OK) return st;
-  return ql::launch_colacc(X, M, (int)K, V, r, s, 1, dA, grad_dt, partial, cs);      // dA = s V^T X
+  return ql::launch_grad_a(X, M, (int)K, Vt, Mp, r, s, dA, grad_dt, partial, cs);        // dA = s V^T X
 }
 
 ql_status qlora_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, void* stream) {

@@ -8,25 +8,35 @@
 // only read.
 //
 // One kernel serves both directions (row-vector convention, tokens are rows):
-//   forward  Y  = X  * W_hat^T + U * (s B)^T     reduction over K (W columns)
-//   backward dX = dY * W_hat   + V * (s A)       reduction over N (W rows)
+//   forward  Y  = X  * W_hat^T + U * (s B)^T,  U = bf16(X  A^T)  (reduction over K)
+//   backward dX = dY * W_hat   + V * (s A),    V = bf16(dY B)    (reduction over N)
 // CTA tile: 128 tokens x 256 outputs, 64 reduction elements per pipeline stage.
-// Warp roles (320 threads):
-//   warp 0      TMA: activation tile (128 x 64 bf16, 128B swizzle) and the
-//               packed NF4 codes of the weight tile into shared memory
+// Two shared-memory rings: a deep one (5-8 stages) for what TMA brings from
+// L2/HBM (activation tile, packed codes, side operand) so the loads run far
+// ahead of the tensor cores, and a 2-stage one for the dequantized weight tile
+// the producers write.
+// The rank-r side product (U or V) is computed in the same main loop from the
+// activation tiles already in shared memory, into a second TMEM accumulator,
+// so the activations are read from HBM once.  After the main loop it is
+// rounded to bf16 and fed back as the A operand of r extra K-steps (the LoRA
+// term) into the main accumulator before the drain.
+//
+// Warp roles (576 threads):
+//   warp 0      TMA: activation tile (128 x 64 bf16), the side operand tile
+//               (A or B^T, rp x 64 bf16) and the packed NF4 codes
 //   warp 1      TMEM allocation; one thread issues tcgen05.mma
-//   warps 2-9   dequant producers: each thread expands one 64-block of codes
-//               through a per-block register lookup table into the swizzled
-//               BF16 operand tile, then (after the main loop) writes the LoRA
-//               operands, and finally drains the TMEM accumulator.
+//   warps 2-17  dequant producers: each pair of threads expands one 64-block
+//               of codes (32 codes each) through a per-block register lookup
+//               table into the swizzled BF16 operand tile; then the LoRA
+//               operands; then the drain of the accumulator.
 // The B operand tile holds W rows as 128-byte rows in both directions: K-major
 // for the forward (rows = output features), MN-major for the backward (rows =
 // the reduction index), so the producers write the same layout either way.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
-#include "trace.cuh"
 #include "sm100.cuh"
+#include "trace.cuh"
 
 namespace ql {
 using namespace sm100;
@@ -36,14 +46,28 @@ namespace gemm {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int STAGES = 3;
-constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-constexpr int B_BYTES = BN * BK * 2;   // 32 KB
+constexpr int A_BYTES = BM * BK * 2;   // 16 KB activation tile
+constexpr int B_BYTES = BN * BK * 2;   // 32 KB dequantized weight tile
 constexpr int C_BYTES = BN * BK / 2;   // 8 KB of packed codes
-constexpr int PRODUCER_WARPS = 8;
+constexpr int B_STAGES = 2;            // dequantized-weight ring
+constexpr int MAX_T_STAGES = 8;        // TMA ring (activation, codes, side tile)
+constexpr int PRODUCER_WARPS = 16;
 constexpr int THREADS = (2 + PRODUCER_WARPS) * 32;
-constexpr int TMEM_COLS = 256;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES + C_BYTES) + 256;
+constexpr int TMEM_COLS = 512;         // main 256 columns + side rp columns
+constexpr int SIDE_COL = 256;
+constexpr int SMEM_LIMIT = 232448;     // opt-in maximum per CTA on sm_100
+constexpr int BAR_BYTES = 512;
+
+// Shared memory: [TMA ring: t_stages x (A | codes | side)] [B ring: 2 x B] [barriers]
+__host__ __device__ constexpr int side_bytes(int rp) { return rp * 128 < 1024 ? 1024 : rp * 128; }
+__host__ __device__ constexpr int t_stage_bytes(int rp) { return A_BYTES + C_BYTES + side_bytes(rp); }
+inline int t_stages_for(int rp) {
+  int n = (SMEM_LIMIT - 1024 - BAR_BYTES - B_STAGES * B_BYTES) / t_stage_bytes(rp);
+  return n > MAX_T_STAGES ? MAX_T_STAGES : n;
+}
+inline size_t smem_bytes_for(int rp) {
+  return 1024 + (size_t)t_stages_for(rp) * t_stage_bytes(rp) + B_STAGES * B_BYTES + BAR_BYTES;
+}
 
 struct Params {
   int M;             // tokens
@@ -51,46 +75,57 @@ struct Params {
   int n_steps;       // main-loop stages (K/64 forward, ceil(N/64) backward)
   int N, K;          // weight shape
   WeightConsts wc;
-  const __nv_bfloat16* lora_a;  // forward U [M, r]; backward V [M, r]
-  const __nv_bfloat16* lora_b;  // forward B [N, r]; backward A [r, K]
-  int r, rp;                    // rank, rank padded to 16
+  int r, rp;         // rank, rank padded to 16 (0 when no adapter)
   float s;
+  const __nv_bfloat16* lora_b;   // forward B [N, r] (scaled by s in-kernel); backward A [r, K]
+  __nv_bfloat16* side_out;       // forward U_out [M, r] (may be NULL); backward V [M, r]
+  __nv_bfloat16* side_out_t;     // backward V^T [r, ld_t] (may be NULL)
+  int ld_t;
   void* out;
   int out_bf16;
   int accumulate;
   NF4Table tab;
   uint32_t wait_limit;
+  int t_stages;
 };
 
 struct Smem {
-  uint8_t* a0;   // STAGES activation tiles, A_BYTES apart
-  uint8_t* b0;   // STAGES weight tiles, B_BYTES apart
-  uint8_t* c0;   // STAGES packed-code tiles, C_BYTES apart
-  __device__ __forceinline__ uint8_t* a(int s) const { return a0 + s * A_BYTES; }
-  __device__ __forceinline__ uint8_t* b(int s) const { return b0 + s * B_BYTES; }
-  __device__ __forceinline__ uint8_t* c(int s) const { return c0 + s * C_BYTES; }
-  uint64_t* full_a;
-  uint64_t* full_c;
-  uint64_t* full_b;
-  uint64_t* empty;
+  uint8_t* base;
+  int ts;        // TMA ring stages
+  int tsb;       // bytes per TMA stage
+  int sideb;     // side tile bytes
+  __device__ __forceinline__ uint8_t* a(int s) const { return base + s * tsb; }
+  __device__ __forceinline__ uint8_t* c(int s) const { return base + s * tsb + A_BYTES; }
+  __device__ __forceinline__ uint8_t* side(int s) const { return base + s * tsb + A_BYTES + C_BYTES; }
+  __device__ __forceinline__ uint8_t* b(int s) const { return base + ts * tsb + s * B_BYTES; }
+  uint64_t* full_a;    // [ts] activation + side tile landed
+  uint64_t* full_c;    // [ts] codes landed
+  uint64_t* empty_t;   // [ts] MMA done with the TMA slot
+  uint64_t* full_b;    // [B_STAGES] producers wrote the weight tile
+  uint64_t* empty_b;   // [B_STAGES] MMA done with the weight tile
+  uint64_t* side_full;
   uint64_t* acc_full;
   uint32_t* tmem_addr;
   int* abort;
 };
 
-__device__ __forceinline__ Smem carve(uint8_t* raw) {
+__device__ __forceinline__ Smem carve(uint8_t* raw, int rp, int ts) {
   Smem s;
   uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-  s.a0 = p; p += STAGES * A_BYTES;
-  s.b0 = p; p += STAGES * B_BYTES;
-  s.c0 = p; p += STAGES * C_BYTES;
+  s.base = p;
+  s.ts = ts;
+  s.tsb = t_stage_bytes(rp);
+  s.sideb = side_bytes(rp);
+  p += ts * s.tsb + B_STAGES * B_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(p);
   s.full_a = bars;
-  s.full_c = bars + STAGES;
-  s.full_b = bars + 2 * STAGES;
-  s.empty = bars + 3 * STAGES;
-  s.acc_full = bars + 4 * STAGES;
-  s.tmem_addr = reinterpret_cast<uint32_t*>(bars + 4 * STAGES + 1);
+  s.full_c = bars + MAX_T_STAGES;
+  s.empty_t = bars + 2 * MAX_T_STAGES;
+  s.full_b = bars + 3 * MAX_T_STAGES;
+  s.empty_b = s.full_b + B_STAGES;
+  s.side_full = s.empty_b + B_STAGES;
+  s.acc_full = s.side_full + 1;
+  s.tmem_addr = reinterpret_cast<uint32_t*>(s.acc_full + 1);
   s.abort = reinterpret_cast<int*>(s.tmem_addr + 1);
   return s;
 }
@@ -106,26 +141,54 @@ __device__ __forceinline__ uint4 scale8(uint4 v, float s) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Raw constant of one 64-block, loaded ahead of use: the fp32 absmax, or the
+// E4M3 code and group scale of the double-quantized form.
+struct RawConst {
+  float v;      // absmax, or the group scale s2
+  uint32_t e;   // E4M3 code (double quant)
+};
+
+__device__ __forceinline__ RawConst load_const(const WeightConsts& wc, int64_t b, bool valid) {
+  RawConst r{0.0f, 0u};
+  if (!valid) return r;
+  if (wc.absmax) {
+    r.v = __ldg(wc.absmax + b);
+  } else {
+    r.e = __ldg(wc.absmax_q + b);
+    r.v = __ldg(wc.scale2 + (b >> 8));
+  }
+  return r;
+}
+
+__device__ __forceinline__ float decode_const(const WeightConsts& wc, RawConst r, float mu) {
+  if (wc.absmax) return r.v;
+  return __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)r.e), r.v), mu);
+}
+
 template <bool BWD>
 __global__ void __launch_bounds__(THREADS, 1)
     qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_codes,
-                      const Params p) {
+                      const __grid_constant__ CUtensorMap tmap_side, const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  Smem sm = carve(smem_raw);
+  Smem sm = carve(smem_raw, p.rp, p.t_stages);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * BM;
   const int j0 = blockIdx.x * BN;   // output-column tile start (W row in fwd, W col in bwd)
-  const int steps = p.n_steps + (p.r > 0 ? 1 : 0);
+  const bool lora = p.r > 0;
   volatile int* abort_flag = sm.abort;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
+    for (int i = 0; i < sm.ts; ++i) {
       mbar_init(&sm.full_a[i], 1);
       mbar_init(&sm.full_c[i], 1);
-      mbar_init(&sm.full_b[i], PRODUCER_WARPS);
-      mbar_init(&sm.empty[i], 1);
+      mbar_init(&sm.empty_t[i], 1);
     }
+    for (int i = 0; i < B_STAGES; ++i) {
+      mbar_init(&sm.full_b[i], PRODUCER_WARPS);
+      mbar_init(&sm.empty_b[i], 1);
+    }
+    mbar_init(sm.side_full, 1);
     mbar_init(sm.acc_full, 1);
     *sm.abort = 0;
     fence_mbar_init();
@@ -133,6 +196,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_act);
     prefetch_tmap(&tmap_codes);
+    if (lora) prefetch_tmap(&tmap_side);
   }
   if (warp == 1) {
     tmem_alloc(sm.tmem_addr, TMEM_COLS);
@@ -146,22 +210,25 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA warp
     if (lane == 0) {
+      const uint32_t a_tx = A_BYTES + (lora ? p.rp * 128 : 0);
+      const int TS = sm.ts;
       int issued = 0;
       for (int i = 0; i < p.n_steps; ++i) {
-        const int s = i % STAGES, use = i / STAGES;
-        if (use > 0 && !mbar_wait(&sm.empty[s], (use - 1) & 1, abort_flag, p.wait_limit)) break;
-        mbar_arrive_expect_tx(&sm.full_a[s], A_BYTES);
-        tma_load_2d(sm.a(s), &tmap_act, &sm.full_a[s], i * BK, m0);
+        const int s = i % TS, use = i / TS;
+        if (use > 0 && !mbar_wait(&sm.empty_t[s], (use - 1) & 1, abort_flag, p.wait_limit)) break;
         mbar_arrive_expect_tx(&sm.full_c[s], C_BYTES);
         if (!BWD)
           tma_load_2d(sm.c(s), &tmap_codes, &sm.full_c[s], i * (BK / 2), j0);
         else
           tma_load_2d(sm.c(s), &tmap_codes, &sm.full_c[s], j0 / 2, i * BK);
+        mbar_arrive_expect_tx(&sm.full_a[s], a_tx);
+        tma_load_2d(sm.a(s), &tmap_act, &sm.full_a[s], i * BK, m0);
+        if (lora) tma_load_2d(sm.side(s), &tmap_side, &sm.full_a[s], i * BK, 0);
         issued = i + 1;
       }
       // before leaving, make sure no copy is still landing in shared memory
-      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
-        const int s = i % STAGES, use = i / STAGES;
+      for (int i = (issued > TS ? issued - TS : 0); i < issued; ++i) {
+        const int s = i % TS, use = i / TS;
         mbar_wait(&sm.full_a[s], use & 1, abort_flag, p.wait_limit);
         mbar_wait(&sm.full_c[s], use & 1, abort_flag, p.wait_limit);
       }
@@ -170,110 +237,189 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC = idesc_bf16(BM, BN, false, BWD);
+      const uint32_t idesc_side = idesc_bf16(BM, lora ? p.rp : 16, false, false);
+      const int TS = sm.ts;
       bool ok = true;
-      for (int i = 0; i < steps && ok; ++i) {
-        const int s = i % STAGES, use = i / STAGES;
-        const bool lora = (i == p.n_steps);
-        if (!lora) ok = mbar_wait(&sm.full_a[s], use & 1, abort_flag, p.wait_limit);
-        if (ok) ok = mbar_wait(&sm.full_b[s], use & 1, abort_flag, p.wait_limit);
+      for (int i = 0; i < p.n_steps && ok; ++i) {
+        const int s = i % TS, use = i / TS;
+        const int sb = i % B_STAGES, useb = i / B_STAGES;
+        ok = mbar_wait(&sm.full_a[s], use & 1, abort_flag, p.wait_limit) &&
+             mbar_wait(&sm.full_b[sb], useb & 1, abort_flag, p.wait_limit);
         if (!ok) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sm.a(s));
-        const uint32_t b_addr = smem_u32(sm.b(s));
-        const int kk_n = lora ? p.rp / 16 : BK / 16;
-        for (int kk = 0; kk < kk_n; ++kk) {
+        const uint32_t b_addr = smem_u32(sm.b(sb));
+        const uint32_t s_addr = smem_u32(sm.side(s));
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
           const uint64_t bd = BWD ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
                                   : sdesc_sw128(b_addr + kk * 32, 16, 1024);
-          mma_bf16(tmem, ad, bd, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          mma_bf16(tmem, ad, bd, IDESC, acc);
+          if (lora) mma_bf16(tmem + SIDE_COL, ad, sdesc_sw128(s_addr + kk * 32, 16, 1024), idesc_side, acc);
         }
-        mma_commit(&sm.empty[s]);
+        mma_commit(&sm.empty_t[s]);
+        mma_commit(&sm.empty_b[sb]);
+      }
+      if (ok && lora) {
+        mma_commit(sm.side_full);
+        // LoRA K-steps: A = bf16 side product, B = scaled adapter, into the main accumulator
+        const int i = p.n_steps;
+        const int s = i % TS, sb = i % B_STAGES, useb = i / B_STAGES;
+        ok = mbar_wait(&sm.full_b[sb], useb & 1, abort_flag, p.wait_limit);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sm.a(s));
+          const uint32_t b_addr = smem_u32(sm.b(sb));
+          for (int kk = 0; kk < p.rp / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = BWD ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                    : sdesc_sw128(b_addr + kk * 32, 16, 1024);
+            mma_bf16(tmem, ad, bd, IDESC, 1u);
+          }
+        }
       }
       mma_commit(sm.acc_full);
     }
   } else {
     // ------------------------------------------------------ dequant producers
-    const int pt = threadIdx.x - 64;   // 0..255
+    // Each producer warp covers 16 weight rows: lanes 0-7 / 8-15 take the two
+    // halves of rows 0-7, lanes 16-23 / 24-31 those of rows 8-15, so every
+    // quarter-warp touches 8 different rows and the swizzled shared-memory
+    // accesses below are free of bank conflicts.
+    const int wp = warp - 2;                                   // 0..15
+    const int half = (lane >> 3) & 1;                          // which 32 codes of the 64-block
+    const int row_local = (lane & 7) + 8 * (lane >> 4);        // 0..15
     const int kblocks = p.K / 64;      // 64-blocks per weight row
     const float mu = p.wc.absmax ? 0.0f : *p.wc.offset;
     // which weight row / 64-block column this thread expands in every stage
     int row_in_tile, col_chunk;
-    if (!BWD) { row_in_tile = pt; col_chunk = 0; }
-    else { row_in_tile = pt & 63; col_chunk = pt >> 6; }
-    bool ok = true;
-    for (int i = 0; i < p.n_steps && ok; ++i) {
-      const int s = i % STAGES, use = i / STAGES;
-      int wrow, kb;   // weight row, 64-block column
+    if (!BWD) { row_in_tile = 16 * wp + row_local; col_chunk = 0; }
+    else { row_in_tile = 16 * (wp & 3) + row_local; col_chunk = wp >> 2; }
+    // byte offset of this thread's 16-byte code chunk in the swizzled code tile
+    uint32_t coff;
+    if (!BWD) {   // 32-byte rows, 32B swizzle: chunk ^= bit 2 of the row
+      coff = row_in_tile * 32 + ((half ^ ((row_in_tile >> 2) & 1)) << 4);
+    } else {      // 128-byte rows, 128B swizzle: chunk ^= row mod 8
+      coff = row_in_tile * 128 + (((2 * col_chunk + half) ^ (row_in_tile & 7)) << 4);
+    }
+    auto step_row = [&](int i, int& wrow, int& kb) {
       if (!BWD) { wrow = j0 + row_in_tile; kb = i; }
       else { wrow = i * BK + row_in_tile; kb = j0 / 64 + col_chunk; }
-      const bool valid = wrow < p.N && kb < kblocks;
-      float c = 0.0f;
-      if (valid) c = block_const(p.wc, (int64_t)wrow * kblocks + kb, mu);
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.full_c[s], use & 1, abort_flag, p.wait_limit));
+    };
+    int wrow, kb;
+    step_row(0, wrow, kb);
+    bool valid = wrow < p.N && kb < kblocks;
+    RawConst next = load_const(p.wc, (int64_t)wrow * kblocks + kb, valid);
+    bool ok = true;
+    const int TS = sm.ts;
+    for (int i = 0; i < p.n_steps && ok; ++i) {
+      const int s = i % TS, use = i / TS;
+      const int sb = i % B_STAGES, useb = i / B_STAGES;
+      const RawConst cur = next;
+      const bool cur_valid = valid;
+      if (i + 1 < p.n_steps) {   // constants of the next stage, one stage ahead
+        step_row(i + 1, wrow, kb);
+        valid = wrow < p.N && kb < kblocks;
+        next = load_const(p.wc, (int64_t)wrow * kblocks + kb, valid);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.full_c[s], use & 1, abort_flag, p.wait_limit) &&
+                                       (useb == 0 || mbar_wait(&sm.empty_b[sb], (useb - 1) & 1, abort_flag,
+                                                               p.wait_limit)));
       if (!ok) break;
-      uint8_t* bt = sm.b(s);
-      if (valid) {
-        const uint8_t* csrc = BWD ? sm.c(s) + row_in_tile * 128 + col_chunk * 32 : sm.c(s) + row_in_tile * 32;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(csrc);
-        const uint4 c1 = *reinterpret_cast<const uint4*>(csrc + 16);
-        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const Lut16 L = make_lut(p.tab, c);
-        uint8_t* base = bt + (BWD ? col_chunk * 8192 : 0);
+      uint8_t* base = sm.b(sb) + (BWD ? col_chunk * 8192 : 0);
+      if (cur_valid) {
+        const uint4 c0 = *reinterpret_cast<const uint4*>(sm.c(s) + coff);
+        const uint32_t w[4] = {c0.x, c0.y, c0.z, c0.w};
+        const Lut16 L = make_lut(p.tab, decode_const(p.wc, cur, mu));
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint4*>(base + sw128_offset(row_in_tile, j)) = lut_lookup8(L, w[j]);
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(base + sw128_offset(row_in_tile, 4 * half + j)) = lut_lookup8(L, w[j]);
       } else {
-        uint8_t* base = bt + (BWD ? col_chunk * 8192 : 0);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(base + sw128_offset(row_in_tile, j)) = zero4();
+        for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(base + sw128_offset(row_in_tile, 4 * half + j)) = zero4();
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.full_b[s]);
+      if (lane == 0) mbar_arrive(&sm.full_b[sb]);
     }
-    // LoRA operands into the stage after the last main step
-    if (ok && p.r > 0) {
+    // LoRA operands into the slots after the last main step
+    if (ok && lora) {
       const int i = p.n_steps;
-      const int s = i % STAGES, use = i / STAGES;
-      if (use > 0) ok = __all_sync(0xffffffffu, mbar_wait(&sm.empty[s], (use - 1) & 1, abort_flag, p.wait_limit));
+      const int s = i % TS, use = i / TS;
+      const int sb = i % B_STAGES, useb = i / B_STAGES;
+      if (use > 0) ok = __all_sync(0xffffffffu, mbar_wait(&sm.empty_t[s], (use - 1) & 1, abort_flag, p.wait_limit));
+      if (ok && useb > 0)
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.empty_b[sb], (useb - 1) & 1, abort_flag, p.wait_limit));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(sm.side_full, 0, abort_flag, p.wait_limit));
       if (ok) {
-        // A operand: U or V tile [128 tokens x rp], K-major
-        {
-          const int row = pt >> 1, half = pt & 1;
+        tc_fence_after();
+        if (warp < 6) {
+          // A operand: the side product (U or V), rounded to bf16, from TMEM
+          const int quad = warp & 3;
+          const int row = quad * 32 + lane;
           const int m = m0 + row;
+          const bool write_side = p.side_out && blockIdx.x == 0 && m < p.M;
+          const bool write_side_t = p.side_out_t && blockIdx.x == 0 && m < p.M;
+          for (int c16 = 0; c16 < p.rp / 16; ++c16) {
+            uint32_t v[16];
+            tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(SIDE_COL + c16 * 16), v);
+            tmem_ld_wait();
+            uint32_t pk[8];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int chunk = half * 4 + q;
-            const int e = chunk * 8;
-            uint4 v = zero4();
-            if (m < p.M && e < p.r) v = *reinterpret_cast<const uint4*>(p.lora_a + (size_t)m * p.r + e);
-            *reinterpret_cast<uint4*>(sm.a(s) + sw128_offset(row, chunk)) = v;
-          }
-        }
-        if (!BWD) {
-          // B operand: (s B)[n, 0..rp) for the 256 output features, K-major
-          const int n = j0 + pt;
+            for (int q = 0; q < 8; ++q) pk[q] = pack_bf16x2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
+            *reinterpret_cast<uint4*>(sm.a(s) + sw128_offset(row, 2 * c16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(sm.a(s) + sw128_offset(row, 2 * c16 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            if (write_side) {
 #pragma unroll
-          for (int chunk = 0; chunk < 8; ++chunk) {
-            const int e = chunk * 8;
-            uint4 v = zero4();
-            if (n < p.N && e < p.r) v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)n * p.r + e), p.s);
-            *reinterpret_cast<uint4*>(sm.b(s) + sw128_offset(pt, chunk)) = v;
+              for (int q = 0; q < 8; ++q) {
+                const int j = c16 * 16 + 2 * q;
+                if (j < p.r) *reinterpret_cast<uint32_t*>(p.side_out + (size_t)m * p.r + j) = pk[q];
+              }
+            }
+            if (write_side_t) {
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const int j = c16 * 16 + q;
+                if (j < p.r) {
+                  const uint32_t h = (q & 1) ? (pk[q >> 1] >> 16) : (pk[q >> 1] & 0xFFFFu);
+                  reinterpret_cast<uint16_t*>(p.side_out_t)[(size_t)j * p.ld_t + m] = (uint16_t)h;
+                }
+              }
+            }
           }
         } else {
-          // B operand: (s A)[0..rp, k] for the 256 output columns, MN-major
-          for (int idx = pt; idx < p.rp * 32; idx += 256) {
-            const int jr = idx >> 5, rem = idx & 31;
-            const int cc = rem >> 3, piece = rem & 7;
-            const int k = j0 + cc * 64 + piece * 8;
-            uint4 v = zero4();
-            if (jr < p.r && k < p.K) v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)jr * p.K + k), p.s);
-            *reinterpret_cast<uint4*>(sm.b(s) + cc * 8192 + sw128_offset(jr, piece)) = v;
+          const int t = threadIdx.x - 6 * 32;   // 0..383
+          constexpr int NT = (PRODUCER_WARPS - 4) * 32;
+          if (!BWD) {
+            // B operand: (s B)[n, 0..rp) for the 256 output features, K-major
+            for (int rr = t; rr < BN; rr += NT) {
+              const int n = j0 + rr;
+              for (int chunk = 0; chunk < p.rp / 8; ++chunk) {
+                const int e = chunk * 8;
+                uint4 v = zero4();
+                if (n < p.N && e < p.r)
+                  v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)n * p.r + e), p.s);
+                *reinterpret_cast<uint4*>(sm.b(sb) + sw128_offset(rr, chunk)) = v;
+              }
+            }
+          } else {
+            // B operand: (s A)[0..rp, k] for the 256 output columns, MN-major
+            for (int idx = t; idx < p.rp * 32; idx += NT) {
+              const int jr = idx >> 5, rem = idx & 31;
+              const int cc = rem >> 3, piece = rem & 7;
+              const int k = j0 + cc * 64 + piece * 8;
+              uint4 v = zero4();
+              if (jr < p.r && k < p.K)
+                v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)jr * p.K + k), p.s);
+              *reinterpret_cast<uint4*>(sm.b(sb) + cc * 8192 + sw128_offset(jr, piece)) = v;
+            }
           }
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.full_b[s]);
+        if (lane == 0) mbar_arrive(&sm.full_b[sb]);
       }
     }
     // ------------------------------------------------------------ epilogue
@@ -281,10 +427,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (acc_ok) {
       tc_fence_after();
       const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
-      const int col_half = (warp - 2) >> 2;      // columns 0-127 or 128-255
+      const int col_q = (warp - 2) >> 2;         // columns 64*col_q .. +63
       const int row = m0 + quad * 32 + lane;
-      for (int cc = 0; cc < 8; ++cc) {
-        const int col = col_half * 128 + cc * 16;
+      for (int cc = 0; cc < 4; ++cc) {
+        const int col = col_q * 64 + cc * 16;
         uint32_t r[16];
         tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)col, r);
         tmem_ld_wait();
@@ -355,13 +501,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D tensor map over a row-major [rows, cols] array.
-static bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
-                     uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+// 2-D tensor map over a row-major [rows, cols] array with row pitch `ld`
+// elements (ld >= cols; ld * elem_bytes must be a multiple of 16).
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
+                 uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+  cuuint64_t strides[1] = {ld * (uint64_t)elem_bytes};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
@@ -370,30 +517,40 @@ static bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, c
 }
 
 template <bool BWD>
-static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64_t M, const void* lora_a,
-                                  const void* lora_b, int r, float s, void* out, ql_dtype out_dt, int accumulate,
-                                  cudaStream_t st) {
+static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64_t M, const void* side_src,
+                                  const void* lora_b, int r, float s, void* side_out, void* side_out_t, int ld_t,
+                                  void* out, ql_dtype out_dt, int accumulate, cudaStream_t st) {
   using namespace gemm;
   static bool attr_set = false;
   if (!attr_set) {
     QL_CUDA_TRY(cudaFuncSetAttribute(qlora_gemm_kernel<BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)SMEM_BYTES));
+                                     SMEM_LIMIT));
     attr_set = true;
   }
   const int N = (int)w->rows, K = (int)w->cols;
-  CUtensorMap map_act, map_codes;
+  const int rp = r > 0 ? (r + 15) / 16 * 16 : 0;
+  const size_t smem = smem_bytes_for(rp);
+  CUtensorMap map_act, map_codes, map_side;
   const int red = BWD ? N : K;   // reduction length = activation row length
-  if (!make_map(&map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, (uint64_t)red, (uint64_t)M, BK, BM,
-                CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, (uint64_t)red, (uint64_t)M, (uint64_t)red, BK,
+                   BM, CU_TENSOR_MAP_SWIZZLE_128B))
     return QL_ERR_CUDA;
   if (!BWD) {
-    if (!make_map(&map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, (uint64_t)K / 2, (uint64_t)N, BK / 2, BN,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_map_2d(&map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, (uint64_t)K / 2, (uint64_t)N,
+                     (uint64_t)K / 2, BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_32B))
       return QL_ERR_CUDA;
   } else {
-    if (!make_map(&map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, (uint64_t)K / 2, (uint64_t)N, BN / 2, BK,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_map_2d(&map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, (uint64_t)K / 2, (uint64_t)N,
+                     (uint64_t)K / 2, BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_128B))
       return QL_ERR_CUDA;
+  }
+  if (r > 0) {
+    // side operand [r, red] bf16: A (forward) or B^T (backward); rows r..rp-1 read as zeros
+    if (!make_map_2d(&map_side, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, side_src, (uint64_t)red, (uint64_t)r,
+                     (uint64_t)red, BK, (uint32_t)rp, CU_TENSOR_MAP_SWIZZLE_128B))
+      return QL_ERR_CUDA;
+  } else {
+    map_side = map_act;   // unused
   }
   Params p;
   p.M = (int)M;
@@ -402,31 +559,39 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
   p.N = N;
   p.K = K;
   p.wc = WeightConsts{w->absmax, w->absmax_q, w->scale2, w->offset};
-  p.lora_a = (const __nv_bfloat16*)lora_a;
-  p.lora_b = (const __nv_bfloat16*)lora_b;
   p.r = r;
-  p.rp = (r + 15) / 16 * 16;
+  p.rp = rp;
   p.s = s;
+  p.lora_b = (const __nv_bfloat16*)lora_b;
+  p.side_out = (__nv_bfloat16*)side_out;
+  p.side_out_t = (__nv_bfloat16*)side_out_t;
+  p.ld_t = ld_t;
   p.out = out;
   p.out_bf16 = out_dt == QL_BF16;
   p.accumulate = accumulate;
   p.tab = nf4_table();
   p.wait_limit = 1u << 22;
+  p.t_stages = t_stages_for(rp);
   dim3 grid((unsigned)((p.n_out + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
   TraceScope ts(BWD ? TK_GEMM_BWD : TK_GEMM_FWD, st);
-  qlora_gemm_kernel<BWD><<<grid, THREADS, SMEM_BYTES, st>>>(map_act, map_codes, p);
+  qlora_gemm_kernel<BWD><<<grid, THREADS, smem, st>>>(map_act, map_codes, map_side, p);
   QL_LAUNCH_CHECK();
   return QL_OK;
 }
 
-ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
-                          float s, void* Y, ql_dtype y_dt, cudaStream_t st) {
-  return launch_gemm_impl<false>(w, X, M, U, B, r, s, Y, y_dt, 0, st);
+// Y = X W_hat^T + U (s B)^T with U = bf16(X A^T) computed in the same kernel;
+// U is also written to U_out when given.
+ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* A, const void* B, int r,
+                          float s, void* U_out, void* Y, ql_dtype y_dt, cudaStream_t st) {
+  return launch_gemm_impl<false>(w, X, M, A, B, r, s, U_out, nullptr, 0, Y, y_dt, 0, st);
 }
 
-ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* V, const void* A, int r,
-                          float s, void* dX, ql_dtype dx_dt, int accumulate, cudaStream_t st) {
-  return launch_gemm_impl<true>(w, dY, M, V, A, r, s, dX, dx_dt, accumulate, st);
+// dX (+)= dY W_hat + V (s A) with V = bf16(dY B) computed in the same kernel
+// from B^T [r, N]; V [M, r] and V^T [r, ld_t] are written for the gradients.
+ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* Bt, const void* A, int r,
+                          float s, void* V, void* Vt, int ld_t, void* dX, ql_dtype dx_dt, int accumulate,
+                          cudaStream_t st) {
+  return launch_gemm_impl<true>(w, dY, M, Bt, A, r, s, V, Vt, ld_t, dX, dx_dt, accumulate, st);
 }
 
 }  // namespace ql

@@ -1,0 +1,297 @@
+// Rank-r adapter gradients on the tensor cores ("QLoRA — Fine-Tuning a 65B
+// Model on One GPU", "Where the gradients actually go": only A and B receive
+// gradients; "Prerequisite: LoRA's low-rank update": B is d x r, A is r x k):
+//   dB = s dY^T U   [N, r]     dA = s V^T X   [r, K]
+// and, when the caller did not keep it from the forward, U = bf16(X A^T).
+//
+// All three are skinny products C[rows x r] = Z_op[rows x red] * G[red x r]
+// with r <= 64: tcgen05.mma with M = 128 output rows and N = r (padded to 16),
+// the long reduction split over CTAs (split-K), fp32 partials in the caller's
+// workspace, then a reduction over the splits in fixed order (deterministic).
+//   dB: Z_op = dY^T (MN-major view of dY [M, N]), G^T = U^T [r, M]
+//   dA: Z_op = X^T  (MN-major view of X  [M, K]), G^T = V^T [r, M]
+//   U:  Z_op = X    (K-major),                     G^T = A   [r, K]
+// They stream one activation matrix once, so they are bound by its HBM read.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "sm100.cuh"
+#include "trace.cuh"
+
+namespace ql {
+using namespace sm100;
+
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
+                 uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+
+namespace skinny {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+constexpr int B_BYTES = 64 * BK * 2;   // 8 KB (r <= 64)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 6 * 32;        // TMA, MMA, 4 drain warps
+constexpr int TMEM_COLS = 64;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+
+struct Params {
+  int rows;             // output rows (M of the MMA)
+  int rp;               // r padded to 16
+  int steps_total;      // ceil(red / 64)
+  int steps_per_split;
+  float* partial;       // [splits][rows][rp]
+  uint32_t wait_limit;
+};
+
+template <bool A_MN>
+__global__ void __launch_bounds__(THREADS, 1)
+    skinny_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                  const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint32_t* tmem_addr = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<int*>(tmem_addr + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * BM;
+  const int step0 = blockIdx.y * p.steps_per_split;
+  const int nsteps = min(p.steps_per_split, p.steps_total - step0);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_addr, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_addr;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmap_a);
+      prefetch_tmap(&tmap_b);
+      const uint32_t tx = A_BYTES + p.rp * 128;
+      int issued = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % STAGES, use = i / STAGES;
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, abort_flag, p.wait_limit)) break;
+        const int k0 = (step0 + i) * BK;
+        uint8_t* a = base + s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[s], tx);
+        if (!A_MN) {
+          tma_load_2d(a, &tmap_a, &full[s], k0, row0);
+        } else {
+          tma_load_2d(a, &tmap_a, &full[s], row0, k0);
+          tma_load_2d(a + 8192, &tmap_a, &full[s], row0 + 64, k0);
+        }
+        tma_load_2d(a + A_BYTES, &tmap_b, &full[s], k0, 0);
+        issued = i + 1;
+      }
+      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+        mbar_wait(&full[i % STAGES], (i / STAGES) & 1, abort_flag, p.wait_limit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(BM, p.rp, A_MN, false);
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % STAGES, use = i / STAGES;
+        if (!mbar_wait(&full[s], use & 1, abort_flag, p.wait_limit)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(base + s * STAGE_BYTES);
+        const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = A_MN ? sdesc_sw128(a_addr + kk * 2048, 8192, 1024) : sdesc_sw128(a_addr + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
+          mma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(acc_full);
+    }
+  } else {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.wait_limit) && !*abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const int quad = warp & 3;
+      const int row = row0 + quad * 32 + lane;
+      for (int c16 = 0; c16 < p.rp / 16; ++c16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(c16 * 16), v);
+        tmem_ld_wait();
+        if (row < p.rows) {
+          float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)blockIdx.y * p.rows + row) * p.rp + c16 * 16);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                                 __uint_as_float(v[4 * q + 3]));
+        }
+      }
+    }
+  }
+  if (warp == 1 && lane == 0 && *abort_flag) mbar_wait(acc_full, 0, abort_flag, p.wait_limit);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// out = scale * sum over splits of partial, in split order.
+// transpose = 0: out [rows, r] (row-major); 1: out [r, rows].
+__global__ void __launch_bounds__(256) reduce_kernel(const float* __restrict__ partial, int splits, int rows, int rp,
+                                                     int r, float scale, int transpose, int out_bf16,
+                                                     void* __restrict__ out) {
+  const int64_t total = (int64_t)rows * r;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    int64_t row, j;
+    if (transpose) { j = idx / rows; row = idx % rows; }   // coalesced writes along rows
+    else { row = idx / r; j = idx % r; }
+    float acc = 0.0f;
+    for (int s = 0; s < splits; ++s) acc = __fadd_rn(acc, partial[((int64_t)s * rows + row) * rp + j]);
+    const float v = __fmul_rn(scale, acc);
+    const int64_t o = transpose ? j * rows + row : row * r + j;
+    if (out_bf16) reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v);
+    else reinterpret_cast<float*>(out)[o] = v;
+  }
+}
+
+// dst [cols, ld_dst] = src [rows, cols]^T (bf16, cols = r <= 64).
+__global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ src, int rows, int cols,
+                                                        uint16_t* __restrict__ dst, int ld_dst) {
+  const int64_t total = (int64_t)rows * cols;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t j = idx / rows, row = idx % rows;
+    dst[j * ld_dst + row] = src[row * cols + j];
+  }
+}
+
+}  // namespace skinny
+
+static int sm_count_tc() {
+  static int count = 0;
+  if (!count) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+    if (count <= 0) count = 148;
+  }
+  return count;
+}
+
+static void split_plan(int rows, int64_t red, int& splits, int& per) {
+  const int tiles = (rows + skinny::BM - 1) / skinny::BM;
+  const int steps = (int)((red + skinny::BK - 1) / skinny::BK);
+  int want = (2 * sm_count_tc() + tiles - 1) / tiles;
+  want = std::max(1, std::min(want, steps));
+  per = (steps + want - 1) / want;
+  splits = (steps + per - 1) / per;
+}
+
+size_t skinny_partial_bytes(int64_t rows, int64_t red, int r) {
+  int splits, per;
+  split_plan((int)rows, red, splits, per);
+  const int rp = (r + 15) / 16 * 16;
+  return (size_t)splits * rows * rp * sizeof(float);
+}
+
+// C = scale * Z_op G, see the file comment.  a_mn: Z_op is the transpose of a
+// row-major [red, rows] array z (ld = rows); else Z_op = z, [rows, red].
+// gt: G^T, row-major [r, red] with row pitch ld_gt.
+static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, const void* gt, int r, int64_t ld_gt,
+                               float scale, int transpose, void* out, ql_dtype out_dt, float* partial, int kind,
+                               cudaStream_t st) {
+  using namespace skinny;
+  static bool attr[2] = {false, false};
+  if (!attr[a_mn]) {
+    if (a_mn) QL_CUDA_TRY(cudaFuncSetAttribute(skinny_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
+    else QL_CUDA_TRY(cudaFuncSetAttribute(skinny_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
+    attr[a_mn] = true;
+  }
+  const int rp = (r + 15) / 16 * 16;
+  CUtensorMap ma, mb;
+  if (a_mn) {
+    if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, z, (uint64_t)rows, (uint64_t)red, (uint64_t)rows, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return QL_ERR_CUDA;
+  } else {
+    if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, z, (uint64_t)red, (uint64_t)rows, (uint64_t)red, BK, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return QL_ERR_CUDA;
+  }
+  if (!make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, gt, (uint64_t)red, (uint64_t)r, (uint64_t)ld_gt, BK,
+                   (uint32_t)rp, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QL_ERR_CUDA;
+  int splits, per;
+  split_plan(rows, red, splits, per);
+  Params p;
+  p.rows = rows;
+  p.rp = rp;
+  p.steps_total = (int)((red + BK - 1) / BK);
+  p.steps_per_split = per;
+  p.partial = partial;
+  p.wait_limit = 1u << 22;
+  dim3 grid((unsigned)((rows + BM - 1) / BM), (unsigned)splits);
+  {
+    TraceScope ts(kind, st);
+    if (a_mn) skinny_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, p);
+    else skinny_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, p);
+  }
+  QL_LAUNCH_CHECK();
+  const int64_t total = (int64_t)rows * r;
+  const unsigned rg = (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count_tc() * 8);
+  {
+    TraceScope ts(TK_COLACC_REDUCE, st);
+    reduce_kernel<<<rg, 256, 0, st>>>(partial, splits, rows, rp, r, scale, transpose, out_dt == QL_BF16, out);
+  }
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
+// U = bf16(X A^T), X [M, K], A [r, K]
+ql_status launch_proj_u(const void* X, int64_t M, int K, const void* A, int r, void* U, float* partial,
+                        cudaStream_t st) {
+  return skinny_launch(false, X, (int)M, K, A, r, K, 1.0f, 0, U, QL_BF16, partial, TK_PROJ, st);
+}
+
+// dB = s dY^T U: dY [M, N], U^T [r, ld_ut]
+ql_status launch_grad_b(const void* dY, int64_t M, int N, const void* Ut, int64_t ld_ut, int r, float s, void* dB,
+                        ql_dtype dt, float* partial, cudaStream_t st) {
+  return skinny_launch(true, dY, N, M, Ut, r, ld_ut, s, 0, dB, dt, partial, TK_COLACC, st);
+}
+
+// dA = s V^T X: X [M, K], V^T [r, ld_vt]; written as [r, K]
+ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t ld_vt, int r, float s, void* dA,
+                        ql_dtype dt, float* partial, cudaStream_t st) {
+  return skinny_launch(true, X, K, M, Vt, r, ld_vt, s, 1, dA, dt, partial, TK_COLACC, st);
+}
+
+// dst [cols, ld_dst] = src [rows, cols]^T, bf16
+ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st) {
+  const int64_t total = rows * cols;
+  const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, (int64_t)sm_count_tc() * 8));
+  TraceScope ts(TK_TRANSPOSE, st);
+  skinny::transpose_kernel<<<g, 256, 0, st>>>((const uint16_t*)src, (int)rows, cols, (uint16_t*)dst, (int)ld_dst);
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
+}  // namespace ql

@@ -18,9 +18,9 @@ std::atomic<int> g_on{0};
 std::mutex g_mu;
 std::vector<Rec> g_recs;
 std::vector<cudaEvent_t> g_free;
-const char* const kNames[TK_COUNT] = {"nf4_quantize",  "dq_tree_sum", "dq_encode",     "nf4_dequant",
-                                      "qlora_gemm_fwd", "qlora_gemm_bwd", "lora_rowproj", "lora_colacc",
-                                      "lora_colacc_reduce", "silu_gate", "smallm_splitk"};
+const char* const kNames[TK_COUNT] = {"nf4_quantize",   "dq_tree_sum",    "dq_encode",       "nf4_dequant",
+                                      "qlora_gemm_fwd", "qlora_gemm_bwd", "lora_u_recompute", "lora_grad",
+                                      "lora_grad_reduce", "silu_gate",    "smallm_splitk",   "lora_transpose"};
 }  // namespace
 
 const char* trace_name(int kind) { return (kind >= 0 && kind < TK_COUNT) ? kNames[kind] : "unknown"; }

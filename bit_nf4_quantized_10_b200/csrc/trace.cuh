@@ -21,6 +21,7 @@ enum TraceKind : int {
   TK_COLACC_REDUCE,
   TK_SILU,
   TK_SMALLM,
+  TK_TRANSPOSE,
   TK_COUNT
 };
 

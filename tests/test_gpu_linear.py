@@ -90,7 +90,7 @@ def test_fwd_bwd_fp32_outputs(q, N, K, M, r, s, dq):
     assert_fp_close(np64(got["Y"]), ref["Y"], "Y")
     assert_fp_close(np64(got["dX"]), ref["dX"], "dX")
     if r:
-        assert_bf16_within_ulp(got["U"][:, :r], ref["U"], "U")
+        assert_bf16_within_ulp(got["U"][:, :r], ref["U"], "U", abs_rms=1e-4)
         assert_fp_close(np64(got["dA"][:r]), ref["dA"], "dA")
         assert_fp_close(np64(got["dB"][:, :r]), ref["dB"], "dB")
 
@@ -122,4 +122,4 @@ def test_projection_workload_full(q):
         assert_fp_close(np64(got[k]), ref[k], k)
     assert_fp_close(np64(got["dA"]), ref["dA"], "dA")
     assert_fp_close(np64(got["dB"]), ref["dB"], "dB")
-    assert_bf16_within_ulp(got["U"], ref["U"], "U")
+    assert_bf16_within_ulp(got["U"], ref["U"], "U", abs_rms=1e-4)
