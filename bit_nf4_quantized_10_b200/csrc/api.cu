@@ -14,16 +14,15 @@ ql_status launch_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q
 ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStream_t st);
 unsigned status_word_codec(cudaStream_t st);
 // gemm.cu
-ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* A, const void* B, int r,
-                          float s, void* U_out, void* Y, ql_dtype y_dt, cudaStream_t st);
-ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* Bt, const void* A, int r,
-                          float s, void* V, void* Vt, int ld_t, void* dX, ql_dtype dx_dt, int accumulate,
-                          cudaStream_t st);
+ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
+                          float s, void* Y, ql_dtype y_dt, cudaStream_t st);
+ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* V, const void* A, int r,
+                          float s, void* dX, ql_dtype dx_dt, int accumulate, cudaStream_t st);
 unsigned status_word_gemm(cudaStream_t st);
 // lora_tc.cu
 size_t skinny_partial_bytes(int64_t rows, int64_t red, int r);
-ql_status launch_proj_u(const void* X, int64_t M, int K, const void* A, int r, void* U, float* partial,
-                        cudaStream_t st);
+ql_status launch_proj(const void* Z, int64_t M, int64_t red, const void* Gt, int64_t ld_gt, int r, void* out,
+                      float* partial, cudaStream_t st);
 ql_status launch_grad_b(const void* dY, int64_t M, int N, const void* Ut, int64_t ld_ut, int r, float s, void* dB,
                         ql_dtype dt, float* partial, cudaStream_t st);
 ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t ld_vt, int r, float s, void* dA,
@@ -65,7 +64,11 @@ ql_status check_gemm_shape(const ql_nf4_weight* w, int64_t M, int r) {
   return QL_OK;
 }
 
-size_t ws_fwd(int64_t, int) { return 0; }
+// Forward workspace: U [M, r] (when U_out is not given), fp32 split-K partials.
+size_t ws_fwd(int64_t M, int64_t K, int r) {
+  if (r == 0) return 0;
+  return align256((size_t)M * r * 2) + align256(ql::skinny_partial_bytes(M, K, r));
+}
 
 // Backward workspace, carved in this order (each piece 256-byte aligned):
 //   B^T [r, N], U^T [r, Mp], U [M, r] (recomputed only when not given),
@@ -87,6 +90,7 @@ BwdWs ws_bwd_layout(int64_t M, int64_t N, int64_t K, int r) {
   size_t part = ql::skinny_partial_bytes(N, M, r);
   part = std::max(part, ql::skinny_partial_bytes(K, M, r));
   part = std::max(part, ql::skinny_partial_bytes(M, K, r));
+  part = std::max(part, ql::skinny_partial_bytes(M, N, r));
   w.part = off; off += align256(part);
   w.total = off;
   return w;
@@ -128,7 +132,17 @@ ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, con
   if (r > 0 && (!aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
   if (U_out && !aligned16(U_out)) return QL_ERR_INVALID_ARG;
   if (M == 0) return QL_OK;
-  return ql::launch_gemm_fwd(w, X, M, A, B, r, s, U_out, Y, y_dt, as_stream(stream));
+  cudaStream_t cs = as_stream(stream);
+  const int64_t K = w->cols;
+  if (r == 0) return ql::launch_gemm_fwd(w, X, M, nullptr, nullptr, 0, s, Y, y_dt, cs);
+  if (ws_bytes < ws_fwd(M, K, r)) return QL_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QL_ERR_INVALID_ARG;
+  uint8_t* wp = reinterpret_cast<uint8_t*>(ws);
+  void* U = U_out ? U_out : wp;
+  float* partial = reinterpret_cast<float*>(wp + align256((size_t)M * r * 2));
+  st = ql::launch_proj(X, M, K, A, K, r, U, partial, cs);                 // U = bf16(X A^T)
+  if (st != QL_OK) return st;
+  return ql::launch_gemm_fwd(w, X, M, U, B, r, s, Y, y_dt, cs);
 }
 
 ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
@@ -153,8 +167,7 @@ ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY
     }
     return QL_OK;
   }
-  if (r == 0)
-    return ql::launch_gemm_bwd(w, dY, M, nullptr, nullptr, 0, s, nullptr, nullptr, 0, dX, dx_dt, accumulate_dx, cs);
+  if (r == 0) return ql::launch_gemm_bwd(w, dY, M, nullptr, nullptr, 0, s, dX, dx_dt, accumulate_dx, cs);
   const BwdWs L = ws_bwd_layout(M, N, K, r);
   uint8_t* wp = reinterpret_cast<uint8_t*>(ws);
   const int64_t Mp = (M + 7) / 8 * 8;
@@ -163,20 +176,24 @@ ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY
   void* V = wp + L.v;
   void* Vt = wp + L.vt;
   float* partial = reinterpret_cast<float*>(wp + L.part);
-  st = ql::launch_transpose(B, N, r, Bt, N, cs);                                         // B^T [r, N]
+  st = ql::launch_transpose(B, N, r, Bt, N, cs);                              // B^T [r, N]
   if (st != QL_OK) return st;
   if (!U) {
-    st = ql::launch_proj_u(X, M, (int)K, A, r, wp + L.u, partial, cs);                  // U = bf16(X A^T)
+    st = ql::launch_proj(X, M, K, A, K, r, wp + L.u, partial, cs);            // U = bf16(X A^T)
     if (st != QL_OK) return st;
     U = wp + L.u;
   }
-  st = ql::launch_transpose(U, M, r, Ut, Mp, cs);                                       // U^T [r, Mp]
+  st = ql::launch_proj(dY, M, N, Bt, N, r, V, partial, cs);                  // V = bf16(dY B)
   if (st != QL_OK) return st;
-  st = ql::launch_gemm_bwd(w, dY, M, Bt, A, r, s, V, Vt, (int)Mp, dX, dx_dt, accumulate_dx, cs);  // dX, V, V^T
+  st = ql::launch_transpose(U, M, r, Ut, Mp, cs);                            // U^T [r, Mp]
   if (st != QL_OK) return st;
-  st = ql::launch_grad_b(dY, M, (int)N, Ut, Mp, r, s, dB, grad_dt, partial, cs);         // dB = s dY^T U
+  st = ql::launch_transpose(V, M, r, Vt, Mp, cs);                            // V^T [r, Mp]
   if (st != QL_OK) return st;
-  return ql::launch_grad_a(X, M, (int)K, Vt, Mp, r, s, dA, grad_dt, partial, cs);        // dA = s V^T X
+  st = ql::launch_gemm_bwd(w, dY, M, V, A, r, s, dX, dx_dt, accumulate_dx, cs);  // dX
+  if (st != QL_OK) return st;
+  st = ql::launch_grad_b(dY, M, (int)N, Ut, Mp, r, s, dB, grad_dt, partial, cs);  // dB = s dY^T U
+  if (st != QL_OK) return st;
+  return ql::launch_grad_a(X, M, (int)K, Vt, Mp, r, s, dA, grad_dt, partial, cs);   // dA = s V^T X
 }
 
 ql_status qlora_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, void* stream) {
@@ -194,7 +211,7 @@ ql_status qlora_silu_gate_bwd(const void* dh, const void* g, const void* u, void
 size_t qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r) {
   switch (op) {
     case QL_OP_DOUBLE_QUANT: return M > 0 ? ql::dq_workspace_bytes(M) : 0;
-    case QL_OP_FWD: return ws_fwd(M, r);
+    case QL_OP_FWD: return ws_fwd(M, K, r);
     case QL_OP_BWD: return ws_bwd(M, N, K, r);
     default: return 0;
   }

@@ -8,28 +8,30 @@
 // only read.
 //
 // One kernel serves both directions (row-vector convention, tokens are rows):
-//   forward  Y  = X  * W_hat^T + U * (s B)^T,  U = bf16(X  A^T)  (reduction over K)
-//   backward dX = dY * W_hat   + V * (s A),    V = bf16(dY B)    (reduction over N)
-// CTA tile: 128 tokens x 256 outputs, 64 reduction elements per pipeline stage.
-// Two shared-memory rings: a deep one (5-8 stages) for what TMA brings from
-// L2/HBM (activation tile, packed codes, side operand) so the loads run far
-// ahead of the tensor cores, and a 2-stage one for the dequantized weight tile
-// the producers write.
-// The rank-r side product (U or V) is computed in the same main loop from the
-// activation tiles already in shared memory, into a second TMEM accumulator,
-// so the activations are read from HBM once.  After the main loop it is
-// rounded to bf16 and fed back as the A operand of r extra K-steps (the LoRA
-// term) into the main accumulator before the drain.
+//   forward  Y  = X  * W_hat^T + U * (s B)^T      reduction over K (W columns)
+//   backward dX = dY * W_hat   + V * (s A)        reduction over N (W rows)
+// U = bf16(X A^T) and V = bf16(dY B) come in precomputed (rank-r side kernels).
 //
+// CTA tile: 256 tokens x 256 outputs, 64 reduction elements per stage.  The
+// 256 tokens are two M = 128 tcgen05.mma accumulators (TMEM columns 0-255 and
+// 256-511) that share one dequantized weight tile, so each expanded weight
+// element feeds 512 multiply-adds and every operand byte read from shared
+// memory does twice the work of a 128-token tile.  Shared memory bandwidth is
+// what bounds this kernel: per stage the tensor cores read 2 x (16 + 32) KB,
+// the producers write the 32 KB weight tile and TMA writes 40 KB.
+// The r LoRA K-steps (U or V against the scaled adapter) run into the same
+// accumulators after the main loop, before the drain.
+//
+// Shared memory: a TMA ring (activation tile 256 x 64 bf16 + the packed codes
+// of the weight tile) and a ring of dequantized weight tiles, 3 stages each.
 // Warp roles (576 threads):
-//   warp 0      TMA: activation tile (128 x 64 bf16), the side operand tile
-//               (A or B^T, rp x 64 bf16) and the packed NF4 codes
+//   warp 0      TMA producer
 //   warp 1      TMEM allocation; one thread issues tcgen05.mma
-//   warps 2-17  dequant producers: each pair of threads expands one 64-block
-//               of codes (32 codes each) through a per-block register lookup
-//               table into the swizzled BF16 operand tile; then the LoRA
-//               operands; then the drain of the accumulator.
-// The B operand tile holds W rows as 128-byte rows in both directions: K-major
+//   warps 2-17  dequant producers: threads pair up on one 64-block of codes
+//               (32 codes each) and expand it through a per-block register
+//               lookup table into the swizzled BF16 weight tile; then the LoRA
+//               operands; then they drain the accumulators to global memory.
+// The weight tile holds W rows as 128-byte rows in both directions: K-major
 // for the forward (rows = output features), MN-major for the backward (rows =
 // the reduction index), so the producers write the same layout either way.
 #include <cudaTypedefs.h>
@@ -43,31 +45,21 @@ using namespace sm100;
 
 namespace gemm {
 
-constexpr int BM = 128;
+constexpr int BM = 256;                 // tokens per CTA (two M = 128 accumulators)
+constexpr int BMH = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int A_BYTES = BM * BK * 2;   // 16 KB activation tile
-constexpr int B_BYTES = BN * BK * 2;   // 32 KB dequantized weight tile
-constexpr int C_BYTES = BN * BK / 2;   // 8 KB of packed codes
-constexpr int B_STAGES = 2;            // dequantized-weight ring
-constexpr int MAX_T_STAGES = 8;        // TMA ring (activation, codes, side tile)
+constexpr int A_BYTES = BM * BK * 2;    // 32 KB activation tile
+constexpr int AH_BYTES = BMH * BK * 2;  // 16 KB: second accumulator's half
+constexpr int B_BYTES = BN * BK * 2;    // 32 KB dequantized weight tile
+constexpr int C_BYTES = BN * BK / 2;    // 8 KB of packed codes
+constexpr int T_STAGES = 3;
+constexpr int B_STAGES = 3;
+constexpr int T_STAGE_BYTES = A_BYTES + C_BYTES;
 constexpr int PRODUCER_WARPS = 16;
 constexpr int THREADS = (2 + PRODUCER_WARPS) * 32;
-constexpr int TMEM_COLS = 512;         // main 256 columns + side rp columns
-constexpr int SIDE_COL = 256;
-constexpr int SMEM_LIMIT = 232448;     // opt-in maximum per CTA on sm_100
-constexpr int BAR_BYTES = 512;
-
-// Shared memory: [TMA ring: t_stages x (A | codes | side)] [B ring: 2 x B] [barriers]
-__host__ __device__ constexpr int side_bytes(int rp) { return rp * 128 < 1024 ? 1024 : rp * 128; }
-__host__ __device__ constexpr int t_stage_bytes(int rp) { return A_BYTES + C_BYTES + side_bytes(rp); }
-inline int t_stages_for(int rp) {
-  int n = (SMEM_LIMIT - 1024 - BAR_BYTES - B_STAGES * B_BYTES) / t_stage_bytes(rp);
-  return n > MAX_T_STAGES ? MAX_T_STAGES : n;
-}
-inline size_t smem_bytes_for(int rp) {
-  return 1024 + (size_t)t_stages_for(rp) * t_stage_bytes(rp) + B_STAGES * B_BYTES + BAR_BYTES;
-}
+constexpr int TMEM_COLS = 512;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)T_STAGES * T_STAGE_BYTES + (size_t)B_STAGES * B_BYTES + 256;
 
 struct Params {
   int M;             // tokens
@@ -77,54 +69,42 @@ struct Params {
   WeightConsts wc;
   int r, rp;         // rank, rank padded to 16 (0 when no adapter)
   float s;
-  const __nv_bfloat16* lora_b;   // forward B [N, r] (scaled by s in-kernel); backward A [r, K]
-  __nv_bfloat16* side_out;       // forward U_out [M, r] (may be NULL); backward V [M, r]
-  __nv_bfloat16* side_out_t;     // backward V^T [r, ld_t] (may be NULL)
-  int ld_t;
+  const __nv_bfloat16* lora_a;   // forward U [M, r]; backward V [M, r]
+  const __nv_bfloat16* lora_b;   // forward B [N, r]; backward A [r, K]; scaled by s here
   void* out;
   int out_bf16;
   int accumulate;
   NF4Table tab;
   uint32_t wait_limit;
-  int t_stages;
 };
 
 struct Smem {
   uint8_t* base;
-  int ts;        // TMA ring stages
-  int tsb;       // bytes per TMA stage
-  int sideb;     // side tile bytes
-  __device__ __forceinline__ uint8_t* a(int s) const { return base + s * tsb; }
-  __device__ __forceinline__ uint8_t* c(int s) const { return base + s * tsb + A_BYTES; }
-  __device__ __forceinline__ uint8_t* side(int s) const { return base + s * tsb + A_BYTES + C_BYTES; }
-  __device__ __forceinline__ uint8_t* b(int s) const { return base + ts * tsb + s * B_BYTES; }
-  uint64_t* full_a;    // [ts] activation + side tile landed
-  uint64_t* full_c;    // [ts] codes landed
-  uint64_t* empty_t;   // [ts] MMA done with the TMA slot
+  __device__ __forceinline__ uint8_t* a(int s) const { return base + s * T_STAGE_BYTES; }
+  __device__ __forceinline__ uint8_t* c(int s) const { return base + s * T_STAGE_BYTES + A_BYTES; }
+  __device__ __forceinline__ uint8_t* b(int s) const { return base + T_STAGES * T_STAGE_BYTES + s * B_BYTES; }
+  uint64_t* full_a;    // [T_STAGES] activation tile landed
+  uint64_t* full_c;    // [T_STAGES] codes landed
+  uint64_t* empty_t;   // [T_STAGES] MMA done with the TMA slot
   uint64_t* full_b;    // [B_STAGES] producers wrote the weight tile
   uint64_t* empty_b;   // [B_STAGES] MMA done with the weight tile
-  uint64_t* side_full;
   uint64_t* acc_full;
   uint32_t* tmem_addr;
   int* abort;
 };
 
-__device__ __forceinline__ Smem carve(uint8_t* raw, int rp, int ts) {
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
   Smem s;
   uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.base = p;
-  s.ts = ts;
-  s.tsb = t_stage_bytes(rp);
-  s.sideb = side_bytes(rp);
-  p += ts * s.tsb + B_STAGES * B_BYTES;
+  p += T_STAGES * T_STAGE_BYTES + B_STAGES * B_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(p);
   s.full_a = bars;
-  s.full_c = bars + MAX_T_STAGES;
-  s.empty_t = bars + 2 * MAX_T_STAGES;
-  s.full_b = bars + 3 * MAX_T_STAGES;
+  s.full_c = bars + T_STAGES;
+  s.empty_t = bars + 2 * T_STAGES;
+  s.full_b = bars + 3 * T_STAGES;
   s.empty_b = s.full_b + B_STAGES;
-  s.side_full = s.empty_b + B_STAGES;
-  s.acc_full = s.side_full + 1;
+  s.acc_full = s.empty_b + B_STAGES;
   s.tmem_addr = reinterpret_cast<uint32_t*>(s.acc_full + 1);
   s.abort = reinterpret_cast<int*>(s.tmem_addr + 1);
   return s;
@@ -141,8 +121,8 @@ __device__ __forceinline__ uint4 scale8(uint4 v, float s) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Raw constant of one 64-block, loaded ahead of use: the fp32 absmax, or the
-// E4M3 code and group scale of the double-quantized form.
+// Raw constant of one 64-block, loaded a stage ahead of use: the fp32 absmax,
+// or the E4M3 code and group scale of the double-quantized form.
 struct RawConst {
   float v;      // absmax, or the group scale s2
   uint32_t e;   // E4M3 code (double quant)
@@ -165,12 +145,16 @@ __device__ __forceinline__ float decode_const(const WeightConsts& wc, RawConst r
   return __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)r.e), r.v), mu);
 }
 
+__device__ __forceinline__ uint64_t b_desc(uint32_t b_addr, int kk, bool bwd) {
+  return bwd ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024) : sdesc_sw128(b_addr + kk * 32, 16, 1024);
+}
+
 template <bool BWD>
 __global__ void __launch_bounds__(THREADS, 1)
     qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_codes,
-                      const __grid_constant__ CUtensorMap tmap_side, const Params p) {
+                      const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  Smem sm = carve(smem_raw, p.rp, p.t_stages);
+  Smem sm = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * BM;
@@ -179,7 +163,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int* abort_flag = sm.abort;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < sm.ts; ++i) {
+    for (int i = 0; i < T_STAGES; ++i) {
       mbar_init(&sm.full_a[i], 1);
       mbar_init(&sm.full_c[i], 1);
       mbar_init(&sm.empty_t[i], 1);
@@ -188,7 +172,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sm.full_b[i], PRODUCER_WARPS);
       mbar_init(&sm.empty_b[i], 1);
     }
-    mbar_init(sm.side_full, 1);
     mbar_init(sm.acc_full, 1);
     *sm.abort = 0;
     fence_mbar_init();
@@ -196,7 +179,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_act);
     prefetch_tmap(&tmap_codes);
-    if (lora) prefetch_tmap(&tmap_side);
   }
   if (warp == 1) {
     tmem_alloc(sm.tmem_addr, TMEM_COLS);
@@ -210,25 +192,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA warp
     if (lane == 0) {
-      const uint32_t a_tx = A_BYTES + (lora ? p.rp * 128 : 0);
-      const int TS = sm.ts;
       int issued = 0;
       for (int i = 0; i < p.n_steps; ++i) {
-        const int s = i % TS, use = i / TS;
+        const int s = i % T_STAGES, use = i / T_STAGES;
         if (use > 0 && !mbar_wait(&sm.empty_t[s], (use - 1) & 1, abort_flag, p.wait_limit)) break;
         mbar_arrive_expect_tx(&sm.full_c[s], C_BYTES);
         if (!BWD)
           tma_load_2d(sm.c(s), &tmap_codes, &sm.full_c[s], i * (BK / 2), j0);
         else
           tma_load_2d(sm.c(s), &tmap_codes, &sm.full_c[s], j0 / 2, i * BK);
-        mbar_arrive_expect_tx(&sm.full_a[s], a_tx);
+        mbar_arrive_expect_tx(&sm.full_a[s], A_BYTES);
         tma_load_2d(sm.a(s), &tmap_act, &sm.full_a[s], i * BK, m0);
-        if (lora) tma_load_2d(sm.side(s), &tmap_side, &sm.full_a[s], i * BK, 0);
         issued = i + 1;
       }
       // before leaving, make sure no copy is still landing in shared memory
-      for (int i = (issued > TS ? issued - TS : 0); i < issued; ++i) {
-        const int s = i % TS, use = i / TS;
+      for (int i = (issued > T_STAGES ? issued - T_STAGES : 0); i < issued; ++i) {
+        const int s = i % T_STAGES, use = i / T_STAGES;
         mbar_wait(&sm.full_a[s], use & 1, abort_flag, p.wait_limit);
         mbar_wait(&sm.full_c[s], use & 1, abort_flag, p.wait_limit);
       }
@@ -236,12 +215,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16(BM, BN, false, BWD);
-      const uint32_t idesc_side = idesc_bf16(BM, lora ? p.rp : 16, false, false);
-      const int TS = sm.ts;
+      constexpr uint32_t IDESC = idesc_bf16(BMH, BN, false, BWD);
       bool ok = true;
       for (int i = 0; i < p.n_steps && ok; ++i) {
-        const int s = i % TS, use = i / TS;
+        const int s = i % T_STAGES, use = i / T_STAGES;
         const int sb = i % B_STAGES, useb = i / B_STAGES;
         ok = mbar_wait(&sm.full_a[s], use & 1, abort_flag, p.wait_limit) &&
              mbar_wait(&sm.full_b[sb], useb & 1, abort_flag, p.wait_limit);
@@ -249,34 +226,29 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sm.a(s));
         const uint32_t b_addr = smem_u32(sm.b(sb));
-        const uint32_t s_addr = smem_u32(sm.side(s));
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
-          const uint64_t bd = BWD ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
-                                  : sdesc_sw128(b_addr + kk * 32, 16, 1024);
+          const uint64_t bd = b_desc(b_addr, kk, BWD);
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16(tmem, ad, bd, IDESC, acc);
-          if (lora) mma_bf16(tmem + SIDE_COL, ad, sdesc_sw128(s_addr + kk * 32, 16, 1024), idesc_side, acc);
+          mma_bf16(tmem, sdesc_sw128(a_addr + kk * 32, 16, 1024), bd, IDESC, acc);
+          mma_bf16(tmem + 256, sdesc_sw128(a_addr + AH_BYTES + kk * 32, 16, 1024), bd, IDESC, acc);
         }
         mma_commit(&sm.empty_t[s]);
         mma_commit(&sm.empty_b[sb]);
       }
       if (ok && lora) {
-        mma_commit(sm.side_full);
-        // LoRA K-steps: A = bf16 side product, B = scaled adapter, into the main accumulator
+        // LoRA K-steps: A = U or V tile, B = scaled adapter, into both accumulators
         const int i = p.n_steps;
-        const int s = i % TS, sb = i % B_STAGES, useb = i / B_STAGES;
+        const int s = i % T_STAGES, sb = i % B_STAGES, useb = i / B_STAGES;
         ok = mbar_wait(&sm.full_b[sb], useb & 1, abort_flag, p.wait_limit);
         if (ok) {
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sm.a(s));
           const uint32_t b_addr = smem_u32(sm.b(sb));
           for (int kk = 0; kk < p.rp / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = BWD ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
-                                    : sdesc_sw128(b_addr + kk * 32, 16, 1024);
-            mma_bf16(tmem, ad, bd, IDESC, 1u);
+            const uint64_t bd = b_desc(b_addr, kk, BWD);
+            mma_bf16(tmem, sdesc_sw128(a_addr + kk * 32, 16, 1024), bd, IDESC, 1u);
+            mma_bf16(tmem + 256, sdesc_sw128(a_addr + AH_BYTES + kk * 32, 16, 1024), bd, IDESC, 1u);
           }
         }
       }
@@ -289,21 +261,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     // quarter-warp touches 8 different rows and the swizzled shared-memory
     // accesses below are free of bank conflicts.
     const int wp = warp - 2;                                   // 0..15
+    const int pt = threadIdx.x - 64;                           // 0..511
     const int half = (lane >> 3) & 1;                          // which 32 codes of the 64-block
     const int row_local = (lane & 7) + 8 * (lane >> 4);        // 0..15
-    const int kblocks = p.K / 64;      // 64-blocks per weight row
+    const int kblocks = p.K / 64;                              // 64-blocks per weight row
     const float mu = p.wc.absmax ? 0.0f : *p.wc.offset;
-    // which weight row / 64-block column this thread expands in every stage
     int row_in_tile, col_chunk;
     if (!BWD) { row_in_tile = 16 * wp + row_local; col_chunk = 0; }
     else { row_in_tile = 16 * (wp & 3) + row_local; col_chunk = wp >> 2; }
     // byte offset of this thread's 16-byte code chunk in the swizzled code tile
     uint32_t coff;
-    if (!BWD) {   // 32-byte rows, 32B swizzle: chunk ^= bit 2 of the row
-      coff = row_in_tile * 32 + ((half ^ ((row_in_tile >> 2) & 1)) << 4);
-    } else {      // 128-byte rows, 128B swizzle: chunk ^= row mod 8
-      coff = row_in_tile * 128 + (((2 * col_chunk + half) ^ (row_in_tile & 7)) << 4);
-    }
+    if (!BWD) coff = row_in_tile * 32 + ((half ^ ((row_in_tile >> 2) & 1)) << 4);          // 32B swizzle
+    else coff = row_in_tile * 128 + (((2 * col_chunk + half) ^ (row_in_tile & 7)) << 4);   // 128B swizzle
     auto step_row = [&](int i, int& wrow, int& kb) {
       if (!BWD) { wrow = j0 + row_in_tile; kb = i; }
       else { wrow = i * BK + row_in_tile; kb = j0 / 64 + col_chunk; }
@@ -313,9 +282,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool valid = wrow < p.N && kb < kblocks;
     RawConst next = load_const(p.wc, (int64_t)wrow * kblocks + kb, valid);
     bool ok = true;
-    const int TS = sm.ts;
     for (int i = 0; i < p.n_steps && ok; ++i) {
-      const int s = i % TS, use = i / TS;
+      const int s = i % T_STAGES, use = i / T_STAGES;
       const int sb = i % B_STAGES, useb = i / B_STAGES;
       const RawConst cur = next;
       const bool cur_valid = valid;
@@ -347,74 +315,46 @@ __global__ void __launch_bounds__(THREADS, 1)
     // LoRA operands into the slots after the last main step
     if (ok && lora) {
       const int i = p.n_steps;
-      const int s = i % TS, use = i / TS;
+      const int s = i % T_STAGES, use = i / T_STAGES;
       const int sb = i % B_STAGES, useb = i / B_STAGES;
-      if (use > 0) ok = __all_sync(0xffffffffu, mbar_wait(&sm.empty_t[s], (use - 1) & 1, abort_flag, p.wait_limit));
-      if (ok && useb > 0)
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.empty_b[sb], (useb - 1) & 1, abort_flag, p.wait_limit));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(sm.side_full, 0, abort_flag, p.wait_limit));
+      ok = __all_sync(0xffffffffu, (use == 0 || mbar_wait(&sm.empty_t[s], (use - 1) & 1, abort_flag, p.wait_limit)) &&
+                                       (useb == 0 || mbar_wait(&sm.empty_b[sb], (useb - 1) & 1, abort_flag,
+                                                               p.wait_limit)));
       if (ok) {
-        tc_fence_after();
-        if (warp < 6) {
-          // A operand: the side product (U or V), rounded to bf16, from TMEM
-          const int quad = warp & 3;
-          const int row = quad * 32 + lane;
+        // A operand: U or V rows m0 .. m0+255, K-major (256 rows x rp)
+        {
+          const int row = pt >> 1, hh = pt & 1;
           const int m = m0 + row;
-          const bool write_side = p.side_out && blockIdx.x == 0 && m < p.M;
-          const bool write_side_t = p.side_out_t && blockIdx.x == 0 && m < p.M;
-          for (int c16 = 0; c16 < p.rp / 16; ++c16) {
-            uint32_t v[16];
-            tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(SIDE_COL + c16 * 16), v);
-            tmem_ld_wait();
-            uint32_t pk[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) pk[q] = pack_bf16x2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
-            *reinterpret_cast<uint4*>(sm.a(s) + sw128_offset(row, 2 * c16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4*>(sm.a(s) + sw128_offset(row, 2 * c16 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            if (write_side) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const int j = c16 * 16 + 2 * q;
-                if (j < p.r) *reinterpret_cast<uint32_t*>(p.side_out + (size_t)m * p.r + j) = pk[q];
-              }
-            }
-            if (write_side_t) {
-#pragma unroll
-              for (int q = 0; q < 16; ++q) {
-                const int j = c16 * 16 + q;
-                if (j < p.r) {
-                  const uint32_t h = (q & 1) ? (pk[q >> 1] >> 16) : (pk[q >> 1] & 0xFFFFu);
-                  reinterpret_cast<uint16_t*>(p.side_out_t)[(size_t)j * p.ld_t + m] = (uint16_t)h;
-                }
-              }
-            }
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = hh * 4 + q;
+            const int e = chunk * 8;
+            if (e >= p.rp) break;
+            uint4 v = zero4();
+            if (m < p.M && e < p.r) v = *reinterpret_cast<const uint4*>(p.lora_a + (size_t)m * p.r + e);
+            *reinterpret_cast<uint4*>(sm.a(s) + (row >> 7) * AH_BYTES + sw128_offset(row & 127, chunk)) = v;
+          }
+        }
+        if (!BWD) {
+          // B operand: (s B)[n, 0..rp) for the 256 output features, K-major
+          const int rr = pt >> 1, hh = pt & 1;
+          const int n = j0 + rr;
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = hh * 4 + q;
+            const int e = chunk * 8;
+            if (e >= p.rp) break;
+            uint4 v = zero4();
+            if (n < p.N && e < p.r) v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)n * p.r + e), p.s);
+            *reinterpret_cast<uint4*>(sm.b(sb) + sw128_offset(rr, chunk)) = v;
           }
         } else {
-          const int t = threadIdx.x - 6 * 32;   // 0..383
-          constexpr int NT = (PRODUCER_WARPS - 4) * 32;
-          if (!BWD) {
-            // B operand: (s B)[n, 0..rp) for the 256 output features, K-major
-            for (int rr = t; rr < BN; rr += NT) {
-              const int n = j0 + rr;
-              for (int chunk = 0; chunk < p.rp / 8; ++chunk) {
-                const int e = chunk * 8;
-                uint4 v = zero4();
-                if (n < p.N && e < p.r)
-                  v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)n * p.r + e), p.s);
-                *reinterpret_cast<uint4*>(sm.b(sb) + sw128_offset(rr, chunk)) = v;
-              }
-            }
-          } else {
-            // B operand: (s A)[0..rp, k] for the 256 output columns, MN-major
-            for (int idx = t; idx < p.rp * 32; idx += NT) {
-              const int jr = idx >> 5, rem = idx & 31;
-              const int cc = rem >> 3, piece = rem & 7;
-              const int k = j0 + cc * 64 + piece * 8;
-              uint4 v = zero4();
-              if (jr < p.r && k < p.K)
-                v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)jr * p.K + k), p.s);
-              *reinterpret_cast<uint4*>(sm.b(sb) + cc * 8192 + sw128_offset(jr, piece)) = v;
-            }
+          // B operand: (s A)[0..rp, k] for the 256 output columns, MN-major
+          for (int idx = pt; idx < p.rp * 32; idx += PRODUCER_WARPS * 32) {
+            const int jr = idx >> 5, rem = idx & 31;
+            const int cc = rem >> 3, piece = rem & 7;
+            const int k = j0 + cc * 64 + piece * 8;
+            uint4 v = zero4();
+            if (jr < p.r && k < p.K) v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)jr * p.K + k), p.s);
+            *reinterpret_cast<uint4*>(sm.b(sb) + cc * 8192 + sw128_offset(jr, piece)) = v;
           }
         }
         fence_proxy_async_smem();
@@ -427,12 +367,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (acc_ok) {
       tc_fence_after();
       const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
-      const int col_q = (warp - 2) >> 2;         // columns 64*col_q .. +63
-      const int row = m0 + quad * 32 + lane;
-      for (int cc = 0; cc < 4; ++cc) {
-        const int col = col_q * 64 + cc * 16;
+      const int g = wp >> 2;                     // 0..3: accumulator g>>1, columns (g&1)*128 ..
+      const int accn = g >> 1;
+      const int row = m0 + accn * BMH + quad * 32 + lane;
+      for (int cc = 0; cc < 8; ++cc) {
+        const int col = (g & 1) * 128 + cc * 16;
         uint32_t r[16];
-        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)col, r);
+        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(accn * 256 + col), r);
         tmem_ld_wait();
         const int gcol = j0 + col;
         if (row < p.M && gcol < p.n_out) {
@@ -473,7 +414,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // ------------------------------------------------------------ teardown
   if (warp == 1 && lane == 0 && *abort_flag) {
-    // let MMAs already issued finish before the accumulator is released
+    // let MMAs already issued finish before the accumulators are released
     mbar_wait(sm.acc_full, 0, abort_flag, p.wait_limit);
   }
   tc_fence_before();
@@ -517,20 +458,18 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const
 }
 
 template <bool BWD>
-static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64_t M, const void* side_src,
-                                  const void* lora_b, int r, float s, void* side_out, void* side_out_t, int ld_t,
-                                  void* out, ql_dtype out_dt, int accumulate, cudaStream_t st) {
+static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64_t M, const void* lora_a,
+                                  const void* lora_b, int r, float s, void* out, ql_dtype out_dt, int accumulate,
+                                  cudaStream_t st) {
   using namespace gemm;
   static bool attr_set = false;
   if (!attr_set) {
     QL_CUDA_TRY(cudaFuncSetAttribute(qlora_gemm_kernel<BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     SMEM_LIMIT));
+                                     (int)SMEM_BYTES));
     attr_set = true;
   }
   const int N = (int)w->rows, K = (int)w->cols;
-  const int rp = r > 0 ? (r + 15) / 16 * 16 : 0;
-  const size_t smem = smem_bytes_for(rp);
-  CUtensorMap map_act, map_codes, map_side;
+  CUtensorMap map_act, map_codes;
   const int red = BWD ? N : K;   // reduction length = activation row length
   if (!make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, (uint64_t)red, (uint64_t)M, (uint64_t)red, BK,
                    BM, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -544,14 +483,6 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
                      (uint64_t)K / 2, BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_128B))
       return QL_ERR_CUDA;
   }
-  if (r > 0) {
-    // side operand [r, red] bf16: A (forward) or B^T (backward); rows r..rp-1 read as zeros
-    if (!make_map_2d(&map_side, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, side_src, (uint64_t)red, (uint64_t)r,
-                     (uint64_t)red, BK, (uint32_t)rp, CU_TENSOR_MAP_SWIZZLE_128B))
-      return QL_ERR_CUDA;
-  } else {
-    map_side = map_act;   // unused
-  }
   Params p;
   p.M = (int)M;
   p.n_out = BWD ? K : N;
@@ -560,38 +491,32 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
   p.K = K;
   p.wc = WeightConsts{w->absmax, w->absmax_q, w->scale2, w->offset};
   p.r = r;
-  p.rp = rp;
+  p.rp = r > 0 ? (r + 15) / 16 * 16 : 0;
   p.s = s;
+  p.lora_a = (const __nv_bfloat16*)lora_a;
   p.lora_b = (const __nv_bfloat16*)lora_b;
-  p.side_out = (__nv_bfloat16*)side_out;
-  p.side_out_t = (__nv_bfloat16*)side_out_t;
-  p.ld_t = ld_t;
   p.out = out;
   p.out_bf16 = out_dt == QL_BF16;
   p.accumulate = accumulate;
   p.tab = nf4_table();
   p.wait_limit = 1u << 22;
-  p.t_stages = t_stages_for(rp);
   dim3 grid((unsigned)((p.n_out + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
   TraceScope ts(BWD ? TK_GEMM_BWD : TK_GEMM_FWD, st);
-  qlora_gemm_kernel<BWD><<<grid, THREADS, smem, st>>>(map_act, map_codes, map_side, p);
+  qlora_gemm_kernel<BWD><<<grid, THREADS, SMEM_BYTES, st>>>(map_act, map_codes, p);
   QL_LAUNCH_CHECK();
   return QL_OK;
 }
 
-// Y = X W_hat^T + U (s B)^T with U = bf16(X A^T) computed in the same kernel;
-// U is also written to U_out when given.
-ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* A, const void* B, int r,
-                          float s, void* U_out, void* Y, ql_dtype y_dt, cudaStream_t st) {
-  return launch_gemm_impl<false>(w, X, M, A, B, r, s, U_out, nullptr, 0, Y, y_dt, 0, st);
+// Y = X W_hat^T + U (s B)^T, U = bf16(X A^T) given [M, r]
+ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
+                          float s, void* Y, ql_dtype y_dt, cudaStream_t st) {
+  return launch_gemm_impl<false>(w, X, M, U, B, r, s, Y, y_dt, 0, st);
 }
 
-// dX (+)= dY W_hat + V (s A) with V = bf16(dY B) computed in the same kernel
-// from B^T [r, N]; V [M, r] and V^T [r, ld_t] are written for the gradients.
-ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* Bt, const void* A, int r,
-                          float s, void* V, void* Vt, int ld_t, void* dX, ql_dtype dx_dt, int accumulate,
-                          cudaStream_t st) {
-  return launch_gemm_impl<true>(w, dY, M, Bt, A, r, s, V, Vt, ld_t, dX, dx_dt, accumulate, st);
+// dX (+)= dY W_hat + V (s A), V = bf16(dY B) given [M, r]
+ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* V, const void* A, int r,
+                          float s, void* dX, ql_dtype dx_dt, int accumulate, cudaStream_t st) {
+  return launch_gemm_impl<true>(w, dY, M, V, A, r, s, dX, dx_dt, accumulate, st);
 }
 
 }  // namespace ql

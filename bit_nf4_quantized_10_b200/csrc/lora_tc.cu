@@ -2,7 +2,7 @@
 // Model on One GPU", "Where the gradients actually go": only A and B receive
 // gradients; "Prerequisite: LoRA's low-rank update": B is d x r, A is r x k):
 //   dB = s dY^T U   [N, r]     dA = s V^T X   [r, K]
-// and, when the caller did not keep it from the forward, U = bf16(X A^T).
+// and the rank-r side products U = bf16(X A^T), V = bf16(dY B).
 //
 // All three are skinny products C[rows x r] = Z_op[rows x red] * G[red x r]
 // with r <= 64: tcgen05.mma with M = 128 output rows and N = r (padded to 16),
@@ -11,6 +11,7 @@
 //   dB: Z_op = dY^T (MN-major view of dY [M, N]), G^T = U^T [r, M]
 //   dA: Z_op = X^T  (MN-major view of X  [M, K]), G^T = V^T [r, M]
 //   U:  Z_op = X    (K-major),                     G^T = A   [r, K]
+//   V:  Z_op = dY   (K-major),                     G^T = B^T [r, N]
 // They stream one activation matrix once, so they are bound by its HBM read.
 #include <cudaTypedefs.h>
 
@@ -266,10 +267,10 @@ static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, 
   return QL_OK;
 }
 
-// U = bf16(X A^T), X [M, K], A [r, K]
-ql_status launch_proj_u(const void* X, int64_t M, int K, const void* A, int r, void* U, float* partial,
-                        cudaStream_t st) {
-  return skinny_launch(false, X, (int)M, K, A, r, K, 1.0f, 0, U, QL_BF16, partial, TK_PROJ, st);
+// side = bf16(Z G): Z [M, red] (X or dY), G^T [r, ld_gt] (A or B^T); out [M, r]
+ql_status launch_proj(const void* Z, int64_t M, int64_t red, const void* Gt, int64_t ld_gt, int r, void* out,
+                      float* partial, cudaStream_t st) {
+  return skinny_launch(false, Z, (int)M, red, Gt, r, ld_gt, 1.0f, 0, out, QL_BF16, partial, TK_PROJ, st);
 }
 
 // dB = s dY^T U: dY [M, N], U^T [r, ld_ut]

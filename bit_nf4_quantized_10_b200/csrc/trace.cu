@@ -19,7 +19,7 @@ std::mutex g_mu;
 std::vector<Rec> g_recs;
 std::vector<cudaEvent_t> g_free;
 const char* const kNames[TK_COUNT] = {"nf4_quantize",   "dq_tree_sum",    "dq_encode",       "nf4_dequant",
-                                      "qlora_gemm_fwd", "qlora_gemm_bwd", "lora_u_recompute", "lora_grad",
+                                      "qlora_gemm_fwd", "qlora_gemm_bwd", "lora_side_proj", "lora_grad",
                                       "lora_grad_reduce", "silu_gate",    "smallm_splitk",   "lora_transpose"};
 }  // namespace
 

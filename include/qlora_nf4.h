@@ -140,12 +140,12 @@ ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* 
  *   s      alpha / r
  *   Y      device out [M, N] of y_dt
  *   U_out  device out bf16 [M, r] (the tensor the backward reuses) or NULL
- *   ws     workspace >= qlora_workspace_size(QL_OP_FWD, M, N, K, r), which
- *          is 0 in this version (ws may be NULL)
+ *   ws     workspace >= qlora_workspace_size(QL_OP_FWD, M, N, K, r) (0 when
+ *          r == 0; ws may then be NULL)
  * The main product accumulates in fp32 on the tensor cores from the exact
- * bf16 W_hat.  U is accumulated in fp32 in the same kernel and rounded to
- * bf16; the adapter term U (s B)^T enters the main fp32 accumulator with
- * s B rounded to bf16 (exact when s is a power of two).
+ * bf16 W_hat.  U is accumulated in fp32 (split over K, summed in a fixed
+ * order) and rounded to bf16; the adapter term U (s B)^T enters the main fp32
+ * accumulator with s B rounded to bf16 (exact when s is a power of two).
  */
 ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M,
                            const void* A, const void* B, int r, float s,

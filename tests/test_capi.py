@@ -53,7 +53,8 @@ def test_storage_bytes_equals_oracle(lib, n):
 def test_workspace_sizes(lib):
     assert lib.qlora_workspace_size(lib.QL_OP_DOUBLE_QUANT, 2048) >= 8
     assert lib.qlora_workspace_size(lib.QL_OP_DOUBLE_QUANT, 64 * 2 ** 20) >= 8 * (2 ** 26 // 2048)
-    assert lib.qlora_workspace_size(lib.QL_OP_FWD, 4096, 4096, 4096, 16) == 0    # U is fused into the GEMM
+    assert lib.qlora_workspace_size(lib.QL_OP_FWD, 4096, 4096, 4096, 16) >= 4096 * 16 * 2
+    assert lib.qlora_workspace_size(lib.QL_OP_FWD, 4096, 4096, 4096, 0) == 0
     assert lib.qlora_workspace_size(lib.QL_OP_BWD, 4096, 4096, 4096, 16) >= 2 * 4096 * 16 * 2
 
 
@@ -75,6 +76,8 @@ def test_argument_errors_return_before_launch(lib):
                               1 << 20, s0) == lib.QL_ERR_INVALID_ARG                            # r % 8
     assert L.qlora_linear_fwd(ctypes.byref(w), fake, 16, fake, fake, 128, 2.0, fake, lib.QL_F32, None, fake,
                               1 << 20, s0) == lib.QL_ERR_UNSUPPORTED                            # r > 64
+    assert L.qlora_linear_fwd(ctypes.byref(w), fake, 16, fake, fake, 8, 2.0, fake, lib.QL_F32, None, fake,
+                              0, s0) == lib.QL_ERR_WORKSPACE
     assert L.qlora_linear_bwd(ctypes.byref(w), fake, fake, 16, fake, fake, 8, 2.0, None, fake, lib.QL_F32, 0,
                               fake, fake, lib.QL_F32, fake, 0, s0) == lib.QL_ERR_WORKSPACE
     assert L.nf4_dequant(None, fake, lib.QL_BF16, s0) == lib.QL_ERR_INVALID_ARG
