@@ -19,32 +19,17 @@ namespace ql {
 QL_DEFINE_STATUS_ACCESSOR(status_word_codec)
 
 // ---------------------------------------------------------------- quantize
-// Code of x: #{j : x > t_j} over the 15 sorted thresholds, found with a
-// branch-free 4-step binary search.  Ties (x == t_j) go to the lower level.
-__device__ __forceinline__ uint32_t nf4_code(float x, const float (&t)[15]) {
-  uint32_t k = (x > t[7]) ? 8u : 0u;
-  float t2 = k ? t[11] : t[3];
+// Code of x: #{j : x > t_j} over the 15 sorted thresholds t_j = fl32(m_j c),
+// found by a 4-step binary search.  The first two steps compare against
+// t_7 and t_3 / t_11 held in registers; the last two read the block's
+// thresholds from shared memory at a data-dependent index (no divergent
+// branches).  Ties (x == t_j) go to the lower level.
+__device__ __forceinline__ uint32_t nf4_code(float x, float t3, float t7, float t11, const float* tb) {
+  uint32_t k = (x > t7) ? 8u : 0u;
+  const float t2 = k ? t11 : t3;
   k += (x > t2) ? 4u : 0u;
-  float t1;
-  switch (k) {  // k in {0,4,8,12}; threshold index k + 1
-    case 0: t1 = t[1]; break;
-    case 4: t1 = t[5]; break;
-    case 8: t1 = t[9]; break;
-    default: t1 = t[13]; break;
-  }
-  k += (x > t1) ? 2u : 0u;
-  float t0;
-  switch (k) {  // k even; threshold index k
-    case 0: t0 = t[0]; break;
-    case 2: t0 = t[2]; break;
-    case 4: t0 = t[4]; break;
-    case 6: t0 = t[6]; break;
-    case 8: t0 = t[8]; break;
-    case 10: t0 = t[10]; break;
-    case 12: t0 = t[12]; break;
-    default: t0 = t[14]; break;
-  }
-  k += (x > t0) ? 1u : 0u;
+  k += (x > tb[k + 1]) ? 2u : 0u;
+  k += (x > tb[k]) ? 1u : 0u;
   return k;
 }
 
@@ -89,13 +74,17 @@ template <typename T>
 __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, int64_t n,
                                                        uint8_t* __restrict__ codes,
                                                        float* __restrict__ absmax, NF4Table tab) {
+  // per warp: 4 blocks x 15 thresholds (row pitch 17 spreads the blocks over banks)
+  __shared__ float thr[8][4][17];
   const int64_t nb = (n + 63) / 64;
   const int lane8 = threadIdx.x & 7;
+  const int wib = threadIdx.x >> 5;              // warp in CTA
+  const int bq = (threadIdx.x >> 3) & 3;         // block within the warp's four
+  float* tb = thr[wib][bq];
   // the whole warp (4 blocks) iterates together so the shuffles see all lanes
   const int64_t warps_per_grid = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t wb = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4; wb < nb;
-       wb += warps_per_grid * 4) {
-    const int64_t b = wb + ((threadIdx.x >> 3) & 3);
+  for (int64_t wb = ((int64_t)blockIdx.x * (blockDim.x >> 5) + wib) * 4; wb < nb; wb += warps_per_grid * 4) {
+    const int64_t b = wb + bq;
     const int64_t e0 = b * 64 + lane8 * 8;   // >= n for a block past the end
     float v[8];
     load8<T>(x, e0, n, v);
@@ -115,15 +104,16 @@ __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, 
     }
     if (anybad && lane8 == 0) raise_status(ST_NONFINITE);
     const float c = amax;
-    float t[15];
-#pragma unroll
-    for (int j = 0; j < 15; ++j) t[j] = __fmul_rn(tab.m[j], c);
+    // the block's 15 thresholds: lane8 j writes t_{2j} and t_{2j+1}
+    __syncwarp();
+    tb[2 * lane8] = __fmul_rn(tab.m[2 * lane8], c);
+    if (lane8 < 7) tb[2 * lane8 + 1] = __fmul_rn(tab.m[2 * lane8 + 1], c);
+    const float t3 = __fmul_rn(tab.m[3], c), t7 = __fmul_rn(tab.m[7], c), t11 = __fmul_rn(tab.m[11], c);
+    __syncwarp();
     uint32_t word = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      uint32_t code = (c == 0.0f) ? 8u : nf4_code(v[i], t);
-      word |= code << (4 * i);
-    }
+    for (int i = 0; i < 8; ++i) word |= nf4_code(v[i], t3, t7, t11, tb) << (4 * i);
+    if (c == 0.0f) word = 0x88888888u;
     if (e0 + 8 <= n) {
       __stcs(reinterpret_cast<uint32_t*>(codes + (e0 >> 1)), word);
     } else if (e0 < n) {
