@@ -20,7 +20,7 @@ QL_OK, QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_WORKSPACE, QL_ERR_CUDA, QL
 QL_F32, QL_BF16 = 0, 1
 QL_OP_DOUBLE_QUANT, QL_OP_FWD, QL_OP_BWD = 0, 1, 2
 
-EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
+EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_double_quant_noalloc", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
            "qlora_silu_gate_fwd", "qlora_silu_gate_bwd", "qlora_workspace_size", "nf4_storage_bytes",
            "nf4_codebook", "qlora_get_status", "qlora_status_string")
 
@@ -46,6 +46,7 @@ def _load() -> ctypes.CDLL:
     sig = {
         "nf4_quantize": (i32, [vp, i32, i64, vp, vp, vp]),
         "nf4_double_quant": (i32, [vp, i64, vp, vp, vp, vp, sz, vp]),
+        "nf4_double_quant_noalloc": (i32, [vp, i64, vp, vp, vp, vp]),
         "nf4_dequant": (i32, [W, vp, i32, vp]),
         "qlora_linear_fwd": (i32, [W, vp, i64, vp, vp, i32, f32, vp, i32, vp, vp, sz, vp]),
         "qlora_linear_bwd": (i32, [W, vp, vp, i64, vp, vp, i32, f32, vp, vp, i32, i32, vp, vp, i32, vp, sz, vp]),
@@ -129,6 +130,14 @@ def nf4_double_quant(absmax: torch.Tensor, absmax_q: torch.Tensor, scale2: torch
                      ws: torch.Tensor, stream=None) -> None:
     _check(LIB.nf4_double_quant(_ptr(absmax), absmax.numel(), _ptr(absmax_q), _ptr(scale2), _ptr(offset),
                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "nf4_double_quant")
+
+
+def nf4_double_quant_noalloc(absmax: torch.Tensor, absmax_q: torch.Tensor, scale2: torch.Tensor,
+                             offset: torch.Tensor, stream=None) -> None:
+    """nf4_double_quant without a workspace, for callers that cannot allocate
+    device memory; the library uses a fixed internal scratch array instead."""
+    _check(LIB.nf4_double_quant_noalloc(_ptr(absmax), absmax.numel(), _ptr(absmax_q), _ptr(scale2), _ptr(offset),
+                                        _stream(stream)), "nf4_double_quant_noalloc")
 
 
 def nf4_dequant(w: "NF4Weight", out: torch.Tensor, stream=None) -> None:

@@ -124,6 +124,28 @@ ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q,
                            void* stream);
 
 /*
+ * nf4_double_quant_noalloc — nf4_double_quant for callers that cannot
+ * allocate device memory (no workspace argument).  The pages have no
+ * counterpart; this is a library convenience.  Callers such as a plugin or
+ * custom operator handed only tensors and a stream by a framework that owns
+ * the device memory pool, or code that must not call cudaMalloc (it can
+ * synchronize the device), use this instead of providing `ws`.
+ *   Same arguments, outputs and results as nf4_double_quant, bit for bit.
+ *   nb must be <= QL_NOALLOC_MAX_BLOCKS (64 Mi constants, i.e. weights of up
+ *   to 4 Gi elements); larger nb returns QL_ERR_UNSUPPORTED.
+ *   The scratch is a fixed 256.5 KiB array of device memory inside the
+ *   library, held by every GPU that loads it until the process exits.  The
+ *   first call on a device looks its address up (cudaGetSymbolAddress), so
+ *   make that first call before any stream capture.  All calls on a device
+ *   share the array: calls whose kernels may overlap on the GPU (different
+ *   streams with no ordering) race and must not be issued.  The library never
+ *   calls cudaMalloc, cudaFree or an allocating routine here.
+ */
+#define QL_NOALLOC_MAX_BLOCKS (1ll << 26)
+ql_status nf4_double_quant_noalloc(const float* absmax, int64_t nb, uint8_t* absmax_q,
+                                   float* scale2, float* offset, void* stream);
+
+/*
  * nf4_dequant — x_hat = bf16(fl32(q_code * c)) ([P3] "Quantization in one
  * paragraph"; [P2] §3 dequantize to BF16), c = absmax[b] or the double-quant
  * reconstruction when w->absmax is NULL.  out: device, rows*cols elements of
