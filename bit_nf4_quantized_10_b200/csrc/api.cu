@@ -28,6 +28,10 @@ ql_status launch_grad_b(const void* dY, int64_t M, int N, const void* Ut, int64_
 ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t ld_vt, int r, float s, void* dA,
                         ql_dtype dt, float* partial, cudaStream_t st);
 ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st);
+// smallm.cu
+size_t smallm_partial_bytes(int64_t N, int64_t K);
+ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
+                            float s, void* Y, ql_dtype y_dt, float* partial, cudaStream_t st);
 // mlp.cu
 ql_status launch_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, cudaStream_t st);
 ql_status launch_silu_gate_bwd(const void* dh, const void* g, const void* u, void* dg, void* du, int64_t n,
@@ -64,10 +68,16 @@ ql_status check_gemm_shape(const ql_nf4_weight* w, int64_t M, int r) {
   return QL_OK;
 }
 
-// Forward workspace: U [M, r] (when U_out is not given), fp32 split-K partials.
-size_t ws_fwd(int64_t M, int64_t K, int r) {
-  if (r == 0) return 0;
-  return align256((size_t)M * r * 2) + align256(ql::skinny_partial_bytes(M, K, r));
+// Tokens up to this count take the small-M (HBM-bound) forward kernel.
+constexpr int64_t kSmallM = 16;
+
+// Forward workspace: U [M, r] (when U_out is not given), then fp32 split-K
+// partials shared by the U projection and, for M <= 16, the small-M kernel.
+size_t ws_fwd(int64_t M, int64_t N, int64_t K, int r) {
+  size_t part = r > 0 ? ql::skinny_partial_bytes(M, K, r) : 0;
+  if (M <= kSmallM) part = std::max(part, ql::smallm_partial_bytes(N, K));
+  if (part == 0) return 0;
+  return align256((size_t)M * r * 2) + align256(part);
 }
 
 // Backward workspace, carved in this order (each piece 256-byte aligned):
@@ -133,15 +143,19 @@ ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, con
   if (U_out && !aligned16(U_out)) return QL_ERR_INVALID_ARG;
   if (M == 0) return QL_OK;
   cudaStream_t cs = as_stream(stream);
-  const int64_t K = w->cols;
-  if (r == 0) return ql::launch_gemm_fwd(w, X, M, nullptr, nullptr, 0, s, Y, y_dt, cs);
-  if (ws_bytes < ws_fwd(M, K, r)) return QL_ERR_WORKSPACE;
+  const int64_t N = w->rows, K = w->cols;
+  const bool small = M <= kSmallM;
+  if (r == 0 && !small) return ql::launch_gemm_fwd(w, X, M, nullptr, nullptr, 0, s, Y, y_dt, cs);
+  if (ws_bytes < ws_fwd(M, N, K, r)) return QL_ERR_WORKSPACE;
   if (!aligned16(ws)) return QL_ERR_INVALID_ARG;
   uint8_t* wp = reinterpret_cast<uint8_t*>(ws);
   void* U = U_out ? U_out : wp;
   float* partial = reinterpret_cast<float*>(wp + align256((size_t)M * r * 2));
-  st = ql::launch_proj(X, M, K, A, K, r, U, partial, cs);                 // U = bf16(X A^T)
-  if (st != QL_OK) return st;
+  if (r > 0) {
+    st = ql::launch_proj(X, M, K, A, K, r, U, partial, cs);                 // U = bf16(X A^T)
+    if (st != QL_OK) return st;
+  }
+  if (small) return ql::launch_smallm_fwd(w, X, M, U, B, r, s, Y, y_dt, partial, cs);
   return ql::launch_gemm_fwd(w, X, M, U, B, r, s, Y, y_dt, cs);
 }
 
@@ -211,7 +225,7 @@ ql_status qlora_silu_gate_bwd(const void* dh, const void* g, const void* u, void
 size_t qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r) {
   switch (op) {
     case QL_OP_DOUBLE_QUANT: return M > 0 ? ql::dq_workspace_bytes(M) : 0;
-    case QL_OP_FWD: return ws_fwd(M, K, r);
+    case QL_OP_FWD: return ws_fwd(M, N, K, r);
     case QL_OP_BWD: return ws_bwd(M, N, K, r);
     default: return 0;
   }

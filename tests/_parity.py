@@ -11,7 +11,9 @@ REL_FRO = 2e-3
 MAX_ABS_RMS = 1e-2
 
 
-def np64(t: torch.Tensor) -> np.ndarray:
+def np64(t) -> np.ndarray:
+    if isinstance(t, np.ndarray):
+        return t.astype(np.float64)
     return t.detach().to("cpu", torch.float64).numpy()
 
 
@@ -64,3 +66,29 @@ def assert_bf16_within_ulp(got_bf16: torch.Tensor, ref64, what="", ulps=1, abs_r
         gv = F.bf16_from_bits(bf16_bits_t(got_bf16)).reshape(ref.shape)
         bad &= np.abs(gv - ref) > abs_rms * rms
     assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond {ulps} bf16 ulp (max {d.max()})"
+
+
+def adjoint_bound(s, U, V, *pairs):
+    """Allowed |<a1, b1> - <a2, b2>| for identities that hold exactly in real
+    arithmetic but whose two sides each use one independently rounded bf16
+    copy of U = X A^T or V = dY B (relative rounding <= 2^-8 per element):
+    s * 2^-7 * sum|U||V|, plus 1e-5 * sum|a||b| for fp32 accumulation."""
+    U, V = np.abs(np.asarray(U, dtype=np.float64)), np.abs(np.asarray(V, dtype=np.float64))
+    acc = sum(float(np.abs(a * b).sum()) for a, b in pairs)
+    return abs(s) * 2.0 ** -7 * float((U * V).sum()) + 1e-5 * acc
+
+
+def assert_chain_close(got, ref, bound, what="", rel_fro=REL_FRO):
+    """An output that sits after bf16 intermediates each side rounds on its own
+    (the MLP chain's g, u, h, dh, dg, du): relative Frobenius error within
+    rel_fro, and every element within `bound`, the most a one-ulp difference
+    in every bf16 intermediate can move it (2^-7 |intermediate| |weight|
+    summed, computed from the oracle's values) plus 1e-5 rms."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.all(np.isfinite(got)), what
+    rf = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rf <= rel_fro, f"{what}: rel Frobenius {rf:.3e}"
+    rms = np.sqrt(np.mean(ref ** 2))
+    excess = np.abs(got - ref) - (bound + 1e-5 * rms)
+    assert excess.max() <= 0, f"{what}: {int((excess > 0).sum())} elements beyond the flip bound"
