@@ -27,10 +27,10 @@
 // Warp roles (576 threads):
 //   warp 0      TMA producer
 //   warp 1      TMEM allocation; one thread issues tcgen05.mma
-//   warps 2-17  dequant producers: threads pair up on one 64-block of codes
-//               (32 codes each) and expand it through a per-block register
-//               lookup table into the swizzled BF16 weight tile; then the LoRA
-//               operands; then they drain the accumulators to global memory.
+//   warps 2-17  dequant producers, two groups of 8 warps on alternate stages;
+//               each thread expands one 64-block of codes through a per-block
+//               register lookup table into the swizzled BF16 weight tile; then
+//               the LoRA operands; then all 16 warps drain the accumulators.
 // The weight tile holds W rows as 128-byte rows in both directions: K-major
 // for the forward (rows = output features), MN-major for the backward (rows =
 // the reduction index), so the producers write the same layout either way.
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sm.empty_t[i], 1);
     }
     for (int i = 0; i < B_STAGES; ++i) {
-      mbar_init(&sm.full_b[i], PRODUCER_WARPS);
+      mbar_init(&sm.full_b[i], PRODUCER_WARPS / 2);
       mbar_init(&sm.empty_b[i], 1);
     }
     mbar_init(sm.acc_full, 1);
@@ -256,39 +256,52 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------ dequant producers
-    // Each producer warp covers 16 weight rows: lanes 0-7 / 8-15 take the two
-    // halves of rows 0-7, lanes 16-23 / 24-31 those of rows 8-15, so every
-    // quarter-warp touches 8 different rows and the swizzled shared-memory
-    // accesses below are free of bank conflicts.
-    const int wp = warp - 2;                                   // 0..15
-    const int pt = threadIdx.x - 64;                           // 0..511
-    const int half = (lane >> 3) & 1;                          // which 32 codes of the 64-block
-    const int row_local = (lane & 7) + 8 * (lane >> 4);        // 0..15
-    const int kblocks = p.K / 64;                              // 64-blocks per weight row
+    // Two groups of 8 warps take alternate stages (group g expands stages
+    // g, g+2, ...), so each group has two stage times for its work and every
+    // thread expands one whole 64-block (one lookup table per block).
+    // fwd: thread t of the group owns weight row t of the 256-row tile;
+    // bwd: thread t owns weight row t % 64 of the 64-row stage and the
+    // 64-column chunk t / 64.  Consecutive lanes take consecutive rows, so the
+    // swizzled shared-memory accesses below are free of bank conflicts.
+    const int wp = warp - 2;                 // 0..15
+    const int grp = wp >> 3;                 // producer group
+    const int gt = ((wp & 7) << 5) | lane;   // thread within the group, 0..255
+    const int kblocks = p.K / 64;            // 64-blocks per weight row
     const float mu = p.wc.absmax ? 0.0f : *p.wc.offset;
     int row_in_tile, col_chunk;
-    if (!BWD) { row_in_tile = 16 * wp + row_local; col_chunk = 0; }
-    else { row_in_tile = 16 * (wp & 3) + row_local; col_chunk = wp >> 2; }
-    // byte offset of this thread's 16-byte code chunk in the swizzled code tile
-    uint32_t coff;
-    if (!BWD) coff = row_in_tile * 32 + ((half ^ ((row_in_tile >> 2) & 1)) << 4);          // 32B swizzle
-    else coff = row_in_tile * 128 + (((2 * col_chunk + half) ^ (row_in_tile & 7)) << 4);   // 128B swizzle
+    if (!BWD) { row_in_tile = gt; col_chunk = 0; }
+    else { row_in_tile = gt & 63; col_chunk = gt >> 6; }
+    // byte offsets of this thread's two 16-byte code chunks in the swizzled code tile
+    uint32_t coff0, coff1;
+    if (!BWD) {   // 32-byte rows, 32B swizzle: chunk ^= bit 2 of the row
+      const uint32_t x = (row_in_tile >> 2) & 1;
+      coff0 = row_in_tile * 32 + ((0 ^ x) << 4);
+      coff1 = row_in_tile * 32 + ((1 ^ x) << 4);
+    } else {      // 128-byte rows, 128B swizzle: chunk ^= row mod 8
+      const uint32_t x = row_in_tile & 7;
+      coff0 = row_in_tile * 128 + (((2 * col_chunk) ^ x) << 4);
+      coff1 = row_in_tile * 128 + (((2 * col_chunk + 1) ^ x) << 4);
+    }
+    // byte offsets of the 8 16-byte chunks this thread writes in a weight tile
+    uint32_t boff[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) boff[j] = (BWD ? col_chunk * 8192 : 0) + sw128_offset(row_in_tile, j);
     auto step_row = [&](int i, int& wrow, int& kb) {
       if (!BWD) { wrow = j0 + row_in_tile; kb = i; }
       else { wrow = i * BK + row_in_tile; kb = j0 / 64 + col_chunk; }
     };
     int wrow, kb;
-    step_row(0, wrow, kb);
-    bool valid = wrow < p.N && kb < kblocks;
+    step_row(grp, wrow, kb);
+    bool valid = grp < p.n_steps && wrow < p.N && kb < kblocks;
     RawConst next = load_const(p.wc, (int64_t)wrow * kblocks + kb, valid);
     bool ok = true;
-    for (int i = 0; i < p.n_steps && ok; ++i) {
+    for (int i = grp; i < p.n_steps && ok; i += 2) {
       const int s = i % T_STAGES, use = i / T_STAGES;
       const int sb = i % B_STAGES, useb = i / B_STAGES;
       const RawConst cur = next;
       const bool cur_valid = valid;
-      if (i + 1 < p.n_steps) {   // constants of the next stage, one stage ahead
-        step_row(i + 1, wrow, kb);
+      if (i + 2 < p.n_steps) {   // constants of this group's next stage
+        step_row(i + 2, wrow, kb);
         valid = wrow < p.N && kb < kblocks;
         next = load_const(p.wc, (int64_t)wrow * kblocks + kb, valid);
       }
@@ -296,24 +309,26 @@ __global__ void __launch_bounds__(THREADS, 1)
                                        (useb == 0 || mbar_wait(&sm.empty_b[sb], (useb - 1) & 1, abort_flag,
                                                                p.wait_limit)));
       if (!ok) break;
-      uint8_t* base = sm.b(sb) + (BWD ? col_chunk * 8192 : 0);
+      uint8_t* base = sm.b(sb);
       if (cur_valid) {
-        const uint4 c0 = *reinterpret_cast<const uint4*>(sm.c(s) + coff);
-        const uint32_t w[4] = {c0.x, c0.y, c0.z, c0.w};
+        const uint4 c0 = *reinterpret_cast<const uint4*>(sm.c(s) + coff0);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(sm.c(s) + coff1);
+        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         const Lut16 L = make_lut(p.tab, decode_const(p.wc, cur, mu));
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(base + sw128_offset(row_in_tile, 4 * half + j)) = lut_lookup8(L, w[j]);
+        for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(base + boff[j]) = lut_lookup8(L, w[j]);
       } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(base + sw128_offset(row_in_tile, 4 * half + j)) = zero4();
+        for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(base + boff[j]) = zero4();
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.full_b[sb]);
     }
-    // LoRA operands into the slots after the last main step
-    if (ok && lora) {
+    const int pt = gt;   // LoRA operand writers below: the group of the step after the last
+    // LoRA operands into the slots after the last main step, written by the
+    // group whose turn that step is
+    if (ok && lora && grp == (p.n_steps & 1)) {
       const int i = p.n_steps;
       const int s = i % T_STAGES, use = i / T_STAGES;
       const int sb = i % B_STAGES, useb = i / B_STAGES;
@@ -323,10 +338,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ok) {
         // A operand: U or V rows m0 .. m0+255, K-major (256 rows x rp)
         {
-          const int row = pt >> 1, hh = pt & 1;
+          const int row = pt;   // 256 threads, one token row each
           const int m = m0 + row;
-          for (int q = 0; q < 4; ++q) {
-            const int chunk = hh * 4 + q;
+          for (int chunk = 0; chunk < 8; ++chunk) {
             const int e = chunk * 8;
             if (e >= p.rp) break;
             uint4 v = zero4();
@@ -336,10 +350,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (!BWD) {
           // B operand: (s B)[n, 0..rp) for the 256 output features, K-major
-          const int rr = pt >> 1, hh = pt & 1;
+          const int rr = pt;
           const int n = j0 + rr;
-          for (int q = 0; q < 4; ++q) {
-            const int chunk = hh * 4 + q;
+          for (int chunk = 0; chunk < 8; ++chunk) {
             const int e = chunk * 8;
             if (e >= p.rp) break;
             uint4 v = zero4();
@@ -348,7 +361,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         } else {
           // B operand: (s A)[0..rp, k] for the 256 output columns, MN-major
-          for (int idx = pt; idx < p.rp * 32; idx += PRODUCER_WARPS * 32) {
+          for (int idx = pt; idx < p.rp * 32; idx += 256) {
             const int jr = idx >> 5, rem = idx & 31;
             const int cc = rem >> 3, piece = rem & 7;
             const int k = j0 + cc * 64 + piece * 8;
