@@ -20,13 +20,12 @@ ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, con
                           float s, void* dX, ql_dtype dx_dt, int accumulate, cudaStream_t st);
 unsigned status_word_gemm(cudaStream_t st);
 // lora_tc.cu
-size_t skinny_partial_bytes(int64_t rows, int64_t red, int r);
 ql_status launch_proj(const void* Z, int64_t M, int64_t red, const void* Gt, int64_t ld_gt, int r, void* out,
-                      float* partial, cudaStream_t st);
+                      void* out_t, int64_t ld_t, cudaStream_t st);
 ql_status launch_grad_b(const void* dY, int64_t M, int N, const void* Ut, int64_t ld_ut, int r, float s, void* dB,
-                        ql_dtype dt, float* partial, cudaStream_t st);
+                        ql_dtype dt, cudaStream_t st);
 ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t ld_vt, int r, float s, void* dA,
-                        ql_dtype dt, float* partial, cudaStream_t st);
+                        ql_dtype dt, cudaStream_t st);
 ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st);
 // smallm.cu
 size_t smallm_partial_bytes(int64_t N, int64_t K);
@@ -71,20 +70,17 @@ ql_status check_gemm_shape(const ql_nf4_weight* w, int64_t M, int r) {
 // Tokens up to this count take the small-M (HBM-bound) forward kernel.
 constexpr int64_t kSmallM = 16;
 
-// Forward workspace: U [M, r] (when U_out is not given), then fp32 split-K
-// partials shared by the U projection and, for M <= 16, the small-M kernel.
+// Forward workspace: U [M, r] (when U_out is not given), then, for M <= 16,
+// the small-M kernel's fp32 split-K partials.
 size_t ws_fwd(int64_t M, int64_t N, int64_t K, int r) {
-  size_t part = r > 0 ? ql::skinny_partial_bytes(M, K, r) : 0;
-  if (M <= kSmallM) part = std::max(part, ql::smallm_partial_bytes(N, K));
-  if (part == 0) return 0;
+  const size_t part = M <= kSmallM ? ql::smallm_partial_bytes(N, K) : 0;
   return align256((size_t)M * r * 2) + align256(part);
 }
 
 // Backward workspace, carved in this order (each piece 256-byte aligned):
-//   B^T [r, N], U^T [r, Mp], U [M, r] (recomputed only when not given),
-//   V [M, r], V^T [r, Mp], fp32 split-K partials.   Mp = M rounded up to 8.
+//   B^T [r, N], U^T [r, Mp], V [M, r], V^T [r, Mp].   Mp = M rounded up to 8.
 struct BwdWs {
-  size_t bt, ut, u, v, vt, part, total;
+  size_t bt, ut, v, vt, total;
 };
 
 BwdWs ws_bwd_layout(int64_t M, int64_t N, int64_t K, int r) {
@@ -94,14 +90,8 @@ BwdWs ws_bwd_layout(int64_t M, int64_t N, int64_t K, int r) {
   size_t off = 0;
   w.bt = off; off += align256((size_t)r * N * 2);
   w.ut = off; off += align256((size_t)r * Mp * 2);
-  w.u = off;  off += align256((size_t)M * r * 2);
   w.v = off;  off += align256((size_t)M * r * 2);
   w.vt = off; off += align256((size_t)r * Mp * 2);
-  size_t part = ql::skinny_partial_bytes(N, M, r);
-  part = std::max(part, ql::skinny_partial_bytes(K, M, r));
-  part = std::max(part, ql::skinny_partial_bytes(M, K, r));
-  part = std::max(part, ql::skinny_partial_bytes(M, N, r));
-  w.part = off; off += align256(part);
   w.total = off;
   return w;
 }
@@ -152,7 +142,7 @@ ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, con
   void* U = U_out ? U_out : wp;
   float* partial = reinterpret_cast<float*>(wp + align256((size_t)M * r * 2));
   if (r > 0) {
-    st = ql::launch_proj(X, M, K, A, K, r, U, partial, cs);                 // U = bf16(X A^T)
+    st = ql::launch_proj(X, M, K, A, K, r, U, nullptr, 0, cs);    // U = bf16(X A^T)
     if (st != QL_OK) return st;
   }
   if (small) return ql::launch_smallm_fwd(w, X, M, U, B, r, s, Y, y_dt, partial, cs);
@@ -189,25 +179,21 @@ ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY
   void* Ut = wp + L.ut;
   void* V = wp + L.v;
   void* Vt = wp + L.vt;
-  float* partial = reinterpret_cast<float*>(wp + L.part);
   st = ql::launch_transpose(B, N, r, Bt, N, cs);                              // B^T [r, N]
   if (st != QL_OK) return st;
   if (!U) {
-    st = ql::launch_proj(X, M, K, A, K, r, wp + L.u, partial, cs);            // U = bf16(X A^T)
-    if (st != QL_OK) return st;
-    U = wp + L.u;
+    st = ql::launch_proj(X, M, K, A, K, r, nullptr, Ut, Mp, cs);     // U^T = bf16(X A^T)^T
+  } else {
+    st = ql::launch_transpose(U, M, r, Ut, Mp, cs);                          // U^T [r, Mp]
   }
-  st = ql::launch_proj(dY, M, N, Bt, N, r, V, partial, cs);                  // V = bf16(dY B)
   if (st != QL_OK) return st;
-  st = ql::launch_transpose(U, M, r, Ut, Mp, cs);                            // U^T [r, Mp]
-  if (st != QL_OK) return st;
-  st = ql::launch_transpose(V, M, r, Vt, Mp, cs);                            // V^T [r, Mp]
+  st = ql::launch_proj(dY, M, N, Bt, N, r, V, Vt, Mp, cs);          // V = bf16(dY B), and V^T
   if (st != QL_OK) return st;
   st = ql::launch_gemm_bwd(w, dY, M, V, A, r, s, dX, dx_dt, accumulate_dx, cs);  // dX
   if (st != QL_OK) return st;
-  st = ql::launch_grad_b(dY, M, (int)N, Ut, Mp, r, s, dB, grad_dt, partial, cs);  // dB = s dY^T U
+  st = ql::launch_grad_b(dY, M, (int)N, Ut, Mp, r, s, dB, grad_dt, cs);  // dB = s dY^T U
   if (st != QL_OK) return st;
-  return ql::launch_grad_a(X, M, (int)K, Vt, Mp, r, s, dA, grad_dt, partial, cs);   // dA = s V^T X
+  return ql::launch_grad_a(X, M, (int)K, Vt, Mp, r, s, dA, grad_dt, cs);   // dA = s V^T X
 }
 
 ql_status qlora_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, void* stream) {

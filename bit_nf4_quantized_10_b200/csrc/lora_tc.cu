@@ -6,8 +6,10 @@
 //
 // All three are skinny products C[rows x r] = Z_op[rows x red] * G[red x r]
 // with r <= 64: tcgen05.mma with M = 128 output rows and N = r (padded to 16),
-// the long reduction split over CTAs (split-K), fp32 partials in the caller's
-// workspace, then a reduction over the splits in fixed order (deterministic).
+// the long reduction split over up to 8 CTAs (split-K) that form one
+// thread-block cluster per row tile; the fp32 partials are summed across the
+// cluster's shared memory in split order (deterministic), and the result is
+// written row-major and/or transposed.
 //   dB: Z_op = dY^T (MN-major view of dY [M, N]), G^T = U^T [r, M]
 //   dA: Z_op = X^T  (MN-major view of X  [M, K]), G^T = V^T [r, M]
 //   U:  Z_op = X    (K-major),                     G^T = A   [r, K]
@@ -39,14 +41,47 @@ constexpr int THREADS = 6 * 32;        // TMA, MMA, 4 drain warps
 constexpr int TMEM_COLS = 64;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
 
+constexpr int MAX_SPLITS = 8;           // portable cluster size
+
 struct Params {
   int rows;             // output rows (M of the MMA)
-  int rp;               // r padded to 16
+  int r, rp;            // rank, padded to 16
   int steps_total;      // ceil(red / 64)
   int steps_per_split;
-  float* partial;       // [splits][rows][rp]
+  float scale;
+  void* out_row;        // [rows, r] of row_bf16 ? bf16 : fp32, or NULL
+  int row_bf16;
+  void* out_t;          // [r, ld_t] of t_bf16 ? bf16 : fp32, or NULL
+  int ld_t;
+  int t_bf16;
   uint32_t wait_limit;
 };
+
+// Final value of output row `row`, columns j .. j+3, written to both layouts.
+__device__ __forceinline__ void store_out4(const Params& p, int row, int j, float4 v) {
+  v.x = __fmul_rn(p.scale, v.x);
+  v.y = __fmul_rn(p.scale, v.y);
+  v.z = __fmul_rn(p.scale, v.z);
+  v.w = __fmul_rn(p.scale, v.w);
+  if (p.out_row) {
+    if (p.row_bf16) {
+      uint2 pk;
+      pk.x = pack_bf16x2(v.x, v.y);
+      pk.y = pack_bf16x2(v.z, v.w);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out_row) + (size_t)row * p.r + j) = pk;
+    } else {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out_row) + (size_t)row * p.r + j) = v;
+    }
+  }
+  if (p.out_t) {
+    const float f[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (p.t_bf16) reinterpret_cast<__nv_bfloat16*>(p.out_t)[(size_t)(j + q) * p.ld_t + row] = __float2bfloat16_rn(f[q]);
+      else reinterpret_cast<float*>(p.out_t)[(size_t)(j + q) * p.ld_t + row] = f[q];
+    }
+  }
+}
 
 template <bool A_MN>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -126,51 +161,66 @@ __global__ void __launch_bounds__(THREADS, 1)
       mma_commit(acc_full);
     }
   } else {
+    // drain (warps 2-5): this CTA's fp32 partial of its 128 rows into shared
+    // memory (the stage buffers are idle once the last MMA has completed);
+    // row stride rp + 4 floats keeps the 16-byte accesses conflict-free
     const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.wait_limit) && !*abort_flag);
-    if (ok) {
-      tc_fence_after();
-      const int quad = warp & 3;
-      const int row = row0 + quad * 32 + lane;
-      for (int c16 = 0; c16 < p.rp / 16; ++c16) {
-        uint32_t v[16];
+    const int quad = warp & 3;
+    const int lrow = quad * 32 + lane;
+    float* red = reinterpret_cast<float*>(base);
+    if (ok) tc_fence_after();
+    for (int c16 = 0; c16 < p.rp / 16; ++c16) {
+      uint32_t v[16];
+      if (ok) {
         tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(c16 * 16), v);
         tmem_ld_wait();
-        if (row < p.rows) {
-          float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)blockIdx.y * p.rows + row) * p.rp + c16 * 16);
+      } else {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
-                                 __uint_as_float(v[4 * q + 3]));
-        }
+        for (int q = 0; q < 16; ++q) v[q] = 0u;
       }
+      float4* dst = reinterpret_cast<float4*>(red + lrow * (p.rp + 4) + c16 * 16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                             __uint_as_float(v[4 * q + 3]));
     }
   }
   if (warp == 1 && lane == 0 && *abort_flag) mbar_wait(acc_full, 0, abort_flag, p.wait_limit);
+
+  // The CTAs of one row tile (one per split of the reduction) form a cluster.
+  // After every partial is in shared memory, CTA k of the cluster sums 1/splits
+  // of the tile's (row, 4 columns) items over all CTAs of the cluster in split
+  // order (so the result does not depend on scheduling) and writes them.
+  cluster_sync();
+  {
+    const int splits = (int)gridDim.y;
+    const int rank = (int)cluster_rank();
+    const int c4s = p.rp / 4;
+    const int items = BM * c4s;
+    const int i0 = (int)((int64_t)items * rank / splits), i1 = (int)((int64_t)items * (rank + 1) / splits);
+    const uint32_t red_base = smem_u32(base);
+    for (int it = i0 + (int)threadIdx.x; it < i1; it += THREADS) {
+      const int c4 = it / BM, lrow = it % BM;     // rows fastest: coalesced transposed stores
+      const int row = row0 + lrow, j = c4 * 4;
+      if (row >= p.rows || j >= p.r) continue;
+      const uint32_t off = red_base + (uint32_t)((lrow * (p.rp + 4) + j) * 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < splits; ++sp) {
+        const float4 x = ld_cluster_f4(cluster_map(off, (uint32_t)sp));
+        acc.x = __fadd_rn(acc.x, x.x);
+        acc.y = __fadd_rn(acc.y, x.y);
+        acc.z = __fadd_rn(acc.z, x.z);
+        acc.w = __fadd_rn(acc.w, x.w);
+      }
+      store_out4(p, row, j, acc);
+    }
+  }
+  cluster_sync();   // no CTA leaves while another still reads its shared memory
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
-  }
-}
-
-// out = scale * sum over splits of partial, in split order.
-// transpose = 0: out [rows, r] (row-major); 1: out [r, rows].
-__global__ void __launch_bounds__(256) reduce_kernel(const float* __restrict__ partial, int splits, int rows, int rp,
-                                                     int r, float scale, int transpose, int out_bf16,
-                                                     void* __restrict__ out) {
-  const int64_t total = (int64_t)rows * r;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    int64_t row, j;
-    if (transpose) { j = idx / rows; row = idx % rows; }   // coalesced writes along rows
-    else { row = idx / r; j = idx % r; }
-    float acc = 0.0f;
-    for (int s = 0; s < splits; ++s) acc = __fadd_rn(acc, partial[((int64_t)s * rows + row) * rp + j]);
-    const float v = __fmul_rn(scale, acc);
-    const int64_t o = transpose ? j * rows + row : row * r + j;
-    if (out_bf16) reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v);
-    else reinterpret_cast<float*>(out)[o] = v;
   }
 }
 
@@ -198,28 +248,24 @@ static int sm_count_tc() {
   return count;
 }
 
+// One wave of CTAs (two per SM) where the row tiles allow, at most
+// MAX_SPLITS CTAs per tile (one cluster), each split a whole number of steps.
 static void split_plan(int rows, int64_t red, int& splits, int& per) {
   const int tiles = (rows + skinny::BM - 1) / skinny::BM;
   const int steps = (int)((red + skinny::BK - 1) / skinny::BK);
-  int want = (2 * sm_count_tc() + tiles - 1) / tiles;
-  want = std::max(1, std::min(want, steps));
+  int want = 2 * sm_count_tc() / tiles;
+  want = std::max(1, std::min(std::min(want, steps), skinny::MAX_SPLITS));
   per = (steps + want - 1) / want;
   splits = (steps + per - 1) / per;
 }
 
-size_t skinny_partial_bytes(int64_t rows, int64_t red, int r) {
-  int splits, per;
-  split_plan((int)rows, red, splits, per);
-  const int rp = (r + 15) / 16 * 16;
-  return (size_t)splits * rows * rp * sizeof(float);
-}
-
 // C = scale * Z_op G, see the file comment.  a_mn: Z_op is the transpose of a
 // row-major [red, rows] array z (ld = rows); else Z_op = z, [rows, red].
-// gt: G^T, row-major [r, red] with row pitch ld_gt.
+// gt: G^T, row-major [r, red] with row pitch ld_gt.  C is written row-major
+// to out_row [rows, r] and/or transposed to out_t [r, ld_t].
 static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, const void* gt, int r, int64_t ld_gt,
-                               float scale, int transpose, void* out, ql_dtype out_dt, float* partial, int kind,
-                               cudaStream_t st) {
+                               float scale, void* out_row, ql_dtype row_dt, void* out_t, int64_t ld_t, ql_dtype t_dt,
+                               int kind, cudaStream_t st) {
   using namespace skinny;
   static bool attr[2] = {false, false};
   if (!attr[a_mn]) {
@@ -243,46 +289,57 @@ static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, 
     return QL_ERR_CUDA;
   int splits, per;
   split_plan(rows, red, splits, per);
+  const int tiles = (rows + BM - 1) / BM;
   Params p;
   p.rows = rows;
+  p.r = r;
   p.rp = rp;
   p.steps_total = (int)((red + BK - 1) / BK);
   p.steps_per_split = per;
-  p.partial = partial;
+  p.scale = scale;
+  p.out_row = out_row;
+  p.row_bf16 = row_dt == QL_BF16;
+  p.out_t = out_t;
+  p.ld_t = (int)ld_t;
+  p.t_bf16 = t_dt == QL_BF16;
   p.wait_limit = 1u << 22;
-  dim3 grid((unsigned)((rows + BM - 1) / BM), (unsigned)splits);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr_c[1];
+  attr_c[0].id = cudaLaunchAttributeClusterDimension;
+  attr_c[0].val.clusterDim.x = 1;
+  attr_c[0].val.clusterDim.y = (unsigned)splits;
+  attr_c[0].val.clusterDim.z = 1;
+  cfg.attrs = attr_c;
+  cfg.numAttrs = 1;
   {
     TraceScope ts(kind, st);
-    if (a_mn) skinny_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, p);
-    else skinny_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, p);
+    if (a_mn) QL_CUDA_TRY(cudaLaunchKernelEx(&cfg, skinny_kernel<true>, ma, mb, p));
+    else QL_CUDA_TRY(cudaLaunchKernelEx(&cfg, skinny_kernel<false>, ma, mb, p));
   }
-  QL_LAUNCH_CHECK();
-  const int64_t total = (int64_t)rows * r;
-  const unsigned rg = (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count_tc() * 8);
-  {
-    TraceScope ts(TK_COLACC_REDUCE, st);
-    reduce_kernel<<<rg, 256, 0, st>>>(partial, splits, rows, rp, r, scale, transpose, out_dt == QL_BF16, out);
-  }
-  QL_LAUNCH_CHECK();
   return QL_OK;
 }
 
-// side = bf16(Z G): Z [M, red] (X or dY), G^T [r, ld_gt] (A or B^T); out [M, r]
+// side = bf16(Z G): Z [M, red] (X or dY), G^T [r, ld_gt] (A or B^T);
+// out [M, r] and/or out_t [r, ld_t], both bf16
 ql_status launch_proj(const void* Z, int64_t M, int64_t red, const void* Gt, int64_t ld_gt, int r, void* out,
-                      float* partial, cudaStream_t st) {
-  return skinny_launch(false, Z, (int)M, red, Gt, r, ld_gt, 1.0f, 0, out, QL_BF16, partial, TK_PROJ, st);
+                      void* out_t, int64_t ld_t, cudaStream_t st) {
+  return skinny_launch(false, Z, (int)M, red, Gt, r, ld_gt, 1.0f, out, QL_BF16, out_t, ld_t, QL_BF16, TK_PROJ, st);
 }
 
-// dB = s dY^T U: dY [M, N], U^T [r, ld_ut]
+// dB = s dY^T U: dY [M, N], U^T [r, ld_ut]; dB [N, r]
 ql_status launch_grad_b(const void* dY, int64_t M, int N, const void* Ut, int64_t ld_ut, int r, float s, void* dB,
-                        ql_dtype dt, float* partial, cudaStream_t st) {
-  return skinny_launch(true, dY, N, M, Ut, r, ld_ut, s, 0, dB, dt, partial, TK_COLACC, st);
+                        ql_dtype dt, cudaStream_t st) {
+  return skinny_launch(true, dY, N, M, Ut, r, ld_ut, s, dB, dt, nullptr, 0, dt, TK_COLACC, st);
 }
 
-// dA = s V^T X: X [M, K], V^T [r, ld_vt]; written as [r, K]
+// dA = s V^T X: X [M, K], V^T [r, ld_vt]; dA [r, K]
 ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t ld_vt, int r, float s, void* dA,
-                        ql_dtype dt, float* partial, cudaStream_t st) {
-  return skinny_launch(true, X, K, M, Vt, r, ld_vt, s, 1, dA, dt, partial, TK_COLACC, st);
+                        ql_dtype dt, cudaStream_t st) {
+  return skinny_launch(true, X, K, M, Vt, r, ld_vt, s, nullptr, dt, dA, K, dt, TK_COLACC, st);
 }
 
 // dst [cols, ld_dst] = src [rows, cols]^T, bf16
