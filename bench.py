@@ -40,6 +40,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-secondary", action="store_true", help="skip the small-M and codec side measurements")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--leg", choices=["projection", "smallm", "codec"], default="projection",
+                   help="with --profile: which workload to run (the bench line is the projection step)")
     p.add_argument("--profile", action="store_true",
                    help="fixed launch sequence for profilers: exactly --warmup then --steps steps, "
                         "no clock-sampling warm-up, no e2e, secondary or CPU legs")
@@ -56,6 +58,28 @@ def peaks():
         return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
     except Exception:
         return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def config(world: int) -> dict:
+    return {"workload": "projection 4096x4096 NF4+DQ, 4096 tokens/GPU, r=16, alpha=32: quantize + "
+                        "double quant + fwd + bwd (dX, dA, dB)",
+            "global_batch": 4096 * world, "N": 4096, "K": 4096, "r": 16,
+            "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, untimed)",
+            "outputs": "Y, dX bf16; dA, dB fp32"}
+
+
+def gemm_traffic():
+    """DRAM bytes per launch of the fused GEMM from the committed ncu summary,
+    or None when the kernel source has changed since it was captured."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            d = json.load(f)["qlora_gemm_kernel"]
+        with open(os.path.join(ROOT, "bit_nf4_quantized_10_b200", "csrc", "gemm.cu"), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        return float(d["dram_bytes_per_launch"]) if d["gemm_cu_sha256"] == sha else None
+    except Exception:
+        return None
 
 
 # ------------------------------------------------------------------ clocks
@@ -183,6 +207,9 @@ def trace_enable(q, on):
 
 
 # --------------------------------------------------------------- CPU oracle
+_ORACLE_INPUTS = {}
+
+
 def cpu_oracle_sample(rows: int = 256, tokens: int = 256):
     """The oracle on a bounded sample of the projection step: quantize + double
     quant + dequant of `rows` weight rows, fwd + bwd for `tokens` tokens."""
@@ -190,7 +217,9 @@ def cpu_oracle_sample(rows: int = 256, tokens: int = 256):
     from oracle import lora, nf4
     from synthetic import inputs as S
     w = S.WORKLOADS["c2"]
-    d = S.linear_inputs(w, 0)
+    if "c2" not in _ORACLE_INPUTS:
+        _ORACLE_INPUTS["c2"] = S.linear_inputs(w, 0)
+    d = _ORACLE_INPUTS["c2"]
     W = d["W"][:rows]
     X, dY = d["X"][:tokens], d["dY"][:tokens, :rows]
     A, B = d["A"], d["B"][:rows]
@@ -295,7 +324,7 @@ def run_reference(args, rank):
     total_f, total_t = 0.0, 0.0
     desc = ""
     for _ in range(args.steps):
-        f, t, desc = cpu_oracle_sample(128, 128)
+        f, t, desc = cpu_oracle_sample(1024, 512)
         total_f += f
         total_t += t
     v = total_f / total_t / 1e12
@@ -303,11 +332,60 @@ def run_reference(args, rank):
             "warmup": args.warmup, "ms_per_step": total_t / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": "projection 4096x4096, 4096 tokens, r=16, alpha=32, NF4+DQ, fwd+bwd",
-                       "global_batch": 4096, "parallelism": "cpu oracle"},
+            "config": config(1),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def profile_leg(args, q, dev):
+    """A fixed launch sequence of one secondary workload for profilers:
+    smallm = the 16-token forward on the 28672 x 8192 weight; codec = quantize
+    + double quant of 256 Mi bf16 elements.  Prints per-call device times."""
+    import torch
+    from synthetic import inputs as S
+    w5 = S.WORKLOADS["c5"]
+    if args.leg == "smallm":
+        lin = w5.linears[0]
+        N, K, r, s, M = lin.N, lin.K, w5.r, w5.s, 16
+        W = S.normal((N, K), w5.wstd, S.seed_of(5, 0, "W"), device=dev)
+        wq = q.quantize_weight(W, dq=True)
+        del W
+        A = S.uniform((r, K), 1.0 / K ** 0.5, S.seed_of(5, 0, "A"), device=dev)
+        B = S.normal((N, r), 0.01, S.seed_of(5, 0, "B"), device=dev, dtype=torch.bfloat16)
+        X = S.normal((M, K), 1.0, S.seed_of(5, 0, "X") + M, device=dev, dtype=torch.bfloat16)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, q.qlora_workspace_size(q.QL_OP_FWD, M, N, K, r)), dtype=torch.uint8, device=dev)
+        call = lambda: q.qlora_linear_fwd(wq, X, A, B, r, s, Y, ws=ws)
+    else:
+        n = 1 << 28
+        x = S.codec_tensor(n, 0.02, S.seed_of(5, 9, "W"), device=dev)
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+        aq = torch.empty(n // 64, dtype=torch.uint8, device=dev)
+        s2 = torch.empty(-(-n // 64 // 256), dtype=torch.float32, device=dev)
+        mu = torch.empty(1, dtype=torch.float32, device=dev)
+        wsq = torch.empty(q.qlora_workspace_size(q.QL_OP_DOUBLE_QUANT, n // 64), dtype=torch.uint8, device=dev)
+
+        def call():
+            q.nf4_quantize(x, codes, absmax)
+            q.nf4_double_quant(absmax, aq, s2, mu, wsq)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        call()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    st = q.qlora_get_status()
+    if st != q.QL_OK:
+        raise RuntimeError(f"device status: {q.status_string(st)}")
+    print(json.dumps({"leg": args.leg, "us_per_call": [round(t, 2) for t in times]}), flush=True)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -317,6 +395,9 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    if args.profile and args.leg != "projection":
+        profile_leg(args, q, dev)
+        return
     hbm_peak, bf16_peak, bf16_sus, peak_src = peaks()
     wl = Projection(q, dev, rank)
     allreduce = None
@@ -437,15 +518,11 @@ def run_ours(args, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "projection 4096x4096 NF4+DQ, 4096 tokens/GPU, r=16, alpha=32: quantize + "
-                                   "double quant + fwd + bwd (dX, dA, dB)",
-                       "global_batch": 4096 * world, "N": 4096, "K": 4096, "r": 16,
-                       "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, untimed)",
-                       "outputs": "Y, dX bf16; dA, dB fp32"},
+            "config": config(world),
             "roofline": {"bound": "tensor", "kernel": "qlora_gemm (fused NF4 dequant + tcgen05 GEMM + LoRA)",
                          "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
                          "frac": achieved / bf16_peak, "peak_source": f"{peak_src} bf16 burst",
-                         "traffic": None, "launches": gemm_launches,
+                         "traffic": gemm_traffic(), "launches": gemm_launches,
                          "avg_launch_us": gemm_ms / max(gemm_launches, 1) * 1e3},
             "kernels": {k: {"ms_total": round(v[0], 4), "launches": v[1]} for k, v in kern.items()},
             "gpu_launches": gpu_launches,
