@@ -19,18 +19,34 @@ namespace ql {
 QL_DEFINE_STATUS_ACCESSOR(status_word_codec)
 
 // ---------------------------------------------------------------- quantize
-// Code of x: #{j : x > t_j} over the 15 sorted thresholds t_j = fl32(m_j c),
-// found by a 4-step binary search.  The first two steps compare against
-// t_7 and t_3 / t_11 held in registers; the last two read the block's
-// thresholds from shared memory at a data-dependent index (no divergent
-// branches).  Ties (x == t_j) go to the lower level.
-__device__ __forceinline__ uint32_t nf4_code(float x, float t3, float t7, float t11, const float* tb) {
-  uint32_t k = (x > t7) ? 8u : 0u;
-  const float t2 = k ? t11 : t3;
-  k += (x > t2) ? 4u : 0u;
-  k += (x > tb[k + 1]) ? 2u : 0u;
-  k += (x > tb[k]) ? 1u : 0u;
-  return k;
+// Code of x: #{j : x > t_j} over the 15 sorted thresholds t_j = fl32(m_j c)
+// (ties go to the lower level).  The search goes through y = x/c, but only to
+// pick a candidate: the 33 bins round(16 y + 16) are 1/16 wide, narrower than
+// the closest two midpoints (0.093 apart), so each bin (widened by 1e-5 on both
+// sides, far more than the rounding of y) holds at most one threshold j.  The
+// bin table gives j and the count of thresholds below the bin; one exact
+// comparison x > fl32(m_j c) then settles the code.  Bins with no threshold
+// carry m = 4, which no |x| <= c exceeds.
+struct QuantBins {
+  float m[64];
+  uint32_t base[64];
+};
+
+QuantBins build_bins(const NF4Table& t) {
+  QuantBins b{};
+  for (int k = 0; k < 64; ++k) {
+    b.m[k] = 4.0f;
+    b.base[k] = 0;
+    if (k > 32) continue;   // reachable only from a NaN y
+    const double lo = (k - 16.5) / 16.0 - 1e-5, hi = (k - 15.5) / 16.0 + 1e-5;
+    uint32_t below = 0;
+    for (int j = 0; j < 15; ++j) {
+      if ((double)t.m[j] < lo) ++below;
+      else if ((double)t.m[j] <= hi) b.m[k] = t.m[j];
+    }
+    b.base[k] = below;
+  }
+  return b;
 }
 
 template <typename T>
@@ -69,18 +85,20 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* x, int
 
 // 8 threads per 64-block, 8 consecutive elements per thread.  The loop runs
 // over blocks, so the 8 threads of a block always iterate together and can
-// reduce the absmax with shuffles.
+// reduce the absmax with shuffles.  The absmax is the integer maximum of the
+// |x| bit patterns (the same order as the values), which also flags NaN and
+// Inf: their patterns are the largest.
 template <typename T>
 __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, int64_t n,
                                                        uint8_t* __restrict__ codes,
-                                                       float* __restrict__ absmax, NF4Table tab) {
-  // per warp: 4 blocks x 15 thresholds (row pitch 17 spreads the blocks over banks)
-  __shared__ float thr[8][4][17];
+                                                       float* __restrict__ absmax, NF4Table tab, QuantBins bins_in) {
+  __shared__ uint2 bins[64];   // (m bits, count below)
+  if (threadIdx.x < 64) bins[threadIdx.x] = make_uint2(__float_as_uint(bins_in.m[threadIdx.x]), bins_in.base[threadIdx.x]);
+  __syncthreads();
   const int64_t nb = (n + 63) / 64;
   const int lane8 = threadIdx.x & 7;
   const int wib = threadIdx.x >> 5;              // warp in CTA
   const int bq = (threadIdx.x >> 3) & 3;         // block within the warp's four
-  float* tb = thr[wib][bq];
   // the whole warp (4 blocks) iterates together so the shuffles see all lanes
   const int64_t warps_per_grid = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t wb = ((int64_t)blockIdx.x * (blockDim.x >> 5) + wib) * 4; wb < nb; wb += warps_per_grid * 4) {
@@ -88,31 +106,35 @@ __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, 
     const int64_t e0 = b * 64 + lane8 * 8;   // >= n for a block past the end
     float v[8];
     load8<T>(x, e0, n, v);
-    float amax = 0.0f;
-    bool bad = false;
+    uint32_t abits = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float a = fabsf(v[i]);
-      bad |= !(a <= 3.402823466e38f);   // NaN or Inf
-      amax = fmaxf(amax, a);
-    }
-    unsigned anybad = bad ? 1u : 0u;
+    for (int i = 0; i < 8; ++i) abits = max(abits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      anybad |= __shfl_xor_sync(0xffffffffu, anybad, o);
-    }
-    if (anybad && lane8 == 0) raise_status(ST_NONFINITE);
-    const float c = amax;
-    // the block's 15 thresholds: lane8 j writes t_{2j} and t_{2j+1}
-    __syncwarp();
-    tb[2 * lane8] = __fmul_rn(tab.m[2 * lane8], c);
-    if (lane8 < 7) tb[2 * lane8 + 1] = __fmul_rn(tab.m[2 * lane8 + 1], c);
-    const float t3 = __fmul_rn(tab.m[3], c), t7 = __fmul_rn(tab.m[7], c), t11 = __fmul_rn(tab.m[11], c);
-    __syncwarp();
+    for (int o = 1; o < 8; o <<= 1) abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
+    if (abits >= 0x7F800000u && lane8 == 0 && b < nb) raise_status(ST_NONFINITE);
+    const float c = __uint_as_float(abits);
     uint32_t word = 0;
+    if (c >= 1e-30f) {
+      // 16/c: c >= 1e-30 keeps it finite; its rounding moves y by < 1e-6
+      const float s16 = __fmul_rn(16.0f, __frcp_rn(c));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) word |= nf4_code(v[i], t3, t7, t11, tb) << (4 * i);
+      for (int i = 0; i < 8; ++i) {
+        // 1.5 * 2^23 + 16: the sum's low bits are round(16 y + 16), in 0..32
+        const float t = __fmaf_rn(v[i], s16, 12582928.0f);
+        const uint2 e = bins[__float_as_uint(t) & 63u];
+        const float th = __fmul_rn(__uint_as_float(e.x), c);
+        word |= (e.y + (v[i] > th ? 1u : 0u)) << (4 * i);
+      }
+    } else {
+      // tiny (or NaN) absmax: count the thresholds directly
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint32_t k = 0;
+#pragma unroll
+        for (int j = 0; j < 15; ++j) k += (v[i] > __fmul_rn(tab.m[j], c)) ? 1u : 0u;
+        word |= k << (4 * i);
+      }
+    }
     if (c == 0.0f) word = 0x88888888u;
     if (e0 + 8 <= n) {
       __stcs(reinterpret_cast<uint32_t*>(codes + (e0 >> 1)), word);
@@ -278,12 +300,13 @@ ql_status launch_quantize(const void* x, ql_dtype dt, int64_t n, uint8_t* codes,
                           cudaStream_t st) {
   const int64_t nb = (n + 63) / 64;
   const unsigned grid = grid_for(nb, 32, 8);   // 32 blocks (8 warps x 4) per CTA-iteration
+  static const QuantBins bins = build_bins(nf4_table());
   TraceScope ts(TK_QUANTIZE, st);
   if (dt == QL_F32)
-    quantize_kernel<float><<<grid, 256, 0, st>>>((const float*)x, n, codes, absmax, nf4_table());
+    quantize_kernel<float><<<grid, 256, 0, st>>>((const float*)x, n, codes, absmax, nf4_table(), bins);
   else
     quantize_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, n, codes, absmax,
-                                                         nf4_table());
+                                                         nf4_table(), bins);
   QL_LAUNCH_CHECK();
   return QL_OK;
 }

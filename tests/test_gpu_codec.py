@@ -142,3 +142,35 @@ def test_codec_4gi_bf16_sampled(q):
         xb = x[b * 64:(b + 1) * 64].cpu()
         packed, cb, _ = nf4.quantize(xb)
         assert np.array_equal(np_u8(codes_dev[b * 32:(b + 1) * 32]), packed), b
+
+
+def _tie_blocks(dtype):
+    """Blocks whose elements sit exactly on the decision thresholds
+    t_j = fl32(m_j c) and one fp32 step either side, for absmax values from
+    fp32-subnormal to near FLT_MAX (both sides of 1e-30)."""
+    m = nf4.midpoints().astype(np.float32)
+    rng = np.random.default_rng(7)
+    mags = [1e-40, 1e-38, 5e-31, 1e-30, 2e-30, 1e-20, 0.0371, 1.0, 3.0, 1e20, 1e37, 3.3e38]
+    blocks = []
+    for cm in mags:
+        for rep in range(3):
+            c = np.float32(cm * rng.uniform(0.5, 1.0))
+            if dtype == torch.bfloat16:
+                c = np.float32(F.bf16(np.array([c]))[0])
+            x = (rng.uniform(-1, 1, 64) * c).astype(np.float32)
+            x[0], x[1] = c, -c
+            t = (m * c).astype(np.float32)
+            k = 2
+            for tj in t:
+                for v in (tj, np.nextafter(tj, np.float32(np.inf)), np.nextafter(tj, np.float32(-np.inf))):
+                    if k < 64:
+                        x[k] = v
+                        k += 1
+            blocks.append(x)
+    x = torch.from_numpy(np.concatenate(blocks))
+    return x.to(dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_threshold_ties_all_magnitudes(q, dtype):
+    check_all(q, _tie_blocks(dtype))
