@@ -12,25 +12,33 @@
 //   backward dX = dY * W_hat   + V * (s A)        reduction over N (W rows)
 // U = bf16(X A^T) and V = bf16(dY B) come in precomputed (rank-r side kernels).
 //
-// CTA tile: 256 tokens x 256 outputs, 64 reduction elements per stage.  The
-// 256 tokens are two M = 128 tcgen05.mma accumulators (TMEM columns 0-255 and
-// 256-511) that share one dequantized weight tile, so each expanded weight
-// element feeds 512 multiply-adds and every operand byte read from shared
-// memory does twice the work of a 128-token tile.  Shared memory bandwidth is
-// what bounds this kernel: per stage the tensor cores read 2 x (16 + 32) KB,
-// the producers write the 32 KB weight tile and TMA writes 40 KB.
+// Two CTAs on two SMs form a pair (a cluster of 2) that shares one tile of 256
+// output columns: each CTA expands only its half of the weight tile (128
+// output columns), and one thread of the even CTA issues cta_group::2 MMAs
+// (M = 256, N = 256) that read both halves.  Each CTA holds 256 tokens as two
+// M = 128 halves, so a pair instruction pairs the even CTA's half h with the
+// odd CTA's half h, into TMEM columns 0-255 (h = 0) and 256-511 (h = 1) of
+// each CTA.  Per expanded weight element this is 512 multiply-adds on each SM,
+// and each SM's tensor core reads only its own 128 rows of B from its shared
+// memory: half the expansion work and half the operand reads of a single-CTA
+// 256 x 256 tile, which is what bounded the single-CTA form.
 // The r LoRA K-steps (U or V against the scaled adapter) run into the same
 // accumulators after the main loop, before the drain.
 //
-// Shared memory: a TMA ring (activation tile 256 x 64 bf16 + the packed codes
-// of the weight tile) and a ring of dequantized weight tiles, 3 stages each.
-// Warp roles (576 threads):
+// Shared memory per CTA: 4 stages of (activation tile 256 x 64 bf16, the
+// packed codes of the CTA's 128 x 64 weight half, the expanded weight half).
+// Synchronisation: TMA loads complete on the local full_t[s]; each producer
+// warp, in both CTAs, arrives on the even CTA's full_b[s] (8 warps) once its
+// part of the weight tile is written and the CTA's activation tile has landed;
+// the MMA commits multicast to empty[s] and acc_full in both CTAs.
+// Warp roles (576 threads per CTA):
 //   warp 0      TMA producer
-//   warp 1      TMEM allocation; one thread issues tcgen05.mma
-//   warps 2-17  dequant producers, two groups of 8 warps on alternate stages;
-//               each thread expands one 64-block of codes through a per-block
-//               register lookup table into the swizzled BF16 weight tile; then
-//               the LoRA operands; then all 16 warps drain the accumulators.
+//   warp 1      TMEM allocation (both CTAs); one thread of the even CTA
+//               issues the MMAs
+//   warps 2-17  dequant producers, four groups of 4 warps on stages
+//               g, g+4, ...; each thread expands one 64-block through a
+//               per-block register lookup table into the swizzled BF16 tile;
+//               then the LoRA operands; then all 16 warps drain TMEM.
 // The weight tile holds W rows as 128-byte rows in both directions: K-major
 // for the forward (rows = output features), MN-major for the backward (rows =
 // the reduction index), so the producers write the same layout either way.
@@ -45,21 +53,23 @@ using namespace sm100;
 
 namespace gemm {
 
-constexpr int BM = 256;                 // tokens per CTA (two M = 128 accumulators)
+constexpr int BM = 256;                 // tokens per CTA (two M = 128 halves)
 constexpr int BMH = 128;
-constexpr int BN = 256;
+constexpr int BN = 256;                 // output columns per pair
+constexpr int BNH = 128;                // output columns expanded by one CTA
 constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;    // 32 KB activation tile
-constexpr int AH_BYTES = BMH * BK * 2;  // 16 KB: second accumulator's half
-constexpr int B_BYTES = BN * BK * 2;    // 32 KB dequantized weight tile
-constexpr int C_BYTES = BN * BK / 2;    // 8 KB of packed codes
-constexpr int T_STAGES = 3;
-constexpr int B_STAGES = 3;
-constexpr int T_STAGE_BYTES = A_BYTES + C_BYTES;
-constexpr int PRODUCER_WARPS = 16;
+constexpr int AH_BYTES = BMH * BK * 2;  // 16 KB: the second half
+constexpr int B_BYTES = BNH * BK * 2;   // 16 KB expanded weight half
+constexpr int C_BYTES = BNH * BK / 2;   // 4 KB of packed codes
+constexpr int STAGES = 4;
+constexpr int GROUPS = 4;               // producer groups, one stage each in turn
+constexpr int GROUP_WARPS = 4;
+constexpr int PRODUCER_WARPS = GROUPS * GROUP_WARPS;
 constexpr int THREADS = (2 + PRODUCER_WARPS) * 32;
 constexpr int TMEM_COLS = 512;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)T_STAGES * T_STAGE_BYTES + (size_t)B_STAGES * B_BYTES + 256;
+constexpr int T_STAGE_BYTES = A_BYTES + C_BYTES;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * T_STAGE_BYTES + (size_t)STAGES * B_BYTES + 256;
 
 struct Params {
   int M;             // tokens
@@ -82,12 +92,10 @@ struct Smem {
   uint8_t* base;
   __device__ __forceinline__ uint8_t* a(int s) const { return base + s * T_STAGE_BYTES; }
   __device__ __forceinline__ uint8_t* c(int s) const { return base + s * T_STAGE_BYTES + A_BYTES; }
-  __device__ __forceinline__ uint8_t* b(int s) const { return base + T_STAGES * T_STAGE_BYTES + s * B_BYTES; }
-  uint64_t* full_a;    // [T_STAGES] activation tile landed
-  uint64_t* full_c;    // [T_STAGES] codes landed
-  uint64_t* empty_t;   // [T_STAGES] MMA done with the TMA slot
-  uint64_t* full_b;    // [B_STAGES] producers wrote the weight tile
-  uint64_t* empty_b;   // [B_STAGES] MMA done with the weight tile
+  __device__ __forceinline__ uint8_t* b(int s) const { return base + STAGES * T_STAGE_BYTES + s * B_BYTES; }
+  uint64_t* full_t;    // [STAGES] activation tile + codes landed (local TMA)
+  uint64_t* full_b;    // [STAGES] even CTA: both CTAs' weight halves written (8 warps)
+  uint64_t* empty;     // [STAGES] pair MMA done with the stage (commit to both CTAs)
   uint64_t* acc_full;
   uint32_t* tmem_addr;
   int* abort;
@@ -97,14 +105,12 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   Smem s;
   uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.base = p;
-  p += T_STAGES * T_STAGE_BYTES + B_STAGES * B_BYTES;
+  p += STAGES * T_STAGE_BYTES + STAGES * B_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(p);
-  s.full_a = bars;
-  s.full_c = bars + T_STAGES;
-  s.empty_t = bars + 2 * T_STAGES;
-  s.full_b = bars + 3 * T_STAGES;
-  s.empty_b = s.full_b + B_STAGES;
-  s.acc_full = s.empty_b + B_STAGES;
+  s.full_t = bars;
+  s.full_b = bars + STAGES;
+  s.empty = bars + 2 * STAGES;
+  s.acc_full = bars + 3 * STAGES;
   s.tmem_addr = reinterpret_cast<uint32_t*>(s.acc_full + 1);
   s.abort = reinterpret_cast<int*>(s.tmem_addr + 1);
   return s;
@@ -157,20 +163,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   Smem sm = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM;
-  const int j0 = blockIdx.x * BN;   // output-column tile start (W row in fwd, W col in bwd)
+  const uint32_t rank = cluster_rank();          // 0 = even CTA (issues the MMAs)
+  const int j0 = (blockIdx.x >> 1) * BN;         // the pair's output-column tile
+  const int jb = j0 + (int)rank * BNH;           // this CTA's weight half
+  const int m0 = blockIdx.y * (2 * BM) + (int)rank * BM;   // this CTA's 256 tokens
   const bool lora = p.r > 0;
   volatile int* abort_flag = sm.abort;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < T_STAGES; ++i) {
-      mbar_init(&sm.full_a[i], 1);
-      mbar_init(&sm.full_c[i], 1);
-      mbar_init(&sm.empty_t[i], 1);
-    }
-    for (int i = 0; i < B_STAGES; ++i) {
-      mbar_init(&sm.full_b[i], PRODUCER_WARPS / 2);
-      mbar_init(&sm.empty_b[i], 1);
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&sm.full_t[i], 1);
+      mbar_init(&sm.full_b[i], 2 * GROUP_WARPS);
+      mbar_init(&sm.empty[i], 1);
     }
     mbar_init(sm.acc_full, 1);
     *sm.abort = 0;
@@ -181,11 +185,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tmap(&tmap_codes);
   }
   if (warp == 1) {
-    tmem_alloc(sm.tmem_addr, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc2(sm.tmem_addr, TMEM_COLS);
+    tmem_relinquish2();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_addr;
 
@@ -194,122 +198,113 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < p.n_steps; ++i) {
-        const int s = i % T_STAGES, use = i / T_STAGES;
-        if (use > 0 && !mbar_wait(&sm.empty_t[s], (use - 1) & 1, abort_flag, p.wait_limit)) break;
-        mbar_arrive_expect_tx(&sm.full_c[s], C_BYTES);
+        const int s = i % STAGES, use = i / STAGES;
+        if (use > 0 && !mbar_wait(&sm.empty[s], (use - 1) & 1, abort_flag, p.wait_limit)) break;
+        mbar_arrive_expect_tx(&sm.full_t[s], A_BYTES + C_BYTES);
         if (!BWD)
-          tma_load_2d(sm.c(s), &tmap_codes, &sm.full_c[s], i * (BK / 2), j0);
+          tma_load_2d(sm.c(s), &tmap_codes, &sm.full_t[s], i * (BK / 2), jb);
         else
-          tma_load_2d(sm.c(s), &tmap_codes, &sm.full_c[s], j0 / 2, i * BK);
-        mbar_arrive_expect_tx(&sm.full_a[s], A_BYTES);
-        tma_load_2d(sm.a(s), &tmap_act, &sm.full_a[s], i * BK, m0);
+          tma_load_2d(sm.c(s), &tmap_codes, &sm.full_t[s], jb / 2, i * BK);
+        tma_load_2d(sm.a(s), &tmap_act, &sm.full_t[s], i * BK, m0);
         issued = i + 1;
       }
       // before leaving, make sure no copy is still landing in shared memory
-      for (int i = (issued > T_STAGES ? issued - T_STAGES : 0); i < issued; ++i) {
-        const int s = i % T_STAGES, use = i / T_STAGES;
-        mbar_wait(&sm.full_a[s], use & 1, abort_flag, p.wait_limit);
-        mbar_wait(&sm.full_c[s], use & 1, abort_flag, p.wait_limit);
-      }
+      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+        mbar_wait(&sm.full_t[i % STAGES], (i / STAGES) & 1, abort_flag, p.wait_limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16(BMH, BN, false, BWD);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(2 * BMH, BN, false, BWD);
       bool ok = true;
       for (int i = 0; i < p.n_steps && ok; ++i) {
-        const int s = i % T_STAGES, use = i / T_STAGES;
-        const int sb = i % B_STAGES, useb = i / B_STAGES;
-        ok = mbar_wait(&sm.full_a[s], use & 1, abort_flag, p.wait_limit) &&
-             mbar_wait(&sm.full_b[sb], useb & 1, abort_flag, p.wait_limit);
+        const int s = i % STAGES, use = i / STAGES;
+        ok = mbar_wait(&sm.full_t[s], use & 1, abort_flag, p.wait_limit) &&
+             mbar_wait_cluster(&sm.full_b[s], use & 1, abort_flag, p.wait_limit);
         if (!ok) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sm.a(s));
-        const uint32_t b_addr = smem_u32(sm.b(sb));
+        const uint32_t b_addr = smem_u32(sm.b(s));
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t bd = b_desc(b_addr, kk, BWD);
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16(tmem, sdesc_sw128(a_addr + kk * 32, 16, 1024), bd, IDESC, acc);
-          mma_bf16(tmem + 256, sdesc_sw128(a_addr + AH_BYTES + kk * 32, 16, 1024), bd, IDESC, acc);
+          mma_bf16_pair(tmem, sdesc_sw128(a_addr + kk * 32, 16, 1024), bd, IDESC, acc);
+          mma_bf16_pair(tmem + 256, sdesc_sw128(a_addr + AH_BYTES + kk * 32, 16, 1024), bd, IDESC, acc);
         }
-        mma_commit(&sm.empty_t[s]);
-        mma_commit(&sm.empty_b[sb]);
+        mma_commit_pair(&sm.empty[s]);
       }
       if (ok && lora) {
         // LoRA K-steps: A = U or V tile, B = scaled adapter, into both accumulators
         const int i = p.n_steps;
-        const int s = i % T_STAGES, sb = i % B_STAGES, useb = i / B_STAGES;
-        ok = mbar_wait(&sm.full_b[sb], useb & 1, abort_flag, p.wait_limit);
+        const int s = i % STAGES, use = i / STAGES;
+        ok = mbar_wait_cluster(&sm.full_b[s], use & 1, abort_flag, p.wait_limit);
         if (ok) {
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sm.a(s));
-          const uint32_t b_addr = smem_u32(sm.b(sb));
+          const uint32_t b_addr = smem_u32(sm.b(s));
           for (int kk = 0; kk < p.rp / 16; ++kk) {
             const uint64_t bd = b_desc(b_addr, kk, BWD);
-            mma_bf16(tmem, sdesc_sw128(a_addr + kk * 32, 16, 1024), bd, IDESC, 1u);
-            mma_bf16(tmem + 256, sdesc_sw128(a_addr + AH_BYTES + kk * 32, 16, 1024), bd, IDESC, 1u);
+            mma_bf16_pair(tmem, sdesc_sw128(a_addr + kk * 32, 16, 1024), bd, IDESC, 1u);
+            mma_bf16_pair(tmem + 256, sdesc_sw128(a_addr + AH_BYTES + kk * 32, 16, 1024), bd, IDESC, 1u);
           }
         }
       }
-      mma_commit(sm.acc_full);
+      mma_commit_pair(sm.acc_full);
     }
   } else {
     // ------------------------------------------------------ dequant producers
-    // Two groups of 8 warps take alternate stages (group g expands stages
-    // g, g+2, ...), so each group has two stage times for its work and every
-    // thread expands one whole 64-block (one lookup table per block).
-    // fwd: thread t of the group owns weight row t of the 256-row tile;
-    // bwd: thread t owns weight row t % 64 of the 64-row stage and the
-    // 64-column chunk t / 64.  Consecutive lanes take consecutive rows, so the
-    // swizzled shared-memory accesses below are free of bank conflicts.
+    // Group g (4 warps, 128 threads) expands stages g, g+4, ...: thread t owns
+    // one 64-block of the CTA's 128 x 64 weight half.
+    // fwd: thread t owns weight row jb + t (the stage is 64-block i of the row);
+    // bwd: thread t owns weight row i*64 + t % 64 and the 64-column chunk t / 64
+    // of the CTA's 128 columns.  Consecutive lanes take consecutive rows, so the
+    // swizzled shared-memory stores below are free of bank conflicts.
     const int wp = warp - 2;                 // 0..15
-    const int grp = wp >> 3;                 // producer group
-    const int gt = ((wp & 7) << 5) | lane;   // thread within the group, 0..255
+    const int grp = wp / GROUP_WARPS;        // producer group
+    const int gt = ((wp % GROUP_WARPS) << 5) | lane;   // thread within the group, 0..127
     const int kblocks = p.K / 64;            // 64-blocks per weight row
     const float mu = p.wc.absmax ? 0.0f : *p.wc.offset;
     int row_in_tile, col_chunk;
     if (!BWD) { row_in_tile = gt; col_chunk = 0; }
     else { row_in_tile = gt & 63; col_chunk = gt >> 6; }
-    // byte offsets of this thread's two 16-byte code chunks in the swizzled code tile
+    // byte offsets of this thread's two 16-byte code chunks in the code tile
     uint32_t coff0, coff1;
     if (!BWD) {   // 32-byte rows, 32B swizzle: chunk ^= bit 2 of the row
       const uint32_t x = (row_in_tile >> 2) & 1;
       coff0 = row_in_tile * 32 + ((0 ^ x) << 4);
       coff1 = row_in_tile * 32 + ((1 ^ x) << 4);
-    } else {      // 128-byte rows, 128B swizzle: chunk ^= row mod 8
-      const uint32_t x = row_in_tile & 7;
-      coff0 = row_in_tile * 128 + (((2 * col_chunk) ^ x) << 4);
-      coff1 = row_in_tile * 128 + (((2 * col_chunk + 1) ^ x) << 4);
+    } else {      // 64-byte rows (the CTA's 128 columns), no swizzle
+      coff0 = row_in_tile * 64 + col_chunk * 32;
+      coff1 = coff0 + 16;
     }
     // byte offsets of the 8 16-byte chunks this thread writes in a weight tile
     uint32_t boff[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) boff[j] = (BWD ? col_chunk * 8192 : 0) + sw128_offset(row_in_tile, j);
     auto step_row = [&](int i, int& wrow, int& kb) {
-      if (!BWD) { wrow = j0 + row_in_tile; kb = i; }
-      else { wrow = i * BK + row_in_tile; kb = j0 / 64 + col_chunk; }
+      if (!BWD) { wrow = jb + row_in_tile; kb = i; }
+      else { wrow = i * BK + row_in_tile; kb = jb / 64 + col_chunk; }
     };
     int wrow, kb;
     step_row(grp, wrow, kb);
     bool valid = grp < p.n_steps && wrow < p.N && kb < kblocks;
     RawConst next = load_const(p.wc, (int64_t)wrow * kblocks + kb, valid);
     bool ok = true;
-    for (int i = grp; i < p.n_steps && ok; i += 2) {
-      const int s = i % T_STAGES, use = i / T_STAGES;
-      const int sb = i % B_STAGES, useb = i / B_STAGES;
+    for (int i = grp; i < p.n_steps && ok; i += GROUPS) {
+      const int s = i % STAGES, use = i / STAGES;
       const RawConst cur = next;
       const bool cur_valid = valid;
-      if (i + 2 < p.n_steps) {   // constants of this group's next stage
-        step_row(i + 2, wrow, kb);
+      if (i + GROUPS < p.n_steps) {   // constants of this group's next stage
+        step_row(i + GROUPS, wrow, kb);
         valid = wrow < p.N && kb < kblocks;
         next = load_const(p.wc, (int64_t)wrow * kblocks + kb, valid);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.full_c[s], use & 1, abort_flag, p.wait_limit) &&
-                                       (useb == 0 || mbar_wait(&sm.empty_b[sb], (useb - 1) & 1, abort_flag,
-                                                               p.wait_limit)));
+      // the stage's codes and activation tile landed (so the pair MMA is done
+      // with this slot's previous use: the TMA refilled it only after that)
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.full_t[s], use & 1, abort_flag, p.wait_limit));
       if (!ok) break;
-      uint8_t* base = sm.b(sb);
+      uint8_t* base = sm.b(s);
       if (cur_valid) {
         const uint4 c0 = *reinterpret_cast<const uint4*>(sm.c(s) + coff0);
         const uint4 c1 = *reinterpret_cast<const uint4*>(sm.c(s) + coff1);
@@ -323,22 +318,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.full_b[sb]);
+      if (lane == 0) mbar_arrive_cluster(&sm.full_b[s], 0);
     }
-    const int pt = gt;   // LoRA operand writers below: the group of the step after the last
-    // LoRA operands into the slots after the last main step, written by the
+    const int pt = gt;
+    // LoRA operands into the slot after the last main step, written by the
     // group whose turn that step is
-    if (ok && lora && grp == (p.n_steps & 1)) {
+    if (ok && lora && grp == (p.n_steps % GROUPS)) {
       const int i = p.n_steps;
-      const int s = i % T_STAGES, use = i / T_STAGES;
-      const int sb = i % B_STAGES, useb = i / B_STAGES;
-      ok = __all_sync(0xffffffffu, (use == 0 || mbar_wait(&sm.empty_t[s], (use - 1) & 1, abort_flag, p.wait_limit)) &&
-                                       (useb == 0 || mbar_wait(&sm.empty_b[sb], (useb - 1) & 1, abort_flag,
-                                                               p.wait_limit)));
+      const int s = i % STAGES, use = i / STAGES;
+      ok = __all_sync(0xffffffffu, use == 0 || mbar_wait(&sm.empty[s], (use - 1) & 1, abort_flag, p.wait_limit));
       if (ok) {
-        // A operand: U or V rows m0 .. m0+255, K-major (256 rows x rp)
-        {
-          const int row = pt;   // 256 threads, one token row each
+        // A operand: U or V rows m0 .. m0+255, K-major (256 rows x rp), two rows per thread
+        for (int row = pt; row < BM; row += 128) {
           const int m = m0 + row;
           for (int chunk = 0; chunk < 8; ++chunk) {
             const int e = chunk * 8;
@@ -349,30 +340,29 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
         if (!BWD) {
-          // B operand: (s B)[n, 0..rp) for the 256 output features, K-major
-          const int rr = pt;
-          const int n = j0 + rr;
+          // B operand: (s B)[n, 0..rp) for the CTA's 128 output features, K-major
+          const int n = jb + pt;
           for (int chunk = 0; chunk < 8; ++chunk) {
             const int e = chunk * 8;
             if (e >= p.rp) break;
             uint4 v = zero4();
             if (n < p.N && e < p.r) v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)n * p.r + e), p.s);
-            *reinterpret_cast<uint4*>(sm.b(sb) + sw128_offset(rr, chunk)) = v;
+            *reinterpret_cast<uint4*>(sm.b(s) + sw128_offset(pt, chunk)) = v;
           }
         } else {
-          // B operand: (s A)[0..rp, k] for the 256 output columns, MN-major
-          for (int idx = pt; idx < p.rp * 32; idx += 256) {
-            const int jr = idx >> 5, rem = idx & 31;
+          // B operand: (s A)[0..rp, k] for the CTA's 128 output columns, MN-major
+          for (int idx = pt; idx < p.rp * 16; idx += 128) {
+            const int jr = idx >> 4, rem = idx & 15;
             const int cc = rem >> 3, piece = rem & 7;
-            const int k = j0 + cc * 64 + piece * 8;
+            const int k = jb + cc * 64 + piece * 8;
             uint4 v = zero4();
             if (jr < p.r && k < p.K) v = scale8(*reinterpret_cast<const uint4*>(p.lora_b + (size_t)jr * p.K + k), p.s);
-            *reinterpret_cast<uint4*>(sm.b(sb) + cc * 8192 + sw128_offset(jr, piece)) = v;
+            *reinterpret_cast<uint4*>(sm.b(s) + cc * 8192 + sw128_offset(jr, piece)) = v;
           }
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.full_b[sb]);
+        if (lane == 0) mbar_arrive_cluster(&sm.full_b[s], 0);
       }
     }
     // ------------------------------------------------------------ epilogue
@@ -380,7 +370,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (acc_ok) {
       tc_fence_after();
       const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
-      const int g = wp >> 2;                     // 0..3: accumulator g>>1, columns (g&1)*128 ..
+      const int g = wp >> 2;                     // 0..3: half g>>1, columns (g&1)*128 ..
       const int accn = g >> 1;
       const int row = m0 + accn * BMH + quad * 32 + lane;
       for (int cc = 0; cc < 8; ++cc) {
@@ -390,12 +380,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld_wait();
         const int gcol = j0 + col;
         if (row < p.M && gcol < p.n_out) {
+          // n_out is a multiple of 8: the last chunk of a row may hold 8 columns
+          const bool full16 = gcol + 16 <= p.n_out;
           const size_t off = (size_t)row * p.n_out + gcol;
           if (p.out_bf16) {
             __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + off;
             uint32_t pk[8];
             if (p.accumulate) {
-              const uint4 o0 = *reinterpret_cast<const uint4*>(o), o1 = *reinterpret_cast<const uint4*>(o + 8);
+              const uint4 o0 = *reinterpret_cast<const uint4*>(o);
+              const uint4 o1 = full16 ? *reinterpret_cast<const uint4*>(o + 8) : zero4();
               const uint32_t old[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
 #pragma unroll
               for (int q = 0; q < 8; ++q)
@@ -406,19 +399,22 @@ __global__ void __launch_bounds__(THREADS, 1)
               for (int q = 0; q < 8; ++q) pk[q] = pack_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
             }
             reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            if (full16) reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           } else {
             float* o = reinterpret_cast<float*>(p.out) + off;
+            const int nq = full16 ? 4 : 2;
             float v[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(r[q]);
             if (p.accumulate) {
 #pragma unroll
-              for (int q = 0; q < 16; ++q) v[q] = __fadd_rn(v[q], o[q]);
+              for (int q = 0; q < 16; ++q)
+                if (q < 4 * nq) v[q] = __fadd_rn(v[q], o[q]);
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              reinterpret_cast<float4*>(o)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              if (q < nq)
+                reinterpret_cast<float4*>(o)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
           }
         }
       }
@@ -426,15 +422,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   // ------------------------------------------------------------ teardown
-  if (warp == 1 && lane == 0 && *abort_flag) {
+  if (warp == 1 && lane == 0 && rank == 0 && *abort_flag) {
     // let MMAs already issued finish before the accumulators are released
     mbar_wait(sm.acc_full, 0, abort_flag, p.wait_limit);
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // neither CTA leaves while the pair's MMAs or arrivals may still touch it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc2(tmem, TMEM_COLS);
   }
 }
 
@@ -489,11 +485,11 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
     return QL_ERR_CUDA;
   if (!BWD) {
     if (!make_map_2d(&map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, (uint64_t)K / 2, (uint64_t)N,
-                     (uint64_t)K / 2, BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_32B))
+                     (uint64_t)K / 2, BK / 2, BNH, CU_TENSOR_MAP_SWIZZLE_32B))
       return QL_ERR_CUDA;
   } else {
     if (!make_map_2d(&map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, (uint64_t)K / 2, (uint64_t)N,
-                     (uint64_t)K / 2, BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_128B))
+                     (uint64_t)K / 2, BNH / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE))
       return QL_ERR_CUDA;
   }
   Params p;
@@ -513,10 +509,20 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
   p.accumulate = accumulate;
   p.tab = nf4_table();
   p.wait_limit = 1u << 22;
-  dim3 grid((unsigned)((p.n_out + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2u * (unsigned)((p.n_out + BN - 1) / BN), (unsigned)((M + 2 * BM - 1) / (2 * BM)));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   TraceScope ts(BWD ? TK_GEMM_BWD : TK_GEMM_FWD, st);
-  qlora_gemm_kernel<BWD><<<grid, THREADS, SMEM_BYTES, st>>>(map_act, map_codes, p);
-  QL_LAUNCH_CHECK();
+  QL_CUDA_TRY(cudaLaunchKernelEx(&cfg, qlora_gemm_kernel<BWD>, map_act, map_codes, p));
   return QL_OK;
 }
 

@@ -78,6 +78,8 @@ SHAPES = [
     (136, 192, 1, 64, 0.25),         # one token, r = 64
     (512, 1024, 130, 16, 0.75),      # s not a power of two
     (256, 256, 64, 0, 1.0),          # no adapter
+    (264, 192, 40, 16, 0.5),         # N = 8 mod 16: a half chunk at the end of each output row
+    (384, 320, 600, 8, 1.0),         # two token tiles of 512, ragged N and M, stage ring wraps
 ]
 
 
