@@ -65,7 +65,8 @@ def config(world: int) -> dict:
                         "double quant + fwd + bwd (dX, dA, dB)",
             "global_batch": 4096 * world, "N": 4096, "K": 4096, "r": 16,
             "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, untimed)",
-            "outputs": "Y, dX bf16; dA, dB fp32"}
+            "outputs": "Y, dX bf16; dA, dB fp32",
+            "launch": "stream order" if os.environ.get("QL_PDL", "1") == "0" else "programmatic dependent launch"}
 
 
 def gemm_traffic():
@@ -204,6 +205,23 @@ def trace_enable(q, on):
     L.qlora_trace_enable.argtypes = [ctypes.c_int]
     L.qlora_trace_enable.restype = None
     L.qlora_trace_enable(1 if on else 0)
+
+
+def trace_enable_kinds(q, names):
+    """Trace only the named kernel kinds (an event pair around a launch keeps it
+    from overlapping the previous kernel, so the timed steps trace only the
+    dominant kernel)."""
+    import ctypes
+    L = q._lib.LIB
+    L.qlora_trace_kind_name.restype = ctypes.c_char_p
+    L.qlora_trace_kind_name.argtypes = [ctypes.c_int]
+    L.qlora_trace_enable_kinds.argtypes = [ctypes.c_uint]
+    L.qlora_trace_enable_kinds.restype = None
+    mask = 0
+    for k in range(32):
+        if L.qlora_trace_kind_name(k).decode() in names:
+            mask |= 1 << k
+    L.qlora_trace_enable_kinds(mask)
 
 
 # --------------------------------------------------------------- CPU oracle
@@ -421,7 +439,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    trace_enable(q, True)
+    trace_enable_kinds(q, ("qlora_gemm_fwd", "qlora_gemm_bwd"))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
@@ -452,7 +470,18 @@ def run_ours(args, rank, world, local_rank):
     gemm_ms = ms_f + ms_b
     gemm_launches = n_f + n_b
     achieved = (n_f * f_fwd + n_b * f_bwd) / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
-    gpu_launches = sum(c for _, c in kern.values())
+
+    # per-kernel breakdown: the same steps again (untimed) with every kind traced
+    trace_enable(q, True)
+    n_br = min(args.steps, 10)
+    for _ in range(n_br):
+        flush.zero_()
+        wl.step(allreduce)
+    torch.cuda.synchronize()
+    breakdown = trace_read(q)
+    trace_enable(q, False)
+    launches_per_step = sum(c for _, c in breakdown.values()) / n_br
+    gpu_launches = int(round(launches_per_step * args.steps))
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -524,7 +553,8 @@ def run_ours(args, rank, world, local_rank):
                          "frac": achieved / bf16_peak, "peak_source": f"{peak_src} bf16 burst",
                          "traffic": gemm_traffic(), "launches": gemm_launches,
                          "avg_launch_us": gemm_ms / max(gemm_launches, 1) * 1e3},
-            "kernels": {k: {"ms_total": round(v[0], 4), "launches": v[1]} for k, v in kern.items()},
+            "kernels": {k: {"us_per_launch": round(v[0] / v[1] * 1e3, 2), "launches_per_step": v[1] / n_br}
+                        for k, v in breakdown.items()},
             "gpu_launches": gpu_launches,
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -13,6 +13,7 @@
 // The quantile is computed by bisection on Phi(x) = erfc(-x/sqrt 2)/2 in double
 // and polished by Newton steps; the level is then rounded to fp32.
 #include <cmath>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -54,6 +55,14 @@ NF4Table build() {
 }
 
 }  // namespace
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("QL_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 const NF4Table& nf4_table() {
   static NF4Table table = build();

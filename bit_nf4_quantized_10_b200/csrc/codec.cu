@@ -92,6 +92,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, int64_t n,
                                                        uint8_t* __restrict__ codes,
                                                        float* __restrict__ absmax, NF4Table tab, QuantBins bins_in) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ uint2 bins[64];   // (m bits, count below)
   if (threadIdx.x < 64) bins[threadIdx.x] = make_uint2(__float_as_uint(bins_in.m[threadIdx.x]), bins_in.base[threadIdx.x]);
   __syncthreads();
@@ -160,6 +162,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) tree_sum_pass(const T* __restrict__ in, int64_t count,
                                                      double* __restrict__ out, int64_t total_nb,
                                                      float* __restrict__ mean_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ double warp_sums[8];
   const int64_t base = (int64_t)blockIdx.x * 2048 + threadIdx.x * 8;
   double v[8];
@@ -184,6 +188,8 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
                                                         const float* __restrict__ mean,
                                                         uint8_t* __restrict__ absmax_q,
                                                         float* __restrict__ scale2) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t ng = (nb + 255) / 256;
   const int lane = threadIdx.x & 31;
   const float mu = *mean;
@@ -223,6 +229,8 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
 __global__ void __launch_bounds__(256) dequant_bf16_kernel(const uint8_t* __restrict__ codes, WeightConsts wc,
                                                            int64_t n, __nv_bfloat16* __restrict__ out,
                                                            NF4Table tab) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t nb = (n + 63) / 64;
   const float mu = wc.absmax ? 0.0f : *wc.offset;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -250,6 +258,8 @@ __global__ void __launch_bounds__(256) dequant_bf16_kernel(const uint8_t* __rest
 // fp32 output: 8 elements per thread, the 16 levels read from shared memory.
 __global__ void __launch_bounds__(256) dequant_f32_kernel(const uint8_t* __restrict__ codes, WeightConsts wc,
                                                           int64_t n, float* __restrict__ out, NF4Table tab) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float q[16];
   if (threadIdx.x < 16) q[threadIdx.x] = tab.q[threadIdx.x];
   __syncthreads();
@@ -303,10 +313,10 @@ ql_status launch_quantize(const void* x, ql_dtype dt, int64_t n, uint8_t* codes,
   static const QuantBins bins = build_bins(nf4_table());
   TraceScope ts(TK_QUANTIZE, st);
   if (dt == QL_F32)
-    quantize_kernel<float><<<grid, 256, 0, st>>>((const float*)x, n, codes, absmax, nf4_table(), bins);
+    QL_CUDA_TRY(launch(quantize_kernel<float>, dim3(grid), dim3(256), 0, st, 1, 1, (const float*)x, n, codes, absmax, nf4_table(), bins));
   else
-    quantize_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, n, codes, absmax,
-                                                         nf4_table(), bins);
+    QL_CUDA_TRY(launch(quantize_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, 1, 1, (const __nv_bfloat16*)x, n, codes, absmax,
+                                                         nf4_table(), bins));
   QL_LAUNCH_CHECK();
   return QL_OK;
 }
@@ -328,13 +338,13 @@ ql_status launch_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q
   int64_t cnt = (nb + 2047) / 2048;
   {
   TraceScope ts(TK_DQ_MEAN, st);
-  tree_sum_pass<float><<<(unsigned)cnt, 256, 0, st>>>(absmax, nb, buf, nb, cnt == 1 ? offset : nullptr);
+  QL_CUDA_TRY(launch(tree_sum_pass<float>, dim3((unsigned)cnt), dim3(256), 0, st, 1, 1, absmax, nb, buf, nb, cnt == 1 ? offset : nullptr));
   QL_LAUNCH_CHECK();
   double* prev = buf;
   while (cnt > 1) {
     int64_t next = (cnt + 2047) / 2048;
     double* dst = prev + cnt;
-    tree_sum_pass<double><<<(unsigned)next, 256, 0, st>>>(prev, cnt, dst, nb, next == 1 ? offset : nullptr);
+    QL_CUDA_TRY(launch(tree_sum_pass<double>, dim3((unsigned)next), dim3(256), 0, st, 1, 1, prev, cnt, dst, nb, next == 1 ? offset : nullptr));
     QL_LAUNCH_CHECK();
     prev = dst;
     cnt = next;
@@ -342,7 +352,7 @@ ql_status launch_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q
   }
   const int64_t ng = (nb + 255) / 256;
   TraceScope ts(TK_DQ_ENCODE, st);
-  dq_encode_kernel<<<grid_for(ng, 8, 8), 256, 0, st>>>(absmax, nb, offset, absmax_q, scale2);
+  QL_CUDA_TRY(launch(dq_encode_kernel, dim3(grid_for(ng, 8, 8)), dim3(256), 0, st, 1, 1, absmax, nb, offset, absmax_q, scale2));
   QL_LAUNCH_CHECK();
   return QL_OK;
 }
@@ -353,11 +363,11 @@ ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStr
   TraceScope ts(TK_DEQUANT, st);
   if (dt == QL_BF16) {
     const int64_t nb = (n + 63) / 64;
-    dequant_bf16_kernel<<<grid_for(nb, 256, 4), 256, 0, st>>>(w->codes, wc, n, (__nv_bfloat16*)out,
-                                                             nf4_table());
+    QL_CUDA_TRY(launch(dequant_bf16_kernel, dim3(grid_for(nb, 256, 4)), dim3(256), 0, st, 1, 1, w->codes, wc, n, (__nv_bfloat16*)out,
+                                                             nf4_table()));
   } else {
-    dequant_f32_kernel<<<grid_for((n + 7) / 8, 256, 8), 256, 0, st>>>(w->codes, wc, n, (float*)out,
-                                                                     nf4_table());
+    QL_CUDA_TRY(launch(dequant_f32_kernel, dim3(grid_for((n + 7) / 8, 256, 8)), dim3(256), 0, st, 1, 1, w->codes, wc, n, (float*)out,
+                                                                     nf4_table()));
   }
   QL_LAUNCH_CHECK();
   return QL_OK;

@@ -126,6 +126,47 @@ __device__ __forceinline__ uint4 lut_lookup8(const Lut16& L, uint32_t w) {
   return r;
 }
 
+// ------------------------------------------------------- dependent launches
+// Every kernel of the library is launched through launch() with programmatic
+// stream serialization, so it can be scheduled (and run its prologue: barrier
+// set-up, TMEM allocation, descriptor prefetch) while the previous kernel on
+// the stream is still finishing.  Each kernel calls pdl_wait() before its
+// first global-memory access (that returns once every earlier kernel on the
+// stream has completed and its writes are visible) and pdl_trigger() once it
+// holds its on-chip resources, which lets the next kernel be scheduled.
+// QL_PDL=0 in the environment launches without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, unsigned cluster_x,
+                   unsigned cluster_y, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  unsigned n = 0;
+  if (cluster_x * cluster_y > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = cluster_x;
+    at[n].val.clusterDim.y = cluster_y;
+    at[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl_enabled()) {
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace ql
 
 #define QL_CUDA_TRY(expr)                               \

@@ -25,12 +25,14 @@
 // The r LoRA K-steps (U or V against the scaled adapter) run into the same
 // accumulators after the main loop, before the drain.
 //
-// Shared memory per CTA: 4 stages of (activation tile 256 x 64 bf16, the
-// packed codes of the CTA's 128 x 64 weight half, the expanded weight half).
-// Synchronisation: TMA loads complete on the local full_t[s]; each producer
-// warp, in both CTAs, arrives on the even CTA's full_b[s] (8 warps) once its
-// part of the weight tile is written and the CTA's activation tile has landed;
-// the MMA commits multicast to empty[s] and acc_full in both CTAs.
+// Shared memory per CTA: rings of 4 activation tiles (256 x 64 bf16), 8
+// packed-code tiles of the CTA's 128 x 64 weight half (loaded 4 stages ahead,
+// so expanding a stage never waits on a TMA) and 4 expanded weight halves.
+// Synchronisation: TMA loads complete on local barriers (full_a, full_c); each
+// producer warp, in both CTAs, arrives on the even CTA's full_b[s] (8 warps)
+// once its part of the weight tile is written (in the odd CTA, also once the
+// CTA's activation tile of the stage has landed); the MMA commits multicast
+// to empty[s] and acc_full in both CTAs.
 // Warp roles (576 threads per CTA):
 //   warp 0      TMA producer
 //   warp 1      TMEM allocation (both CTAs); one thread of the even CTA
@@ -62,14 +64,16 @@ constexpr int A_BYTES = BM * BK * 2;    // 32 KB activation tile
 constexpr int AH_BYTES = BMH * BK * 2;  // 16 KB: the second half
 constexpr int B_BYTES = BNH * BK * 2;   // 16 KB expanded weight half
 constexpr int C_BYTES = BNH * BK / 2;   // 4 KB of packed codes
-constexpr int STAGES = 4;
+constexpr int STAGES = 4;               // activation and expanded-weight rings
+constexpr int C_STAGES = 8;             // packed-code ring, filled 4 stages ahead
+constexpr int C_AHEAD = C_STAGES - STAGES;
 constexpr int GROUPS = 4;               // producer groups, one stage each in turn
 constexpr int GROUP_WARPS = 4;
 constexpr int PRODUCER_WARPS = GROUPS * GROUP_WARPS;
 constexpr int THREADS = (2 + PRODUCER_WARPS) * 32;
 constexpr int TMEM_COLS = 512;
-constexpr int T_STAGE_BYTES = A_BYTES + C_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * T_STAGE_BYTES + (size_t)STAGES * B_BYTES + 256;
+constexpr size_t SMEM_BYTES =
+    1024 + (size_t)STAGES * A_BYTES + (size_t)C_STAGES * C_BYTES + (size_t)STAGES * B_BYTES + 256;
 
 struct Params {
   int M;             // tokens
@@ -90,11 +94,12 @@ struct Params {
 
 struct Smem {
   uint8_t* base;
-  __device__ __forceinline__ uint8_t* a(int s) const { return base + s * T_STAGE_BYTES; }
-  __device__ __forceinline__ uint8_t* c(int s) const { return base + s * T_STAGE_BYTES + A_BYTES; }
-  __device__ __forceinline__ uint8_t* b(int s) const { return base + STAGES * T_STAGE_BYTES + s * B_BYTES; }
-  uint64_t* full_t;    // [STAGES] activation tile + codes landed (local TMA)
-  uint64_t* full_b;    // [STAGES] even CTA: both CTAs' weight halves written (8 warps)
+  __device__ __forceinline__ uint8_t* a(int s) const { return base + s * A_BYTES; }
+  __device__ __forceinline__ uint8_t* b(int s) const { return base + STAGES * A_BYTES + s * B_BYTES; }
+  __device__ __forceinline__ uint8_t* c(int s) const { return base + STAGES * (A_BYTES + B_BYTES) + s * C_BYTES; }
+  uint64_t* full_a;    // [STAGES] activation tile landed (local TMA)
+  uint64_t* full_c;    // [C_STAGES] packed codes landed (local TMA)
+  uint64_t* full_b;    // [STAGES] even CTA: both CTAs' weight halves written and activations landed
   uint64_t* empty;     // [STAGES] pair MMA done with the stage (commit to both CTAs)
   uint64_t* acc_full;
   uint32_t* tmem_addr;
@@ -105,12 +110,13 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   Smem s;
   uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.base = p;
-  p += STAGES * T_STAGE_BYTES + STAGES * B_BYTES;
+  p += STAGES * (A_BYTES + B_BYTES) + C_STAGES * C_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(p);
-  s.full_t = bars;
-  s.full_b = bars + STAGES;
-  s.empty = bars + 2 * STAGES;
-  s.acc_full = bars + 3 * STAGES;
+  s.full_a = bars;
+  s.full_c = bars + STAGES;
+  s.full_b = s.full_c + C_STAGES;
+  s.empty = s.full_b + STAGES;
+  s.acc_full = s.empty + STAGES;
   s.tmem_addr = reinterpret_cast<uint32_t*>(s.acc_full + 1);
   s.abort = reinterpret_cast<int*>(s.tmem_addr + 1);
   return s;
@@ -172,10 +178,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&sm.full_t[i], 1);
+      mbar_init(&sm.full_a[i], 1);
       mbar_init(&sm.full_b[i], 2 * GROUP_WARPS);
       mbar_init(&sm.empty[i], 1);
     }
+    for (int i = 0; i < C_STAGES; ++i) mbar_init(&sm.full_c[i], 1);
     mbar_init(sm.acc_full, 1);
     *sm.abort = 0;
     fence_mbar_init();
@@ -192,25 +199,42 @@ __global__ void __launch_bounds__(THREADS, 1)
   cluster_sync();   // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_addr;
+  pdl_wait();       // earlier kernels on the stream are complete from here on
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA warp
+    // Codes run C_AHEAD stages ahead of the activations.  The code slot of
+    // stage j was last used by stage j - 8, whose producers read it before
+    // the pair MMA of stage j - 8 could start; codes for stage j are issued
+    // after waiting for that MMA (the activation slot wait for stage j - 4).
     if (lane == 0) {
-      int issued = 0;
+      auto load_codes = [&](int j) {
+        const int c = j % C_STAGES;
+        mbar_arrive_expect_tx(&sm.full_c[c], C_BYTES);
+        if (!BWD)
+          tma_load_2d(sm.c(c), &tmap_codes, &sm.full_c[c], j * (BK / 2), jb);
+        else
+          tma_load_2d(sm.c(c), &tmap_codes, &sm.full_c[c], jb / 2, j * BK);
+      };
+      int issued_c = 0, issued_a = 0;
+      for (; issued_c < C_AHEAD && issued_c < p.n_steps; ++issued_c) load_codes(issued_c);
       for (int i = 0; i < p.n_steps; ++i) {
         const int s = i % STAGES, use = i / STAGES;
         if (use > 0 && !mbar_wait(&sm.empty[s], (use - 1) & 1, abort_flag, p.wait_limit)) break;
-        mbar_arrive_expect_tx(&sm.full_t[s], A_BYTES + C_BYTES);
-        if (!BWD)
-          tma_load_2d(sm.c(s), &tmap_codes, &sm.full_t[s], i * (BK / 2), jb);
-        else
-          tma_load_2d(sm.c(s), &tmap_codes, &sm.full_t[s], jb / 2, i * BK);
-        tma_load_2d(sm.a(s), &tmap_act, &sm.full_t[s], i * BK, m0);
-        issued = i + 1;
+        mbar_arrive_expect_tx(&sm.full_a[s], A_BYTES);
+        tma_load_2d(sm.a(s), &tmap_act, &sm.full_a[s], i * BK, m0);
+        issued_a = i + 1;
+        if (i + C_AHEAD < p.n_steps) {
+          load_codes(i + C_AHEAD);
+          issued_c = i + C_AHEAD + 1;
+        }
       }
       // before leaving, make sure no copy is still landing in shared memory
-      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-        mbar_wait(&sm.full_t[i % STAGES], (i / STAGES) & 1, abort_flag, p.wait_limit);
+      for (int i = (issued_a > STAGES ? issued_a - STAGES : 0); i < issued_a; ++i)
+        mbar_wait(&sm.full_a[i % STAGES], (i / STAGES) & 1, abort_flag, p.wait_limit);
+      for (int j = (issued_c > C_STAGES ? issued_c - C_STAGES : 0); j < issued_c; ++j)
+        mbar_wait(&sm.full_c[j % C_STAGES], (j / C_STAGES) & 1, abort_flag, p.wait_limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -219,7 +243,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       for (int i = 0; i < p.n_steps && ok; ++i) {
         const int s = i % STAGES, use = i / STAGES;
-        ok = mbar_wait(&sm.full_t[s], use & 1, abort_flag, p.wait_limit) &&
+        ok = mbar_wait(&sm.full_a[s], use & 1, abort_flag, p.wait_limit) &&
              mbar_wait_cluster(&sm.full_b[s], use & 1, abort_flag, p.wait_limit);
         if (!ok) break;
         tc_fence_after();
@@ -300,14 +324,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         valid = wrow < p.N && kb < kblocks;
         next = load_const(p.wc, (int64_t)wrow * kblocks + kb, valid);
       }
-      // the stage's codes and activation tile landed (so the pair MMA is done
-      // with this slot's previous use: the TMA refilled it only after that)
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.full_t[s], use & 1, abort_flag, p.wait_limit));
+      // the stage's codes landed, and the pair MMA is done with the slot's previous use
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.full_c[i % C_STAGES], (i / C_STAGES) & 1, abort_flag, p.wait_limit) &&
+                                       (use == 0 || mbar_wait(&sm.empty[s], (use - 1) & 1, abort_flag, p.wait_limit)));
       if (!ok) break;
       uint8_t* base = sm.b(s);
+      const uint8_t* cs = sm.c(i % C_STAGES);
       if (cur_valid) {
-        const uint4 c0 = *reinterpret_cast<const uint4*>(sm.c(s) + coff0);
-        const uint4 c1 = *reinterpret_cast<const uint4*>(sm.c(s) + coff1);
+        const uint4 c0 = *reinterpret_cast<const uint4*>(cs + coff0);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(cs + coff1);
         const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         const Lut16 L = make_lut(p.tab, decode_const(p.wc, cur, mu));
 #pragma unroll
@@ -317,8 +342,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(base + boff[j]) = zero4();
       }
       fence_proxy_async_smem();
+      // the odd CTA's arrival also vouches for its activation tile of the stage
+      if (rank != 0) ok = __all_sync(0xffffffffu, mbar_wait(&sm.full_a[s], use & 1, abort_flag, p.wait_limit));
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(&sm.full_b[s], 0);
+      if (lane == 0 && ok) mbar_arrive_cluster(&sm.full_b[s], 0);
     }
     const int pt = gt;
     // LoRA operands into the slot after the last main step, written by the
@@ -509,20 +536,9 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
   p.accumulate = accumulate;
   p.tab = nf4_table();
   p.wait_limit = 1u << 22;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2u * (unsigned)((p.n_out + BN - 1) / BN), (unsigned)((M + 2 * BM - 1) / (2 * BM)));
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  const dim3 grid(2u * (unsigned)((p.n_out + BN - 1) / BN), (unsigned)((M + 2 * BM - 1) / (2 * BM)));
   TraceScope ts(BWD ? TK_GEMM_BWD : TK_GEMM_FWD, st);
-  QL_CUDA_TRY(cudaLaunchKernelEx(&cfg, qlora_gemm_kernel<BWD>, map_act, map_codes, p));
+  QL_CUDA_TRY(launch(qlora_gemm_kernel<BWD>, grid, dim3(THREADS), SMEM_BYTES, st, 2, 1, map_act, map_codes, p));
   return QL_OK;
 }
 

@@ -116,6 +116,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_addr;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -227,6 +229,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 // dst [cols, ld_dst] = src [rows, cols]^T (bf16, cols = r <= 64).
 __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ src, int rows, int cols,
                                                         uint16_t* __restrict__ dst, int ld_dst) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t total = (int64_t)rows * cols;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
@@ -303,22 +307,11 @@ static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, 
   p.ld_t = (int)ld_t;
   p.t_bf16 = t_dt == QL_BF16;
   p.wait_limit = 1u << 22;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits);
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr_c[1];
-  attr_c[0].id = cudaLaunchAttributeClusterDimension;
-  attr_c[0].val.clusterDim.x = 1;
-  attr_c[0].val.clusterDim.y = (unsigned)splits;
-  attr_c[0].val.clusterDim.z = 1;
-  cfg.attrs = attr_c;
-  cfg.numAttrs = 1;
+  const dim3 grid((unsigned)tiles, (unsigned)splits);
   {
     TraceScope ts(kind, st);
-    if (a_mn) QL_CUDA_TRY(cudaLaunchKernelEx(&cfg, skinny_kernel<true>, ma, mb, p));
-    else QL_CUDA_TRY(cudaLaunchKernelEx(&cfg, skinny_kernel<false>, ma, mb, p));
+    if (a_mn) QL_CUDA_TRY(launch(skinny_kernel<true>, grid, dim3(THREADS), SMEM_BYTES, st, 1, (unsigned)splits, ma, mb, p));
+    else QL_CUDA_TRY(launch(skinny_kernel<false>, grid, dim3(THREADS), SMEM_BYTES, st, 1, (unsigned)splits, ma, mb, p));
   }
   return QL_OK;
 }
@@ -347,7 +340,7 @@ ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, i
   const int64_t total = rows * cols;
   const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, (int64_t)sm_count_tc() * 8));
   TraceScope ts(TK_TRANSPOSE, st);
-  skinny::transpose_kernel<<<g, 256, 0, st>>>((const uint16_t*)src, (int)rows, cols, (uint16_t*)dst, (int)ld_dst);
+  QL_CUDA_TRY(launch(skinny::transpose_kernel, dim3(g), dim3(256), 0, st, 1, 1, (const uint16_t*)src, (int)rows, cols, (uint16_t*)dst, (int)ld_dst));
   QL_LAUNCH_CHECK();
   return QL_OK;
 }

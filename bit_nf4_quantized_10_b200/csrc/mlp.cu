@@ -13,6 +13,8 @@ __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf
 
 __global__ void __launch_bounds__(256) silu_gate_fwd_kernel(const uint4* __restrict__ g, const uint4* __restrict__ u,
                                                             uint4* __restrict__ h, int64_t n8) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
     const uint4 gv = g[i], uv = u[i];
     const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
@@ -29,6 +31,8 @@ __global__ void __launch_bounds__(256) silu_gate_fwd_kernel(const uint4* __restr
 __global__ void __launch_bounds__(256) silu_gate_bwd_kernel(const uint4* __restrict__ dh, const uint4* __restrict__ g,
                                                             const uint4* __restrict__ u, uint4* __restrict__ dg,
                                                             uint4* __restrict__ du, int64_t n8) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
     const uint4 dv = dh[i], gv = g[i], uv = u[i];
     const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
@@ -66,7 +70,7 @@ ql_status launch_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n,
   if (n % 8) return QL_ERR_UNSUPPORTED;
   const int64_t n8 = n / 8;
   TraceScope ts(TK_SILU, st);
-  silu_gate_fwd_kernel<<<elem_grid(n8), 256, 0, st>>>((const uint4*)g, (const uint4*)u, (uint4*)h, n8);
+  QL_CUDA_TRY(launch(silu_gate_fwd_kernel, dim3(elem_grid(n8)), dim3(256), 0, st, 1, 1, (const uint4*)g, (const uint4*)u, (uint4*)h, n8));
   QL_LAUNCH_CHECK();
   return QL_OK;
 }
@@ -76,8 +80,8 @@ ql_status launch_silu_gate_bwd(const void* dh, const void* g, const void* u, voi
   if (n % 8) return QL_ERR_UNSUPPORTED;
   const int64_t n8 = n / 8;
   TraceScope ts(TK_SILU, st);
-  silu_gate_bwd_kernel<<<elem_grid(n8), 256, 0, st>>>((const uint4*)dh, (const uint4*)g, (const uint4*)u,
-                                                      (uint4*)dg, (uint4*)du, n8);
+  QL_CUDA_TRY(launch(silu_gate_bwd_kernel, dim3(elem_grid(n8)), dim3(256), 0, st, 1, 1, (const uint4*)dh, (const uint4*)g, (const uint4*)u,
+                                                      (uint4*)dg, (uint4*)du, n8));
   QL_LAUNCH_CHECK();
   return QL_OK;
 }

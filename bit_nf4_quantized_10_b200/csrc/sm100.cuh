@@ -85,13 +85,15 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   return false;
 }
 
-// Arrive (release, cluster scope) on the barrier at the same shared-memory
-// offset in CTA `rank` of the cluster.
+// Arrive on the barrier at the same shared-memory offset in CTA `rank` of the
+// cluster (default release semantics; the waiting side acquires at cluster
+// scope).  The writes it publishes are shared-memory operands that the caller
+// has already fenced to the async proxy.
 __device__ __forceinline__ void mbar_arrive_cluster(uint64_t* bar, uint32_t rank) {
   asm volatile(
       "{\n .reg .b32 ra;\n"
       " mapa.shared::cluster.u32 ra, %0, %1;\n"
-      " mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n}" ::"r"(smem_u32(bar)),
+      " mbarrier.arrive.shared::cluster.b64 _, [ra];\n}" ::"r"(smem_u32(bar)),
       "r"(rank)
       : "memory");
 }

@@ -123,6 +123,8 @@ __global__ void __launch_bounds__(THREADS, 3)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_addr;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -265,6 +267,8 @@ __global__ void __launch_bounds__(256) smallm_reduce_kernel(const float* __restr
                                                             const __nv_bfloat16* __restrict__ U,
                                                             const __nv_bfloat16* __restrict__ B, int r, float s,
                                                             int out_bf16, void* __restrict__ Y) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float us[TN * 64];
   for (int i = threadIdx.x; i < M * r; i += blockDim.x) us[i] = __bfloat162float(U[i]);
   __syncthreads();
@@ -348,15 +352,15 @@ ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, co
   dim3 grid((unsigned)((N + TM - 1) / TM), (unsigned)splits);
   {
     TraceScope ts(TK_SMALLM, st);
-    smallm_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(map_x, map_codes, p);
+    QL_CUDA_TRY(launch(smallm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, st, 1, 1, map_x, map_codes, p));
   }
   QL_LAUNCH_CHECK();
   const unsigned rg =
       (unsigned)std::max<int64_t>(1, std::min<int64_t>((M * (int64_t)N + 255) / 256, (int64_t)sm_count_sm() * 8));
   {
     TraceScope ts(TK_COLACC_REDUCE, st);
-    smallm_reduce_kernel<<<rg, 256, 0, st>>>(partial, splits, (int)M, N, (const __nv_bfloat16*)U,
-                                             (const __nv_bfloat16*)B, r, s, y_dt == QL_BF16, Y);
+    QL_CUDA_TRY(launch(smallm_reduce_kernel, dim3(rg), dim3(256), 0, st, 1, 1, partial, splits, (int)M, N, (const __nv_bfloat16*)U,
+                                             (const __nv_bfloat16*)B, r, s, y_dt == QL_BF16, Y));
   }
   QL_LAUNCH_CHECK();
   return QL_OK;

@@ -14,7 +14,7 @@ struct Rec {
   int kind;
   cudaEvent_t a, b;
 };
-std::atomic<int> g_on{0};
+std::atomic<unsigned> g_on{0};
 std::mutex g_mu;
 std::vector<Rec> g_recs;
 std::vector<cudaEvent_t> g_free;
@@ -24,7 +24,7 @@ const char* const kNames[TK_COUNT] = {"nf4_quantize",   "dq_tree_sum",    "dq_en
 }  // namespace
 
 const char* trace_name(int kind) { return (kind >= 0 && kind < TK_COUNT) ? kNames[kind] : "unknown"; }
-bool trace_on() { return g_on.load(std::memory_order_relaxed) != 0; }
+bool trace_on(int kind) { return (g_on.load(std::memory_order_relaxed) >> kind) & 1u; }
 
 cudaEvent_t trace_event() {
   std::lock_guard<std::mutex> lk(g_mu);
@@ -47,7 +47,9 @@ void trace_push(int kind, cudaEvent_t a, cudaEvent_t b) {
 
 extern "C" {
 
-void qlora_trace_enable(int on) {
+void qlora_trace_enable(int on) { qlora_trace_enable_kinds(on ? 0xFFFFFFFFu : 0u); }
+
+void qlora_trace_enable_kinds(unsigned mask) {
   std::lock_guard<std::mutex> lk(ql::g_mu);
   for (auto& r : ql::g_recs) {
     cudaEventSynchronize(r.b);
@@ -55,7 +57,7 @@ void qlora_trace_enable(int on) {
     ql::g_free.push_back(r.b);
   }
   ql::g_recs.clear();
-  ql::g_on.store(on ? 1 : 0);
+  ql::g_on.store(mask);
 }
 
 int qlora_trace_read(double* total_ms, int* launches, int max_kinds) {

@@ -1,6 +1,7 @@
-// Optional per-kernel device timing.  When enabled (qlora_trace_enable), every
-// launch site records a CUDA event pair around its kernel on the caller's
-// stream; qlora_trace_read waits for the events and reports, per kernel kind,
+// Optional per-kernel device timing.  When enabled for a kernel kind
+// (qlora_trace_enable, qlora_trace_enable_kinds), its launch sites record a
+// CUDA event pair around the kernel on the caller's stream (which also keeps
+// that launch from overlapping the previous kernel's tail); qlora_trace_read waits for the events and reports, per kernel kind,
 // the launch count and total device time.  Disabled, a launch site costs one
 // relaxed atomic load.
 #pragma once
@@ -26,7 +27,7 @@ enum TraceKind : int {
 };
 
 const char* trace_name(int kind);
-bool trace_on();
+bool trace_on(int kind);
 void trace_push(int kind, cudaEvent_t start, cudaEvent_t stop);
 cudaEvent_t trace_event();
 
@@ -36,7 +37,7 @@ struct TraceScope {
   cudaStream_t st;
   cudaEvent_t a = nullptr, b = nullptr;
   TraceScope(int k, cudaStream_t s) : kind(k), st(s) {
-    if (trace_on()) {
+    if (trace_on(k)) {
       a = trace_event();
       b = trace_event();
       if (a && b) cudaEventRecord(a, st);

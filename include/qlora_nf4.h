@@ -225,13 +225,19 @@ ql_status qlora_get_status(void* stream);
 /*
  * Per-kernel device timing, for profiling.  qlora_trace_enable(1) starts
  * recording a CUDA event pair around every kernel the library launches (on the
- * caller's stream); qlora_trace_enable(0) stops; either call discards earlier
- * records.  qlora_trace_read waits for the recorded events, writes for each
- * kernel kind k < max_kinds the total device milliseconds and launch count,
- * clears the records and returns the number of kinds written.  Kind names
- * come from qlora_trace_kind_name.  Host-side only; the caller owns the arrays.
+ * caller's stream); qlora_trace_enable(0) stops; qlora_trace_enable_kinds(mask)
+ * records only the kinds k with bit k of mask set.  Each of these calls
+ * discards earlier records.  An event pair around a kernel also keeps that
+ * launch from starting while the previous kernel on the stream finishes (the
+ * library otherwise overlaps consecutive launches: programmatic dependent
+ * launch), so trace only the kinds you need.  qlora_trace_read waits for the
+ * recorded events, writes for each kernel kind k < max_kinds the total device
+ * milliseconds and launch count, clears the records and returns the number of
+ * kinds written.  Kind names come from qlora_trace_kind_name.  Host-side only;
+ * the caller owns the arrays.  No counterpart on the pages (instrumentation).
  */
 void qlora_trace_enable(int on);
+void qlora_trace_enable_kinds(unsigned mask);
 int qlora_trace_read(double* total_ms, int* launches, int max_kinds);
 const char* qlora_trace_kind_name(int kind);
 
