@@ -182,8 +182,7 @@ class Projection:
         q.qlora_linear_bwd(self.wq, self.X, self.dY, self.A, self.B, self.r, self.s, self.U, self.dX, self.dA,
                            self.dB, ws=self.ws)
         if allreduce:
-            allreduce(self.dA)
-            allreduce(self.dB)
+            allreduce(self.dA, self.dB)
 
 
 def trace_read(q):
@@ -420,7 +419,8 @@ def run_ours(args, rank, world, local_rank):
     wl = Projection(q, dev, rank)
     allreduce = None
     if world > 1:
-        allreduce = lambda t: dist.all_reduce(t)
+        from bit_nf4_quantized_10_b200.dp import allreduce_adapter_grads
+        allreduce = allreduce_adapter_grads
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2 (126 MB)
 
     clocks = ClockSampler(local_rank)

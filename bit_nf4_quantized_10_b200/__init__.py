@@ -8,7 +8,7 @@ from ._lib import (  # noqa: F401
     LIB_PATH, QLoraError, NF4Weight, quantize_weight,
     nf4_quantize, nf4_double_quant, nf4_dequant, qlora_linear_fwd, qlora_linear_bwd,
     qlora_silu_gate_fwd, qlora_silu_gate_bwd, qlora_workspace_size, nf4_storage_bytes,
-    nf4_codebook, qlora_get_status, status_string,
+    nf4_codebook, qlora_get_status, status_string, qlora_selftest_wait_timeout,
     QL_F32, QL_BF16, QL_OP_DOUBLE_QUANT, QL_OP_FWD, QL_OP_BWD,
     QL_OK, QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_WORKSPACE, QL_ERR_CUDA, QL_ERR_NONFINITE, QL_ERR_TIMEOUT,
 )

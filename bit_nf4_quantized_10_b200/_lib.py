@@ -22,7 +22,7 @@ QL_OP_DOUBLE_QUANT, QL_OP_FWD, QL_OP_BWD = 0, 1, 2
 
 EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_double_quant_noalloc", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
            "qlora_silu_gate_fwd", "qlora_silu_gate_bwd", "qlora_workspace_size", "nf4_storage_bytes",
-           "nf4_codebook", "qlora_get_status", "qlora_status_string")
+           "nf4_codebook", "qlora_get_status", "qlora_status_string", "qlora_selftest_wait_timeout")
 
 
 class QLoraError(RuntimeError):
@@ -57,6 +57,7 @@ def _load() -> ctypes.CDLL:
         "nf4_codebook": (None, [ctypes.POINTER(ctypes.c_float)]),
         "qlora_get_status": (i32, [vp]),
         "qlora_status_string": (ctypes.c_char_p, [i32]),
+        "qlora_selftest_wait_timeout": (i32, [i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -118,6 +119,12 @@ def qlora_workspace_size(op: int, M: int, N: int = 0, K: int = 0, r: int = 0) ->
 
 def qlora_get_status(stream=None) -> int:
     return int(LIB.qlora_get_status(_stream(stream)))
+
+
+def qlora_selftest_wait_timeout(polls: int, stream=None) -> None:
+    """Launch the bounded-wait self-test (a wait nothing satisfies, limited to
+    `polls` polls); the next qlora_get_status reports QL_ERR_TIMEOUT."""
+    _check(LIB.qlora_selftest_wait_timeout(int(polls), _stream(stream)), "qlora_selftest_wait_timeout")
 
 
 # ------------------------------------------------------------------ device calls

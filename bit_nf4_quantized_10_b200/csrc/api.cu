@@ -19,6 +19,10 @@ ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, cons
 ql_status launch_gemm_bwd(const ql_nf4_weight* w, const void* dY, int64_t M, const void* V, const void* A, int r,
                           float s, void* dX, ql_dtype dx_dt, int accumulate, cudaStream_t st);
 unsigned status_word_gemm(cudaStream_t st);
+unsigned status_word_lora(cudaStream_t st);
+unsigned status_word_smallm(cudaStream_t st);
+unsigned status_word_diag(cudaStream_t st);
+ql_status launch_wait_timeout(uint32_t polls, cudaStream_t st);
 // lora_tc.cu
 ql_status launch_proj(const void* Z, int64_t M, int64_t red, const void* Gt, int64_t ld_gt, int r, void* out,
                       void* out_t, int64_t ld_t, cudaStream_t st);
@@ -28,9 +32,9 @@ ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t
                         ql_dtype dt, cudaStream_t st);
 ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st);
 // smallm.cu
-size_t smallm_partial_bytes(int64_t N, int64_t K);
+bool smallm_supported(int64_t N, int64_t K);
 ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
-                            float s, void* Y, ql_dtype y_dt, float* partial, cudaStream_t st);
+                            float s, void* Y, ql_dtype y_dt, cudaStream_t st);
 // mlp.cu
 ql_status launch_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, cudaStream_t st);
 ql_status launch_silu_gate_bwd(const void* dh, const void* g, const void* u, void* dg, void* du, int64_t n,
@@ -67,14 +71,17 @@ ql_status check_gemm_shape(const ql_nf4_weight* w, int64_t M, int r) {
   return QL_OK;
 }
 
-// Tokens up to this count take the small-M (HBM-bound) forward kernel.
+// Tokens up to this count take the small-M (HBM-bound) forward kernel, for
+// K up to 40960 (its K slice of X must fit in shared memory).
 constexpr int64_t kSmallM = 16;
 
-// Forward workspace: U [M, r] (when U_out is not given), then, for M <= 16,
-// the small-M kernel's fp32 split-K partials.
+bool use_smallm(int64_t M, int64_t N, int64_t K) { return M <= kSmallM && ql::smallm_supported(N, K); }
+
+// Forward workspace: U [M, r] (when U_out is not given).
 size_t ws_fwd(int64_t M, int64_t N, int64_t K, int r) {
-  const size_t part = M <= kSmallM ? ql::smallm_partial_bytes(N, K) : 0;
-  return align256((size_t)M * r * 2) + align256(part);
+  (void)N;
+  (void)K;
+  return align256((size_t)M * r * 2);
 }
 
 // Backward workspace, carved in this order (each piece 256-byte aligned):
@@ -134,18 +141,16 @@ ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, con
   if (M == 0) return QL_OK;
   cudaStream_t cs = as_stream(stream);
   const int64_t N = w->rows, K = w->cols;
-  const bool small = M <= kSmallM;
+  const bool small = use_smallm(M, N, K);
   if (r == 0 && !small) return ql::launch_gemm_fwd(w, X, M, nullptr, nullptr, 0, s, Y, y_dt, cs);
   if (ws_bytes < ws_fwd(M, N, K, r)) return QL_ERR_WORKSPACE;
   if (!aligned16(ws)) return QL_ERR_INVALID_ARG;
-  uint8_t* wp = reinterpret_cast<uint8_t*>(ws);
-  void* U = U_out ? U_out : wp;
-  float* partial = reinterpret_cast<float*>(wp + align256((size_t)M * r * 2));
+  void* U = U_out ? U_out : ws;
   if (r > 0) {
     st = ql::launch_proj(X, M, K, A, K, r, U, nullptr, 0, cs);    // U = bf16(X A^T)
     if (st != QL_OK) return st;
   }
-  if (small) return ql::launch_smallm_fwd(w, X, M, U, B, r, s, Y, y_dt, partial, cs);
+  if (small) return ql::launch_smallm_fwd(w, X, M, U, B, r, s, Y, y_dt, cs);
   return ql::launch_gemm_fwd(w, X, M, U, B, r, s, Y, y_dt, cs);
 }
 
@@ -196,6 +201,11 @@ ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY
   return ql::launch_grad_a(X, M, (int)K, Vt, Mp, r, s, dA, grad_dt, cs);   // dA = s V^T X
 }
 
+ql_status qlora_selftest_wait_timeout(int64_t polls, void* stream) {
+  if (polls < 1 || polls > (1 << 20)) return QL_ERR_INVALID_ARG;
+  return ql::launch_wait_timeout((uint32_t)polls, as_stream(stream));
+}
+
 ql_status qlora_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, void* stream) {
   if (n <= 0 || !aligned16(g) || !aligned16(u) || !aligned16(h)) return QL_ERR_INVALID_ARG;
   return ql::launch_silu_gate_fwd(g, u, h, n, as_stream(stream));
@@ -231,10 +241,14 @@ void nf4_codebook(float out[16]) {
 ql_status qlora_get_status(void* stream) {
   cudaStream_t cs = as_stream(stream);
   if (cudaStreamSynchronize(cs) != cudaSuccess) return QL_ERR_CUDA;
-  const unsigned a = ql::status_word_codec(cs);
-  const unsigned b = ql::status_word_gemm(cs);
-  if (a == ~0u || b == ~0u) return QL_ERR_CUDA;
-  const unsigned v = a | b;
+  // one status word per translation unit that raises status bits
+  unsigned v = 0;
+  for (unsigned (*word)(cudaStream_t) : {ql::status_word_codec, ql::status_word_gemm, ql::status_word_lora,
+                                         ql::status_word_smallm, ql::status_word_diag}) {
+    const unsigned w = word(cs);
+    if (w == ~0u) return QL_ERR_CUDA;
+    v |= w;
+  }
   if (v & ql::ST_NONFINITE) return QL_ERR_NONFINITE;
   if (v & ql::ST_TIMEOUT) return QL_ERR_TIMEOUT;
   return QL_OK;

@@ -26,6 +26,8 @@
 namespace ql {
 using namespace sm100;
 
+QL_DEFINE_STATUS_ACCESSOR(status_word_lora)
+
 bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
                  uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
 

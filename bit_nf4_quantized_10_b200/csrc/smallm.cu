@@ -3,22 +3,26 @@
 // With a handful of tokens each dequantized weight element meets at most 16
 // activations, so the layer is bound by reading the packed 4-bit weight from
 // HBM ("QLoRA — Fine-Tuning a 65B Model on One GPU", "Pitfalls":
-// memory-bandwidth-bound generation has less to read with 4-bit weights), and
-// the dequantization must keep pace with HBM.  The design differs from the
-// large-M kernel accordingly:
-//   * operands are swapped: the dequantized weight tile is the MMA's A operand
-//     (M = 128 weight rows) and lives in TMEM, written with tcgen05.st straight
-//     from the producer registers, so it costs no shared-memory bandwidth;
-//     the tokens are the N = 16 operand (zero-padded by TMA);
-//   * the expansion reads the 16 fp32 levels from a shared-memory table (one
-//     conflict-free LDS per element), multiplies by the block constant in fp32
-//     and packs pairs to bf16 — the same bf16(fl32(q * c)) as everywhere else,
-//     with fewer integer operations than the register lookup table;
-//   * each TMA stage brings 128 contiguous bytes (256 codes) of every weight
-//     row, four 64-deep MMA sub-steps, so HBM is read in whole 128-byte lines;
-//   * the reduction over K is split across CTAs (partials stay in L2) and a
-//     second kernel adds the partials in fixed order together with the rank-r
-//     term s * U * B^T in fp32.
+// memory-bandwidth-bound generation has less to read with 4-bit weights) and
+// by the integer work of expanding it, which must keep pace with HBM.
+//   * Operands are swapped: the expanded weight tile is the MMA's A operand
+//     (M = 128 weight rows) and lives in TMEM, written with tcgen05.st from the
+//     producer registers; the tokens are the N = 16 operand (zero-padded).
+//   * Expansion: the 16 fp32 levels sit in a shared-memory table (one
+//     conflict-free LDS per element), times the block constant in fp32, pairs
+//     packed to bf16: bf16(fl32(q * c)), as everywhere else.
+//   * Persistent clusters: the CTAs of a cluster (up to 8) split K, so each
+//     CTA owns one fixed K slice and keeps the tokens' slice of X in shared
+//     memory for the whole kernel; the clusters walk over 128-row weight
+//     tiles.  Each TMA stage brings 128 contiguous bytes (256 codes) of every
+//     row of the tile.
+//   * The split-K partials meet in shared memory: each CTA drains its 128 x 16
+//     fp32 partial (TMEM, double-buffered) into shared memory, and CTA q of the
+//     cluster adds the slices of its share of the tile's outputs in slice
+//     order through distributed shared memory, adds s * U * B^T in fp32 and
+//     writes Y.  Hand-offs between the CTAs go through mbarriers with remote
+//     arrivals (release/acquire at cluster scope), so the expansion of the
+//     next tile overlaps the reduction of the last.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -30,33 +34,49 @@
 namespace ql {
 using namespace sm100;
 
+QL_DEFINE_STATUS_ACCESSOR(status_word_smallm)
+
 bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
                  uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
 
 namespace smallm {
 
-constexpr int TM = 128;           // weight rows per CTA (MMA M)
+constexpr int TM = 128;           // weight rows per tile (MMA M)
 constexpr int TN = 16;            // token slots (MMA N)
 constexpr int BK = 64;            // reduction elements per MMA sub-step (one 64-block per row)
-constexpr int SUB = 4;            // sub-steps per TMA stage: 256 codes = 128 contiguous bytes per row
-constexpr int STAGES = 2;         // TMA ring
-constexpr int A_STAGES = 3;       // TMEM ring of dequantized 128 x 64 A tiles
-constexpr int C_BYTES = TM * BK * SUB / 2;   // 16 KB packed codes
-constexpr int X_SUB_BYTES = TN * BK * 2;     // 2 KB activation sub-tile
-constexpr int STAGE_BYTES = C_BYTES + SUB * X_SUB_BYTES;
-constexpr int PRODUCER_WARPS = 8;
-constexpr int THREADS = (2 + PRODUCER_WARPS) * 32;
-constexpr int TMEM_COLS = 128;    // D: 16 columns; A stages: 32 columns each from column 32 (3 CTAs per SM)
-constexpr int A_COL0 = 32;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+constexpr int SUB = 4;            // sub-steps per code stage: 256 codes = 128 contiguous bytes per row
+constexpr int C_STAGE_BYTES = TM * BK * SUB / 2;   // 16 KB packed codes
+constexpr int MAX_C_STAGES = 8;
+constexpr int X_SUB_BYTES = TN * BK * 2;           // 2 KB activation sub-tile
+constexpr int MAX_PER = 80;       // sub-steps per K slice (bounded by shared memory)
+constexpr int MAX_CS = 8;         // CTAs per cluster (portable cluster size)
+constexpr int A_STAGES = 3;       // TMEM ring of expanded A stages (128 rows x 256 codes each)
+constexpr int GROUP_WARPS = 8;    // producer warps per group; two groups take alternate sub-steps
+constexpr int PRODUCER_WARPS = 2 * GROUP_WARPS;
+constexpr int DRAIN_WARP0 = 2 + PRODUCER_WARPS;
+constexpr int DRAIN_WARPS = 4;
+constexpr int THREADS = (DRAIN_WARP0 + DRAIN_WARPS) * 32;
+constexpr int TMEM_COLS = 512;    // D[b] at columns 16 b; A stage s at 128 + 128 s (32 per sub-step)
+constexpr int A_COL0 = 128;
+constexpr int A_STAGE_COLS = 128;
+constexpr int RED_LD = 18;        // floats per row of a reduction buffer (conflict-free float2 reads)
+constexpr int RED_BYTES = TM * RED_LD * 4;
+constexpr int MAX_R = 64;
 
 struct Params {
-  int M, N, K;
-  int stages_total, stages_per_split;   // in TMA stages of SUB * BK reduction elements
-  int sub_total;                        // K / 64 (the last stage may be partial)
+  int M, N, K, r;
+  int kb_total;       // K / 64
+  int per;            // sub-steps per K slice (the last slice may be shorter)
+  int tiles;          // ceil(N / 128)
+  int c_stages;       // code ring depth (a power of two)
+  int c_log;          // log2(c_stages)
+  float s;
   WeightConsts wc;
-  float* partial;          // [splits][N][16]
   NF4Table tab;
+  const __nv_bfloat16* U;   // [M, r]
+  const __nv_bfloat16* B;   // [N, r]
+  void* Y;
+  int y_bf16;
   uint32_t wait_limit;
 };
 
@@ -80,38 +100,88 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
-__global__ void __launch_bounds__(THREADS, 3)
+// Arrive on the barrier at this offset in CTA `rank`, release at cluster
+// scope: publishes this thread's (and, through a preceding warp barrier, its
+// warp's) shared-memory accesses to the other CTA.
+__device__ __forceinline__ void arrive_remote_release(uint64_t* bar, uint32_t rank) {
+  asm volatile(
+      "{\n .reg .b32 ra;\n"
+      " mapa.shared::cluster.u32 ra, %0, %1;\n"
+      " mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n}" ::"r"(smem_u32(bar)),
+      "r"(rank)
+      : "memory");
+}
+
+// (a * c, b * c), each an IEEE fp32 product rounded to nearest (one packed instruction)
+__device__ __forceinline__ void mul2_rn(float a, float b, float c, float& ra, float& rb) {
+  asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %4};\n"
+      " mul.rn.f32x2 z, x, y;\n mov.b64 {%0, %1}, z;\n}"
+      : "=f"(ra), "=f"(rb)
+      : "f"(a), "f"(b), "f"(c));
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
     smallm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
                   const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ float qtab[16];
+  __shared__ float us[TN * MAX_R];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_c = reinterpret_cast<uint64_t*>(base + STAGES * STAGE_BYTES);
-  uint64_t* full_x = full_c + STAGES;
-  uint64_t* empty_t = full_x + STAGES;   // MMA done with a TMA stage
-  uint64_t* full_a = empty_t + STAGES;   // producers stored a TMEM A sub-stage
-  uint64_t* empty_a = full_a + A_STAGES; // MMA done with a TMEM A sub-stage
-  uint64_t* acc_full = empty_a + A_STAGES;
-  uint32_t* tmem_addr = reinterpret_cast<uint32_t*>(acc_full + 1);
+  const int cs = (int)gridDim.x;                 // CTAs per cluster = K slices
+  const int q = (int)blockIdx.x;                 // this CTA's slice (its cluster rank)
+  const int kb0 = q * p.per;
+  const int per_q = min(p.per, p.kb_total - kb0);
+  const int nst = (per_q + SUB - 1) / SUB;       // code stages per tile
+  const int nt = (p.tiles - (int)blockIdx.y + (int)gridDim.y - 1) / (int)gridDim.y;   // tiles of this cluster
+  const int C = p.c_stages;
+  uint8_t* xs = base;                                            // per_q x 2 KB
+  uint8_t* cring = xs + p.per * X_SUB_BYTES;                     // C x 16 KB
+  float* red = reinterpret_cast<float*>(cring + C * C_STAGE_BYTES);   // 2 x 128 x RED_LD
+  // the 16 fp32 levels, 256-byte aligned: an LDS address is the table base
+  // with the level's byte offset (4 * code) in its low byte
+  float* qtab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(red) + 2 * RED_BYTES);
+  uint64_t* full_x = reinterpret_cast<uint64_t*>(qtab + 64);
+  uint64_t* full_c = full_x + 1;
+  uint64_t* empty_c = full_c + MAX_C_STAGES;
+  uint64_t* a_full = empty_c + MAX_C_STAGES;
+  uint64_t* a_empty = a_full + A_STAGES;
+  uint64_t* acc_full = a_empty + A_STAGES;
+  uint64_t* tmem_free = acc_full + 2;
+  uint64_t* ready = tmem_free + 2;
+  uint64_t* freed = ready + 2;
+  uint32_t* tmem_addr = reinterpret_cast<uint32_t*>(freed + 2);
   volatile int* abort_flag = reinterpret_cast<int*>(tmem_addr + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * TM;
-  const int st0 = blockIdx.y * p.stages_per_split;
-  const int nst = min(p.stages_per_split, p.stages_total - st0);
-  const int nsub = min(nst * SUB, p.sub_total - st0 * SUB);
+  auto tile_of = [&](int ti) { return (int)blockIdx.y + ti * (int)gridDim.y; };
 
   if (threadIdx.x < 16) qtab[threadIdx.x] = p.tab.q[threadIdx.x];
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
+    mbar_init(full_x, 1);
+    for (int i = 0; i < MAX_C_STAGES; ++i) {
       mbar_init(&full_c[i], 1);
-      mbar_init(&full_x[i], 1);
-      mbar_init(&empty_t[i], 1);
+      mbar_init(&empty_c[i], 1);
     }
     for (int i = 0; i < A_STAGES; ++i) {
-      mbar_init(&full_a[i], PRODUCER_WARPS);
-      mbar_init(&empty_a[i], 1);
+      mbar_init(&a_full[i], GROUP_WARPS);
+      mbar_init(&a_empty[i], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&tmem_free[i], DRAIN_WARPS);
+      mbar_init(&ready[i], cs * DRAIN_WARPS);
+      mbar_init(&freed[i], cs * DRAIN_WARPS);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -120,173 +190,268 @@ __global__ void __launch_bounds__(THREADS, 3)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // every CTA's barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem = *tmem_addr;
   pdl_wait();
   pdl_trigger();
 
   if (warp == 0) {
+    // ------------------------------------------------------------ TMA warp
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
       prefetch_tmap(&tmap_codes);
+      mbar_arrive_expect_tx(full_x, per_q * X_SUB_BYTES);
+      for (int j = 0; j < per_q; ++j) tma_load_2d(xs + j * X_SUB_BYTES, &tmap_x, full_x, (kb0 + j) * BK, 0);
       int issued = 0;
-      for (int i = 0; i < nst; ++i) {
-        const int s = i % STAGES, use = i / STAGES;
-        if (use > 0 && !mbar_wait(&empty_t[s], (use - 1) & 1, abort_flag, p.wait_limit)) break;
-        const int kst = st0 + i;
-        uint8_t* st = base + s * STAGE_BYTES;
-        mbar_arrive_expect_tx(&full_c[s], C_BYTES);
-        tma_load_2d(st, &tmap_codes, &full_c[s], kst * (SUB * BK / 2), n0);
-        mbar_arrive_expect_tx(&full_x[s], SUB * X_SUB_BYTES);
-#pragma unroll
-        for (int u = 0; u < SUB; ++u)
-          tma_load_2d(st + C_BYTES + u * X_SUB_BYTES, &tmap_x, &full_x[s], (kst * SUB + u) * BK, 0);
-        issued = i + 1;
+      bool ok = true;
+      for (int ti = 0; ti < nt && ok; ++ti) {
+        for (int st = 0; st < nst; ++st) {
+          const int g = ti * nst + st, cslot = g % C;
+          if (g >= C && !mbar_wait(&empty_c[cslot], ((g / C) - 1) & 1, abort_flag, p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_c[cslot], C_STAGE_BYTES);
+          tma_load_2d(cring + cslot * C_STAGE_BYTES, &tmap_codes, &full_c[cslot], (kb0 + st * SUB) * (BK / 2),
+                      tile_of(ti) * TM);
+          issued = g + 1;
+        }
       }
-      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
-        mbar_wait(&full_c[i % STAGES], (i / STAGES) & 1, abort_flag, 1u << 22);
-        mbar_wait(&full_x[i % STAGES], (i / STAGES) & 1, abort_flag, 1u << 22);
-      }
+      // before leaving, make sure no copy is still landing in shared memory
+      mbar_wait(full_x, 0, abort_flag, p.wait_limit);
+      for (int g = (issued > C ? issued - C : 0); g < issued; ++g)
+        mbar_wait(&full_c[g % C], (g / C) & 1, abort_flag, p.wait_limit);
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(TM, TN, false, false);
-      bool ok = true;
-      for (int j = 0; j < nsub && ok; ++j) {
-        const int i = j / SUB, u = j % SUB;
-        const int s = i % STAGES, use = i / STAGES;
-        const int sa = j % A_STAGES, usea = j / A_STAGES;
-        ok = (u != 0 || mbar_wait(&full_x[s], use & 1, abort_flag, p.wait_limit)) &&
-             mbar_wait(&full_a[sa], usea & 1, abort_flag, p.wait_limit);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t x_addr = smem_u32(base + s * STAGE_BYTES + C_BYTES + u * X_SUB_BYTES);
-        const uint32_t a_col = A_COL0 + sa * 32;
+      bool ok = mbar_wait(full_x, 0, abort_flag, p.wait_limit);
+      for (int ti = 0; ti < nt && ok; ++ti) {
+        const int b = ti & 1;
+        if (ti >= 2) ok = mbar_wait(&tmem_free[b], ((ti >> 1) - 1) & 1, abort_flag, p.wait_limit);
+        // one A stage = one code stage: up to four 64-deep sub-steps, 16 MMAs
+        for (int st = 0; st < nst && ok; ++st) {
+          const int G = ti * nst + st, aslot = G % A_STAGES;
+          ok = mbar_wait(&a_full[aslot], (G / A_STAGES) & 1, abort_flag, p.wait_limit);
+          if (!ok) break;
+          tc_fence_after();
+          const int nsub = min(SUB, per_q - st * SUB);
+          for (int u = 0; u < nsub; ++u) {
+            const int j = st * SUB + u;
+            const uint32_t x_addr = smem_u32(xs + j * X_SUB_BYTES);
+            const uint32_t a_col = A_COL0 + aslot * A_STAGE_COLS + u * 32;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          mma_ts(tmem, tmem + a_col + kk * 8, sdesc_sw128(x_addr + kk * 32, 16, 1024), idesc, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&empty_a[sa]);
-        if (u == SUB - 1 || j == nsub - 1) mma_commit(&empty_t[s]);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_ts(tmem + 16 * b, tmem + a_col + kk * 8, sdesc_sw128(x_addr + kk * 32, 16, 1024), idesc,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&a_empty[aslot]);
+          mma_commit(&empty_c[G % C]);
+        }
+        if (ok) mma_commit(&acc_full[b]);
       }
-      mma_commit(acc_full);
     }
-  } else {
-    // producers: warp w covers TMEM lanes 32*(w&3)..+31 (weight rows) and the
-    // half (w-2)>>2 of the 64 codes of each row's block in a sub-step
+  } else if (warp < DRAIN_WARP0) {
+    // ------------------------------------------------------ dequant producers
+    // group grp expands the A stages G = grp, grp+2, ... of this CTA's
+    // sequence (tile by tile; one A stage = the up to four 64-deep sub-steps
+    // of one code stage); warp: TMEM lanes 32*(warp&3) (weight rows) and half
+    // of the 64 codes of each sub-step
+    const int grp = (warp - 2) / GROUP_WARPS;
+    const int half = ((warp - 2) >> 2) & 1;
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
-    const int wrow = n0 + row;
-    const bool valid = wrow < p.N;
-    const int kblocks = p.K / 64;
     const float mu = p.wc.absmax ? 0.0f : *p.wc.offset;
-    const char* qb = reinterpret_cast<const char*>(qtab);
-    // block constant, loaded one sub-step ahead
-    auto load_c = [&](int j) -> float2 {
-      float2 r = make_float2(0.0f, 0.0f);
-      if (!valid || j >= nsub) return r;
-      const int64_t b = (int64_t)wrow * kblocks + (int64_t)st0 * SUB + j;
-      if (p.wc.absmax) r.x = __ldg(p.wc.absmax + b);
-      else { r.x = __ldg(p.wc.scale2 + (b >> 8)); r.y = __uint_as_float((uint32_t)__ldg(p.wc.absmax_q + b)); }
-      return r;
+    const uint32_t qbase = smem_u32(qtab);   // low byte 0
+    // block constants of the sub-steps of stage st of tile ti (raw: absmax, or
+    // scale2 and the E4M3 code)
+    auto load_c = [&](int ti, int st, float2 (&r)[SUB]) {
+#pragma unroll
+      for (int u = 0; u < SUB; ++u) r[u] = make_float2(0.0f, 0.0f);
+      if (ti >= nt) return;
+      const int n = tile_of(ti) * TM + row;
+      if (n >= p.N) return;
+#pragma unroll
+      for (int u = 0; u < SUB; ++u) {
+        const int j = st * SUB + u;
+        if (j >= per_q) break;
+        const int64_t b = (int64_t)n * p.kb_total + kb0 + j;
+        if (p.wc.absmax) r[u].x = __ldg(p.wc.absmax + b);
+        else { r[u].x = __ldg(p.wc.scale2 + (b >> 8)); r[u].y = __uint_as_float((uint32_t)__ldg(p.wc.absmax_q + b)); }
+      }
     };
-    float2 nxt = load_c(0);
+    // (tile, stage) two stages further on: this group's next stage
+    auto advance2 = [&](int& ti, int& st) {
+      st += 2;
+      while (st >= nst) { st -= nst; ++ti; }
+    };
+    int ti = 0, st = grp;
+    while (st >= nst) { st -= nst; ++ti; }
+    int nti = ti, nst2 = st;
+    advance2(nti, nst2);
+    float2 cur[SUB], nxt[SUB];
+    load_c(ti, st, cur);
     bool ok = true;
-    for (int j = 0; j < nsub && ok; ++j) {
-      const int i = j / SUB, u = j % SUB;
-      const int s = i % STAGES, use = i / STAGES;
-      const int sa = j % A_STAGES, usea = j / A_STAGES;
-      const float2 cur = nxt;
-      nxt = load_c(j + 1);
-      ok = __all_sync(0xffffffffu, mbar_wait(&full_c[s], use & 1, abort_flag, p.wait_limit) &&
-                                       (usea == 0 || mbar_wait(&empty_a[sa], (usea - 1) & 1, abort_flag, p.wait_limit)));
+    for (int G = grp; ti < nt && ok; G += 2) {
+      const int cslot = G & (C - 1);
+      const int aslot = G % A_STAGES;
+      const bool valid = tile_of(ti) * TM + row < p.N;
+      const int nsub = min(SUB, per_q - st * SUB);
+      load_c(nti, nst2, nxt);
+      ok = __all_sync(0xffffffffu, mbar_wait(&full_c[cslot], (G >> p.c_log) & 1, abort_flag, p.wait_limit) &&
+                                       (G < A_STAGES ||
+                                        mbar_wait(&a_empty[aslot], ((G / A_STAGES) - 1) & 1, abort_flag, p.wait_limit)));
       if (!ok) break;
       tc_fence_after();
-      uint32_t out[16];
-      if (valid) {
-        const float c = p.wc.absmax ? cur.x
-                                    : __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)__float_as_uint(cur.y)), cur.x), mu);
-        // 128-byte code rows with the 128B swizzle: 16-byte chunk ^= row mod 8
-        const uint32_t coff = row * 128 + (((2 * u + half) ^ (row & 7)) << 4);
-        const uint4 cw = *reinterpret_cast<const uint4*>(base + s * STAGE_BYTES + coff);
-        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+      const uint8_t* cst = cring + cslot * C_STAGE_BYTES;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint32_t e4 = (w[q4] << 2) & 0x3C3C3C3Cu;   // 4 * low nibble of each byte
-          const uint32_t o4 = (w[q4] >> 2) & 0x3C3C3C3Cu;   // 4 * high nibble of each byte
+      for (int u = 0; u < SUB; ++u) {
+        if (u >= nsub) break;
+        uint32_t out[16];
+        if (valid) {
+          const float c = p.wc.absmax ? cur[u].x
+                                      : __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)__float_as_uint(cur[u].y)), cur[u].x), mu);
+          // 128-byte code rows with the 128B swizzle: 16-byte chunk ^= row mod 8
+          const uint32_t coff = row * 128 + (((2 * u + half) ^ (row & 7)) << 4);
+          const uint4 cw = *reinterpret_cast<const uint4*>(cst + coff);
+          const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const uint32_t ae = __byte_perm(e4, 0u, 0x4440u | b);
-            const uint32_t ao = __byte_perm(o4, 0u, 0x4440u | b);
-            const float fe = *reinterpret_cast<const float*>(qb + ae);
-            const float fo = *reinterpret_cast<const float*>(qb + ao);
-            out[4 * q4 + b] = pack_bf16x2(__fmul_rn(fe, c), __fmul_rn(fo, c));
+          for (int q4 = 0; q4 < 4; ++q4) {
+            // element i of the word is nibble i; its level sits at qbase + 4 * nibble
+            const uint32_t e4 = (w[q4] << 2) & 0x3C3C3C3Cu;   // 4 * low nibble of each byte
+            const uint32_t o4 = (w[q4] >> 2) & 0x3C3C3C3Cu;   // 4 * high nibble of each byte
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+              // byte bb of e4 / o4 under the table base's upper three bytes
+              const float fe = lds_f32(__byte_perm(e4, qbase, 0x7650u | bb));
+              const float fo = lds_f32(__byte_perm(o4, qbase, 0x7650u | bb));
+              float pe, po;
+              mul2_rn(fe, fo, c, pe, po);
+              out[4 * q4 + bb] = pack_bf16x2(pe, po);
+            }
           }
-        }
-      } else {
+        } else {
 #pragma unroll
-        for (int t = 0; t < 16; ++t) out[t] = 0u;
+          for (int t = 0; t < 16; ++t) out[t] = 0u;
+        }
+        tmem_st16(tmem + ((uint32_t)(quad * 32) << 16) +
+                      (uint32_t)(A_COL0 + aslot * A_STAGE_COLS + u * 32 + half * 16),
+                  out);
       }
-      tmem_st16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(A_COL0 + sa * 32 + half * 16), out);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full_a[sa]);
-    }
-    // drain: warps 2-5 read the 128 x 16 accumulator and write the partial
-    if (half == 0) {
-      const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.wait_limit) && !*abort_flag);
-      if (acc_ok) {
-        tc_fence_after();
-        uint32_t v[16];
-        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16), v);
-        tmem_ld_wait();
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)blockIdx.y * p.N + wrow) * TN);
+      if (lane == 0) mbar_arrive(&a_full[aslot]);
 #pragma unroll
-          for (int t = 0; t < 4; ++t)
-            dst[t] = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]), __uint_as_float(v[4 * t + 2]),
-                                 __uint_as_float(v[4 * t + 3]));
+      for (int u = 0; u < SUB; ++u) cur[u] = nxt[u];
+      ti = nti;
+      st = nst2;
+      advance2(nti, nst2);
+    }
+  } else {
+    // ---------------------------------------- drain, cluster reduction, output
+    const int t = threadIdx.x - DRAIN_WARP0 * 32;   // 0..127
+    const int quad = warp & 3;
+    const int drow = quad * 32 + lane;              // the TMEM lane this thread drains
+    for (int i = t; i < p.M * p.r; i += DRAIN_WARPS * 32) us[i] = __bfloat162float(p.U[i]);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // this CTA's share of the tile's (row, token pair) outputs, token pair fastest
+    const int items = TM * (TN / 2);
+    const int i0 = items * q / cs, i1 = items * (q + 1) / cs;
+    // adapter row of an item, 16-byte loads issued together
+    uint4 bv[MAX_R / 8];
+    auto load_brow = [&](int n) {
+#pragma unroll
+      for (int c8 = 0; c8 < MAX_R / 8; ++c8)
+        if (c8 * 8 < p.r && n < p.N) bv[c8] = *reinterpret_cast<const uint4*>(p.B + (size_t)n * p.r + c8 * 8);
+    };
+    bool ok = true;
+    for (int ti = 0; ti < nt && ok; ++ti) {
+      const int b = ti & 1;
+      const int n0 = tile_of(ti) * TM;
+      float* rb = red + b * (TM * RED_LD);
+      // the first item's adapter row is fetched while the tile is still being computed
+      if (p.r > 0 && i0 + t < i1) load_brow(n0 + ((i0 + t) >> 3));
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], (ti >> 1) & 1, abort_flag, p.wait_limit));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v[16];
+      tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(16 * b), v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tmem_free[b]);
+      // the other CTAs are done reading this buffer's previous tile
+      if (ti >= 2) ok = __all_sync(0xffffffffu, mbar_wait_cluster(&freed[b], ((ti >> 1) - 1) & 1, abort_flag, p.wait_limit));
+      if (!ok) break;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<float2*>(rb + drow * RED_LD + 2 * k) =
+            make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+      __syncwarp();
+      if (lane == 0)
+        for (int pr = 0; pr < cs; ++pr) arrive_remote_release(&ready[b], (uint32_t)pr);
+      ok = __all_sync(0xffffffffu, mbar_wait_cluster(&ready[b], (ti >> 1) & 1, abort_flag, p.wait_limit));
+      if (!ok) break;
+      const uint32_t rb_addr = smem_u32(rb);
+      for (int it = i0 + t; it < i1; it += DRAIN_WARPS * 32) {
+        const int r_in = it >> 3, tp = it & 7;
+        const int n = n0 + r_in, m0 = 2 * tp;
+        if (p.r > 0 && it != i0 + t) load_brow(n);
+        if (n >= p.N || m0 >= p.M) continue;
+        const uint32_t off = rb_addr + (uint32_t)((r_in * RED_LD + m0) * 4);
+        // every slice's partial in flight at once, added in slice order
+        float2 x[MAX_CS];
+#pragma unroll
+        for (int pr = 0; pr < MAX_CS; ++pr)
+          if (pr < cs) x[pr] = ld_cluster_f2(cluster_map(off, (uint32_t)pr));
+        float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int pr = 0; pr < MAX_CS; ++pr)
+          if (pr < cs) {
+            acc.x = __fadd_rn(acc.x, x[pr].x);
+            acc.y = __fadd_rn(acc.y, x[pr].y);
+          }
+        float o[2] = {acc.x, acc.y};
+        if (p.r > 0) {
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm) {
+            if (m0 + mm >= p.M) break;
+            const float* um = us + (m0 + mm) * p.r;
+            float l = 0.0f;
+#pragma unroll
+            for (int c8 = 0; c8 < MAX_R / 8; ++c8) {
+              if (c8 * 8 >= p.r) break;
+              const uint32_t bw[4] = {bv[c8].x, bv[c8].y, bv[c8].z, bv[c8].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                l = fmaf(um[c8 * 8 + 2 * e], bf16_lo(bw[e]), l);
+                l = fmaf(um[c8 * 8 + 2 * e + 1], bf16_hi(bw[e]), l);
+              }
+            }
+            o[mm] = __fadd_rn(o[mm], __fmul_rn(p.s, l));
+          }
+        }
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm) {
+          if (m0 + mm >= p.M) break;
+          const size_t yo = (size_t)(m0 + mm) * p.N + n;
+          if (p.y_bf16) reinterpret_cast<__nv_bfloat16*>(p.Y)[yo] = __float2bfloat16_rn(o[mm]);
+          else reinterpret_cast<float*>(p.Y)[yo] = o[mm];
         }
       }
+      __syncwarp();
+      if (lane == 0)
+        for (int pr = 0; pr < cs; ++pr) arrive_remote_release(&freed[b], (uint32_t)pr);
     }
   }
-  if (warp == 1 && lane == 0 && *abort_flag) mbar_wait(acc_full, 0, abort_flag, 1u << 22);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // no CTA leaves while another may still read its shared memory or arrive on its barriers
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
-  }
-}
-
-// One thread per output (m, n), m fastest: Y[m][n] = sum over splits (fixed
-// order) of partial[split][n][m] + s * sum_j U[m][j] * B[n][j], in fp32.
-__global__ void __launch_bounds__(256) smallm_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N,
-                                                            const __nv_bfloat16* __restrict__ U,
-                                                            const __nv_bfloat16* __restrict__ B, int r, float s,
-                                                            int out_bf16, void* __restrict__ Y) {
-  pdl_wait();
-  pdl_trigger();
-  __shared__ float us[TN * 64];
-  for (int i = threadIdx.x; i < M * r; i += blockDim.x) us[i] = __bfloat162float(U[i]);
-  __syncthreads();
-  const int64_t total = (int64_t)N * M;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int n = (int)(idx / M), m = (int)(idx % M);
-    float acc = 0.0f;
-    for (int sp = 0; sp < splits; ++sp) acc = __fadd_rn(acc, partial[((int64_t)sp * N + n) * TN + m]);
-    if (r > 0) {
-      float l = 0.0f;
-      const __nv_bfloat16* brow = B + (int64_t)n * r;
-      for (int j = 0; j < r; ++j) l = fmaf(us[m * r + j], __bfloat162float(brow[j]), l);
-      acc = __fadd_rn(acc, __fmul_rn(s, l));
-    }
-    const int64_t o = (int64_t)m * N + n;
-    if (out_bf16) reinterpret_cast<__nv_bfloat16*>(Y)[o] = __float2bfloat16_rn(acc);
-    else reinterpret_cast<float*>(Y)[o] = acc;
   }
 }
 
@@ -303,32 +468,114 @@ static int sm_count_sm() {
   return count;
 }
 
-static void smallm_plan(int64_t N, int64_t K, int& splits, int& per) {
-  const int tiles = (int)((N + smallm::TM - 1) / smallm::TM);
-  const int stages = (int)((K + smallm::BK * smallm::SUB - 1) / (smallm::BK * smallm::SUB));
-  // three resident CTAs per SM, about two work units each
-  int want = std::max(1, (6 * sm_count_sm() + tiles - 1) / tiles);
-  want = std::min(want, stages);
-  per = (stages + want - 1) / want;
-  splits = (stages + per - 1) / per;
-}
+struct SmallmPlan {
+  int cs, per, c_stages, c_log, clusters;
+  size_t smem;
+};
 
-size_t smallm_partial_bytes(int64_t N, int64_t K) {
-  int splits, per;
-  smallm_plan(N, K, splits, per);
-  return (size_t)splits * N * smallm::TN * sizeof(float);
-}
+static size_t smallm_static_smem() { return sizeof(float) * (smallm::TN * smallm::MAX_R); }
 
-// Y = X W_hat^T + s U B^T for M <= 16; U [M, r] given (bf16), partial from the workspace.
-ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
-                            float s, void* Y, ql_dtype y_dt, float* partial, cudaStream_t st) {
+// Shared memory for a K slice of `per` sub-steps; false if it cannot fit.
+static bool smallm_layout(int per, SmallmPlan& pl) {
   using namespace smallm;
-  static bool attr_set = false;
-  if (!attr_set) {
-    QL_CUDA_TRY(cudaFuncSetAttribute(smallm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
-    attr_set = true;
+  if (per > MAX_PER) return false;
+  // alignment slack, the X slice, two reduction buffers, the level table,
+  // 33 mbarriers + TMEM address + abort flag
+  const size_t fixed = 1024 + (size_t)per * X_SUB_BYTES + 2 * RED_BYTES + 256 + 512;
+  const size_t limit = 227 * 1024 - smallm_static_smem();
+  if (fixed + 2 * C_STAGE_BYTES > limit) return false;
+  int c = 2, lg = 1;
+  while (c * 2 <= MAX_C_STAGES && fixed + (size_t)(c * 2) * C_STAGE_BYTES <= limit) {
+    c *= 2;
+    ++lg;
   }
+  pl.per = per;
+  pl.c_stages = c;
+  pl.c_log = lg;
+  pl.smem = fixed + (size_t)c * C_STAGE_BYTES;
+  return true;
+}
+
+static bool smallm_attr() {
+  static bool set = false;
+  if (!set) {
+    if (cudaFuncSetAttribute(smallm::smallm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(227 * 1024 - smallm_static_smem())) != cudaSuccess)
+      return false;
+    set = true;
+  }
+  return true;
+}
+
+// Cluster size (CTAs sharing K) and cluster count: the tiles are handed out in
+// rounds of `clusters`, each round costing about `per` sub-steps, so pick the
+// split with the fewest rounds x per among the cluster sizes that fit (the
+// cluster count comes from the occupancy calculator: a cluster's CTAs must
+// share a GPC, which caps it below SMs / cs).
+static bool smallm_plan(int64_t N, int64_t K, SmallmPlan& best, bool query) {
+  using namespace smallm;
+  const int kb = (int)(K / BK);
+  if (kb < 1) return false;
+  const int tiles = (int)((N + TM - 1) / TM);
+  bool found = false;
+  long best_cost = 0;
+  for (int cs0 = std::min(MAX_CS, kb); cs0 >= 1; --cs0) {
+    SmallmPlan pl;
+    const int per = (kb + cs0 - 1) / cs0;
+    if (!smallm_layout(per, pl)) continue;
+    pl.cs = (kb + per - 1) / per;
+    int maxc = sm_count_sm() / pl.cs;
+    if (query) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)pl.cs, (unsigned)std::max(1, maxc));
+      cfg.blockDim = dim3(THREADS);
+      cfg.dynamicSmemBytes = pl.smem;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = (unsigned)pl.cs;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, smallm_kernel, &cfg) == cudaSuccess && n > 0) maxc = std::min(maxc, n);
+      else cudaGetLastError();
+    }
+    pl.clusters = std::max(1, std::min(tiles, maxc));
+    const long rounds = (tiles + pl.clusters - 1) / pl.clusters;
+    const long cost = rounds * per;
+    if (!found || cost < best_cost) {
+      best = pl;
+      best_cost = cost;
+      found = true;
+    }
+  }
+  return found;
+}
+
+// Whether the small-token kernel handles this shape (its K slice of X must fit
+// in shared memory: K <= 40960 with eight slices).
+bool smallm_supported(int64_t N, int64_t K) {
+  SmallmPlan pl;
+  return smallm_plan(N, K, pl, false);
+}
+
+// Y = X W_hat^T + s U B^T for M <= 16; U [M, r] given (bf16).
+ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
+                            float s, void* Y, ql_dtype y_dt, cudaStream_t st) {
+  using namespace smallm;
+  if (M < 1 || M > TN || r > MAX_R) return QL_ERR_UNSUPPORTED;
   const int N = (int)w->rows, K = (int)w->cols;
+  if (!smallm_attr()) return QL_ERR_CUDA;
+  // the plan for a weight shape is fixed, so it is computed once per shape
+  static int64_t cached_N = -1, cached_K = -1;
+  static SmallmPlan cached;
+  if (N != cached_N || K != cached_K) {
+    if (!smallm_plan(N, K, cached, true)) return QL_ERR_UNSUPPORTED;
+    cached_N = N;
+    cached_K = K;
+  }
+  const SmallmPlan pl = cached;
   CUtensorMap map_x, map_codes;
   if (!make_map_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, TN,
                    CU_TENSOR_MAP_SWIZZLE_128B))
@@ -336,33 +583,27 @@ ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, co
   if (!make_map_2d(&map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, (uint64_t)K / 2, (uint64_t)N,
                    (uint64_t)K / 2, SUB * BK / 2, TM, CU_TENSOR_MAP_SWIZZLE_128B))
     return QL_ERR_CUDA;
-  int splits, per;
-  smallm_plan(N, K, splits, per);
   Params p;
   p.M = (int)M;
   p.N = N;
   p.K = K;
-  p.stages_total = (K + BK * SUB - 1) / (BK * SUB);
-  p.sub_total = K / BK;
-  p.stages_per_split = per;
+  p.r = r;
+  p.kb_total = K / BK;
+  p.per = pl.per;
+  p.tiles = (N + TM - 1) / TM;
+  p.c_stages = pl.c_stages;
+  p.c_log = pl.c_log;
+  p.s = s;
   p.wc = WeightConsts{w->absmax, w->absmax_q, w->scale2, w->offset};
-  p.partial = partial;
   p.tab = nf4_table();
+  p.U = (const __nv_bfloat16*)U;
+  p.B = (const __nv_bfloat16*)B;
+  p.Y = Y;
+  p.y_bf16 = y_dt == QL_BF16;
   p.wait_limit = 1u << 22;
-  dim3 grid((unsigned)((N + TM - 1) / TM), (unsigned)splits);
-  {
-    TraceScope ts(TK_SMALLM, st);
-    QL_CUDA_TRY(launch(smallm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, st, 1, 1, map_x, map_codes, p));
-  }
-  QL_LAUNCH_CHECK();
-  const unsigned rg =
-      (unsigned)std::max<int64_t>(1, std::min<int64_t>((M * (int64_t)N + 255) / 256, (int64_t)sm_count_sm() * 8));
-  {
-    TraceScope ts(TK_COLACC_REDUCE, st);
-    QL_CUDA_TRY(launch(smallm_reduce_kernel, dim3(rg), dim3(256), 0, st, 1, 1, partial, splits, (int)M, N, (const __nv_bfloat16*)U,
-                                             (const __nv_bfloat16*)B, r, s, y_dt == QL_BF16, Y));
-  }
-  QL_LAUNCH_CHECK();
+  TraceScope ts(TK_SMALLM, st);
+  QL_CUDA_TRY(launch(smallm_kernel, dim3((unsigned)pl.cs, (unsigned)pl.clusters), dim3(THREADS), pl.smem, st,
+                     (unsigned)pl.cs, 1, map_x, map_codes, p));
   return QL_OK;
 }
 

@@ -241,6 +241,18 @@ void qlora_trace_enable_kinds(unsigned mask);
 int qlora_trace_read(double* total_ms, int* launches, int max_kinds);
 const char* qlora_trace_kind_name(int kind);
 
+/*
+ * Failure-detection self-test (no counterpart on the pages).  Every pipelined
+ * kernel of the library waits on mbarriers with a bounded number of polls
+ * (each poll suspends at most about 1 us); a wait that runs out records
+ * QL_ERR_TIMEOUT in the device status word and the kernel returns instead of
+ * hanging.  This entry point launches one CTA whose wait nothing ever
+ * satisfies, limited to `polls` polls, on `stream`; the next qlora_get_status
+ * returns QL_ERR_TIMEOUT and the CUDA context stays usable.
+ * polls: 1 .. 2^20 (QL_ERR_INVALID_ARG otherwise).  Allocates nothing.
+ */
+ql_status qlora_selftest_wait_timeout(int64_t polls, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* qlora_status_string(ql_status s);
 

@@ -82,3 +82,5 @@ def test_argument_errors_return_before_launch(lib):
                               fake, fake, lib.QL_F32, fake, 0, s0) == lib.QL_ERR_WORKSPACE
     assert L.nf4_dequant(None, fake, lib.QL_BF16, s0) == lib.QL_ERR_INVALID_ARG
     assert lib.status_string(lib.QL_ERR_TIMEOUT) == "device wait timed out"
+    for polls in (0, -1, (1 << 20) + 1):
+        assert L.qlora_selftest_wait_timeout(polls, s0) == lib.QL_ERR_INVALID_ARG
