@@ -328,6 +328,92 @@ def small_m_and_codec(q, dev, hbm_peak):
                              "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3), "bytes": moved}
     del x, codes, absmax, aq
     torch.cuda.empty_cache()
+    out.update(large_token_legs(q, dev))
+    return out
+
+
+def _time_calls(fn, flush, n_warm=2, n=5):
+    import torch
+    for _ in range(n_warm):
+        fn()
+    times = []
+    for _ in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times) / 1e3
+
+
+def large_token_legs(q, dev):
+    """The other two large-token workloads, forward + backward: the 7B MLP block
+    (gate/up 11008 x 4096, down 4096 x 11008, 8192 tokens, r = 64, SiLU-gated)
+    and the seven 70B-shaped layer linears (2048 tokens, r = 16), each step
+    timed whole with CUDA events; TFLOP/s counts 4MNK + 6Mr(K+N) per linear."""
+    import torch
+    from synthetic import inputs as S
+    from bit_nf4_quantized_10_b200.mlp import QLoRAMLP
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # 7B MLP
+    w3 = S.WORKLOADS["c3"]
+    D, H, M, r, s = 4096, 11008, w3.M, w3.r, w3.s
+    ws = [q.quantize_weight(S.custom_weight(n, k, w3.wstd, 3000 + i, device=dev), dq=True)
+          for i, (n, k) in enumerate(((H, D), (H, D), (D, H)))]
+    Ag = S.uniform((r, D), 1 / D ** 0.5, 3003, device=dev)
+    Au = S.uniform((r, D), 1 / D ** 0.5, 3004, device=dev)
+    Ad = S.uniform((r, H), 1 / H ** 0.5, 3005, device=dev)
+    Bg = S.normal((H, r), 0.01, 3006, device=dev, dtype=torch.bfloat16)
+    Bu = S.normal((H, r), 0.01, 3007, device=dev, dtype=torch.bfloat16)
+    Bd = S.normal((D, r), 0.01, 3008, device=dev, dtype=torch.bfloat16)
+    X = S.normal((M, D), 1.0, 3009, device=dev, dtype=torch.bfloat16)
+    dy = S.normal((M, D), 1.0, 3010, device=dev, dtype=torch.bfloat16)
+    mlp = QLoRAMLP(ws[0], ws[1], ws[2], Ag, Bg, Au, Bu, Ad, Bd, r, s, M)
+    y = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+
+    def mlp_step():
+        mlp.forward(X, y)
+        mlp.backward(X, dy)
+
+    t = _time_calls(mlp_step, flush)
+    out["mlp_7b"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(mlp.flops() / t / 1e12, 1),
+                     "tokens": M, "r": r}
+    del mlp, ws, X, dy, y
+    torch.cuda.empty_cache()
+    # 70B-shaped layer linears
+    w4 = S.WORKLOADS["c4"]
+    M, r, s = w4.M, w4.r, w4.s
+    legs, flops = [], 0.0
+    for j, lin in enumerate(w4.linears):
+        d = S.linear_inputs(w4, j, device=dev)
+        wq = q.quantize_weight(d["W"], dq=True)
+        del d["W"]
+        N, K = lin.N, lin.K
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        U = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+        dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        dA = torch.empty(r, K, dtype=torch.float32, device=dev)
+        dB = torch.empty(N, r, dtype=torch.float32, device=dev)
+        wsb = torch.empty(max(q.qlora_workspace_size(q.QL_OP_FWD, M, N, K, r),
+                              q.qlora_workspace_size(q.QL_OP_BWD, M, N, K, r), 16), dtype=torch.uint8, device=dev)
+        legs.append((wq, d, Y, U, dX, dA, dB, wsb))
+        flops += 4.0 * M * N * K + 6.0 * M * r * (K + N)
+
+    def layer_step():
+        for wq, d, Y, U, dX, dA, dB, wsb in legs:
+            q.qlora_linear_fwd(wq, d["X"], d["A"], d["B"], r, s, Y, U_out=U, ws=wsb)
+            q.qlora_linear_bwd(wq, d["X"], d["dY"], d["A"], d["B"], r, s, U, dX, dA, dB, ws=wsb)
+
+    t = _time_calls(layer_step, flush)
+    out["layer_70b_linears"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(flops / t / 1e12, 1), "tokens": M, "r": r}
+    st = q.qlora_get_status()
+    if st != q.QL_OK:
+        raise RuntimeError(f"device status after the large-token legs: {q.status_string(st)}")
+    del legs
+    torch.cuda.empty_cache()
     return out
 
 
