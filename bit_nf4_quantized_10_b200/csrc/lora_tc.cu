@@ -18,6 +18,8 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -228,16 +230,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// dst [cols, ld_dst] = src [rows, cols]^T (bf16, cols = r <= 64).
+// dst [cols, ld_dst] = src [rows, cols]^T (bf16, cols = r <= 64, a multiple of
+// 8): one thread per source row reads it with 16-byte loads; for each output
+// row the warp's 32 consecutive source rows give 64 contiguous bytes.
 __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ src, int rows, int cols,
                                                         uint16_t* __restrict__ dst, int ld_dst) {
   pdl_wait();
   pdl_trigger();
-  const int64_t total = (int64_t)rows * cols;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t j = idx / rows, row = idx % rows;
-    dst[j * ld_dst + row] = src[row * cols + j];
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= rows) return;
+  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)row * cols);
+  for (int c8 = 0; c8 < cols / 8; ++c8) {
+    const uint4 v = s[c8];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      dst[(size_t)(c8 * 8 + 2 * e) * ld_dst + row] = (uint16_t)(w[e] & 0xFFFFu);
+      dst[(size_t)(c8 * 8 + 2 * e + 1) * ld_dst + row] = (uint16_t)(w[e] >> 16);
+    }
   }
 }
 
@@ -254,15 +264,60 @@ static int sm_count_tc() {
   return count;
 }
 
-// One wave of CTAs (two per SM) where the row tiles allow, at most
-// MAX_SPLITS CTAs per tile (one cluster), each split a whole number of steps.
-static void split_plan(int rows, int64_t red, int& splits, int& per) {
+// One wave of clusters where the row tiles allow: the most splits (at most
+// MAX_SPLITS, one cluster of CTAs per row tile) such that every tile's cluster
+// is resident at once, per the occupancy calculator (a cluster's CTAs share a
+// GPC); each split a whole number of 64-deep steps.
+static void split_plan_compute(bool a_mn, int rows, int64_t red, int& splits, int& per) {
   const int tiles = (rows + skinny::BM - 1) / skinny::BM;
   const int steps = (int)((red + skinny::BK - 1) / skinny::BK);
-  int want = 2 * sm_count_tc() / tiles;
-  want = std::max(1, std::min(std::min(want, steps), skinny::MAX_SPLITS));
+  int want = std::max(1, std::min(std::min(2 * sm_count_tc() / tiles, steps), skinny::MAX_SPLITS));
+  for (; want > 1; --want) {
+    const int pw = (steps + want - 1) / want;
+    const int sp = (steps + pw - 1) / pw;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)tiles, (unsigned)sp);
+    cfg.blockDim = dim3(skinny::THREADS);
+    cfg.dynamicSmemBytes = skinny::SMEM_BYTES;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = (unsigned)sp;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = a_mn ? cudaOccupancyMaxActiveClusters(&n, skinny::skinny_kernel<true>, &cfg)
+                               : cudaOccupancyMaxActiveClusters(&n, skinny::skinny_kernel<false>, &cfg);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      break;   // no answer: keep the arithmetic choice
+    }
+    if (n >= tiles) break;
+  }
   per = (steps + want - 1) / want;
   splits = (steps + per - 1) / per;
+}
+
+// The plan depends only on the shape; launches repeat the same few shapes.
+static void split_plan(bool a_mn, int rows, int64_t red, int& splits, int& per) {
+  struct Entry {
+    bool a_mn;
+    int rows;
+    int64_t red;
+    int splits, per;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  std::lock_guard<std::mutex> lk(mu);
+  for (const Entry& e : cache)
+    if (e.a_mn == a_mn && e.rows == rows && e.red == red) {
+      splits = e.splits;
+      per = e.per;
+      return;
+    }
+  split_plan_compute(a_mn, rows, red, splits, per);
+  if (cache.size() < 256) cache.push_back(Entry{a_mn, rows, red, splits, per});
 }
 
 // C = scale * Z_op G, see the file comment.  a_mn: Z_op is the transpose of a
@@ -275,8 +330,10 @@ static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, 
   using namespace skinny;
   static bool attr[2] = {false, false};
   if (!attr[a_mn]) {
-    if (a_mn) QL_CUDA_TRY(cudaFuncSetAttribute(skinny_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
-    else QL_CUDA_TRY(cudaFuncSetAttribute(skinny_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
+    // two CTAs per SM need the largest shared-memory carveout
+    auto k = a_mn ? skinny_kernel<true> : skinny_kernel<false>;
+    QL_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
+    QL_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     attr[a_mn] = true;
   }
   const int rp = (r + 15) / 16 * 16;
@@ -294,7 +351,7 @@ static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, 
                    (uint32_t)rp, CU_TENSOR_MAP_SWIZZLE_128B))
     return QL_ERR_CUDA;
   int splits, per;
-  split_plan(rows, red, splits, per);
+  split_plan(a_mn, rows, red, splits, per);
   const int tiles = (rows + BM - 1) / BM;
   Params p;
   p.rows = rows;
@@ -339,11 +396,11 @@ ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t
 
 // dst [cols, ld_dst] = src [rows, cols]^T, bf16
 ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st) {
-  const int64_t total = rows * cols;
-  const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, (int64_t)sm_count_tc() * 8));
+  if (cols % 8 != 0 || rows <= 0) return QL_ERR_UNSUPPORTED;
+  const unsigned g = (unsigned)((rows + 255) / 256);
   TraceScope ts(TK_TRANSPOSE, st);
-  QL_CUDA_TRY(launch(skinny::transpose_kernel, dim3(g), dim3(256), 0, st, 1, 1, (const uint16_t*)src, (int)rows, cols, (uint16_t*)dst, (int)ld_dst));
-  QL_LAUNCH_CHECK();
+  QL_CUDA_TRY(launch(skinny::transpose_kernel, dim3(g), dim3(256), 0, st, 1, 1, (const uint16_t*)src, (int)rows, cols,
+                     (uint16_t*)dst, (int)ld_dst));
   return QL_OK;
 }
 

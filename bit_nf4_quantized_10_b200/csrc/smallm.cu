@@ -502,6 +502,9 @@ static bool smallm_attr() {
     if (cudaFuncSetAttribute(smallm::smallm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024 - smallm_static_smem())) != cudaSuccess)
       return false;
+    if (cudaFuncSetAttribute(smallm::smallm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+        cudaSuccess)
+      return false;
     set = true;
   }
   return true;
