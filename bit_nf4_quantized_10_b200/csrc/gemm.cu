@@ -38,8 +38,9 @@
 //   warp 1      TMEM allocation (both CTAs); one thread of the even CTA
 //               issues the MMAs
 //   warps 2-17  dequant producers, four groups of 4 warps on stages
-//               g, g+4, ...; each thread expands one 64-block through a
-//               per-block register lookup table into the swizzled BF16 tile;
+//               g, g+4, ...; each thread expands one 64-block (levels from a
+//               shared fp32 table, times the block constant, packed to bf16)
+//               into the swizzled BF16 tile;
 //               then the LoRA operands; then all 16 warps drain TMEM.
 // The weight tile holds W rows as 128-byte rows in both directions: K-major
 // for the forward (rows = output features), MN-major for the backward (rows =
@@ -166,6 +167,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_codes,
                       const Params p) {
   extern __shared__ uint8_t smem_raw[];
+  // the 16 fp32 levels, 256-byte aligned: an LDS address is the table base with
+  // the level's byte offset (4 * code) in its low byte
+  __shared__ __align__(256) float qlev[64];
+  if (threadIdx.x < 16) qlev[threadIdx.x] = p.tab.q[threadIdx.x];
   Smem sm = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -289,6 +294,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int gt = ((wp % GROUP_WARPS) << 5) | lane;   // thread within the group, 0..127
     const int kblocks = p.K / 64;            // 64-blocks per weight row
     const float mu = p.wc.absmax ? 0.0f : *p.wc.offset;
+    const uint32_t qbase = smem_u32(qlev);   // low byte 0
     int row_in_tile, col_chunk;
     if (!BWD) { row_in_tile = gt; col_chunk = 0; }
     else { row_in_tile = gt & 63; col_chunk = gt >> 6; }
@@ -334,9 +340,25 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint4 c0 = *reinterpret_cast<const uint4*>(cs + coff0);
         const uint4 c1 = *reinterpret_cast<const uint4*>(cs + coff1);
         const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const Lut16 L = make_lut(p.tab, decode_const(p.wc, cur, mu));
+        // w_hat = bf16(fl32(q[code] * c)): the level from the shared table (one
+        // byte permute forms the address), a packed pair of RN fp32 products,
+        // one conversion per pair
+        const float c = decode_const(p.wc, cur, mu);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(base + boff[j]) = lut_lookup8(L, w[j]);
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t e4 = (w[j] << 2) & 0x3C3C3C3Cu;   // 4 * low nibble of each byte
+          const uint32_t o4 = (w[j] >> 2) & 0x3C3C3C3Cu;   // 4 * high nibble of each byte
+          uint32_t o[4];
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) {
+            const float fe = lds_f32(__byte_perm(e4, qbase, 0x7650u | bb));
+            const float fo = lds_f32(__byte_perm(o4, qbase, 0x7650u | bb));
+            float pe, po;
+            mul2_rn(fe, fo, c, pe, po);
+            o[bb] = pack_bf16x2(pe, po);
+          }
+          *reinterpret_cast<uint4*>(base + boff[j]) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
       } else {
 #pragma unroll
         for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(base + boff[j]) = zero4();

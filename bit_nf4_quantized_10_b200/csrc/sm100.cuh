@@ -267,5 +267,19 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
   return v;
 }
 
+// (a * c, b * c), each an IEEE fp32 product rounded to nearest (one packed instruction)
+__device__ __forceinline__ void mul2_rn(float a, float b, float c, float& ra, float& rb) {
+  asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %4};\n"
+      " mul.rn.f32x2 z, x, y;\n mov.b64 {%0, %1}, z;\n}"
+      : "=f"(ra), "=f"(rb)
+      : "f"(a), "f"(b), "f"(c));
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
 }  // namespace sm100
 }  // namespace ql

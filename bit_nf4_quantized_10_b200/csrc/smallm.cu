@@ -112,20 +112,6 @@ __device__ __forceinline__ void arrive_remote_release(uint64_t* bar, uint32_t ra
       : "memory");
 }
 
-// (a * c, b * c), each an IEEE fp32 product rounded to nearest (one packed instruction)
-__device__ __forceinline__ void mul2_rn(float a, float b, float c, float& ra, float& rb) {
-  asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %4};\n"
-      " mul.rn.f32x2 z, x, y;\n mov.b64 {%0, %1}, z;\n}"
-      : "=f"(ra), "=f"(rb)
-      : "f"(a), "f"(b), "f"(c));
-}
-
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-
 __device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared::cluster.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
