@@ -162,7 +162,8 @@ class Projection:
         self.dX = torch.empty(self.M, self.K, dtype=torch.bfloat16, device=dev)
         self.dA = torch.empty(self.r, self.K, dtype=torch.float32, device=dev)
         self.dB = torch.empty(self.N, self.r, dtype=torch.float32, device=dev)
-        self.ws = torch.empty(q.qlora_workspace_size(q.QL_OP_BWD, self.M, self.N, self.K, self.r),
+        self.ws = torch.empty(max(q.qlora_workspace_size(q.QL_OP_FWD, self.M, self.N, self.K, self.r),
+                                  q.qlora_workspace_size(q.QL_OP_BWD, self.M, self.N, self.K, self.r)),
                               dtype=torch.uint8, device=dev)
 
     @property

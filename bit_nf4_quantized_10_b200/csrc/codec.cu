@@ -49,37 +49,61 @@ QuantBins build_bins(const NF4Table& t) {
   return b;
 }
 
+// Eight consecutive elements as loaded (raw words), and as fp32 values.
 template <typename T>
-__device__ __forceinline__ void load8(const T* x, int64_t e0, int64_t n, float (&v)[8]);
+struct Raw8;
+template <>
+struct Raw8<float> {
+  uint32_t w[8];
+};
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint32_t w[4];
+};
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* x, int64_t e0, int64_t n, Raw8<T>& r);
 
 template <>
-__device__ __forceinline__ void load8<float>(const float* x, int64_t e0, int64_t n, float (&v)[8]) {
+__device__ __forceinline__ void load8<float>(const float* x, int64_t e0, int64_t n, Raw8<float>& r) {
   if (e0 + 8 <= n) {
-    float4 a = __ldcs(reinterpret_cast<const float4*>(x + e0));
-    float4 b = __ldcs(reinterpret_cast<const float4*>(x + e0) + 1);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(x + e0));
+    const uint4 b = __ldcs(reinterpret_cast<const uint4*>(x + e0) + 1);
+    r.w[0] = a.x; r.w[1] = a.y; r.w[2] = a.z; r.w[3] = a.w;
+    r.w[4] = b.x; r.w[5] = b.y; r.w[6] = b.z; r.w[7] = b.w;
   } else {
+    const uint32_t* u = reinterpret_cast<const uint32_t*>(x);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = (e0 + i < n) ? x[e0 + i] : 0.0f;
+    for (int i = 0; i < 8; ++i) r.w[i] = (e0 + i < n) ? u[e0 + i] : 0u;
   }
 }
 
 template <>
 __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* x, int64_t e0, int64_t n,
-                                                     float (&v)[8]) {
+                                                     Raw8<__nv_bfloat16>& r) {
   if (e0 + 8 <= n) {
-    uint4 a = __ldcs(reinterpret_cast<const uint4*>(x + e0));
-    uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = bf16_lo(w[i]);
-      v[2 * i + 1] = bf16_hi(w[i]);
-    }
+    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(x + e0));
+    r.w[0] = a.x; r.w[1] = a.y; r.w[2] = a.z; r.w[3] = a.w;
   } else {
     const uint16_t* u = reinterpret_cast<const uint16_t*>(x);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = (e0 + i < n) ? __uint_as_float(((uint32_t)u[e0 + i]) << 16) : 0.0f;
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = (e0 + 2 * i < n) ? u[e0 + 2 * i] : 0u;
+      const uint32_t hi = (e0 + 2 * i + 1 < n) ? u[e0 + 2 * i + 1] : 0u;
+      r.w[i] = lo | (hi << 16);
+    }
+  }
+}
+
+__device__ __forceinline__ void unpack8(const Raw8<float>& r, float (&v)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r.w[i]);
+}
+__device__ __forceinline__ void unpack8(const Raw8<__nv_bfloat16>& r, float (&v)[8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = bf16_lo(r.w[i]);
+    v[2 * i + 1] = bf16_hi(r.w[i]);
   }
 }
 
@@ -103,11 +127,17 @@ __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, 
   const int bq = (threadIdx.x >> 3) & 3;         // block within the warp's four
   // the whole warp (4 blocks) iterates together so the shuffles see all lanes
   const int64_t warps_per_grid = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t wb = ((int64_t)blockIdx.x * (blockDim.x >> 5) + wib) * 4; wb < nb; wb += warps_per_grid * 4) {
+  // the next iteration's eight elements are loaded (as raw words) while this
+  // one is coded
+  int64_t wb = ((int64_t)blockIdx.x * (blockDim.x >> 5) + wib) * 4;
+  Raw8<T> nxt;
+  if (wb < nb) load8<T>(x, (wb + bq) * 64 + lane8 * 8, n, nxt);
+  for (; wb < nb; wb += warps_per_grid * 4) {
     const int64_t b = wb + bq;
     const int64_t e0 = b * 64 + lane8 * 8;   // >= n for a block past the end
     float v[8];
-    load8<T>(x, e0, n, v);
+    unpack8(nxt, v);
+    if (wb + warps_per_grid * 4 < nb) load8<T>(x, (wb + warps_per_grid * 4 + bq) * 64 + lane8 * 8, n, nxt);
     uint32_t abits = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) abits = max(abits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
@@ -309,7 +339,16 @@ static unsigned grid_for(int64_t work_items, int per_cta, int ctas_per_sm) {
 ql_status launch_quantize(const void* x, ql_dtype dt, int64_t n, uint8_t* codes, float* absmax,
                           cudaStream_t st) {
   const int64_t nb = (n + 63) / 64;
-  const unsigned grid = grid_for(nb, 32, 8);   // 32 blocks (8 warps x 4) per CTA-iteration
+  // one resident wave of CTAs (grid-stride loop), 32 blocks (8 warps x 4) per CTA iteration
+  static int per_sm[2] = {0, 0};
+  int& bps = per_sm[dt == QL_F32 ? 0 : 1];
+  if (!bps) {
+    const cudaError_t e = dt == QL_F32
+                              ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, quantize_kernel<float>, 256, 0)
+                              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, quantize_kernel<__nv_bfloat16>, 256, 0);
+    if (e != cudaSuccess || bps < 1) bps = 4;
+  }
+  const unsigned grid = grid_for(nb, 32, bps);
   static const QuantBins bins = build_bins(nf4_table());
   TraceScope ts(TK_QUANTIZE, st);
   if (dt == QL_F32)

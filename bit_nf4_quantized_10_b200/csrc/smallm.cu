@@ -497,10 +497,10 @@ static bool smallm_attr() {
 }
 
 // Cluster size (CTAs sharing K) and cluster count: the tiles are handed out in
-// rounds of `clusters`, each round costing about `per` sub-steps, so pick the
-// split with the fewest rounds x per among the cluster sizes that fit (the
-// cluster count comes from the occupancy calculator: a cluster's CTAs must
-// share a GPC, which caps it below SMs / cs).
+// rounds of `clusters`, each round costing about `per` sub-steps, scaled up
+// when the code ring is shallower than 8 stages; pick the cheapest among the
+// cluster sizes that fit (the cluster count comes from the occupancy
+// calculator: a cluster's CTAs must share a GPC, which caps it below SMs / cs).
 static bool smallm_plan(int64_t N, int64_t K, SmallmPlan& best, bool query) {
   using namespace smallm;
   const int kb = (int)(K / BK);
@@ -532,7 +532,9 @@ static bool smallm_plan(int64_t N, int64_t K, SmallmPlan& best, bool query) {
     }
     pl.clusters = std::max(1, std::min(tiles, maxc));
     const long rounds = (tiles + pl.clusters - 1) / pl.clusters;
-    const long cost = rounds * per;
+    // a CTA streams its codes at a rate that grows with the bytes it has in
+    // flight, up to about 8 stages (128 KB): shallower rings cost in proportion
+    const long cost = rounds * per * (MAX_C_STAGES / pl.c_stages);
     if (!found || cost < best_cost) {
       best = pl;
       best_cost = cost;
