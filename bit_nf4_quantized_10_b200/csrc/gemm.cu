@@ -41,11 +41,15 @@
 //               g, g+4, ...; each thread expands one 64-block (levels from a
 //               shared fp32 table, times the block constant, packed to bf16)
 //               into the swizzled BF16 tile;
-//               then the LoRA operands; then all 16 warps drain TMEM.
+//               then the LoRA operands; then all 16 warps drain TMEM
+//               (a bf16 output is staged in the idle activation ring and
+//               leaves by bulk tensor stores, 128-byte lines).
 // The weight tile holds W rows as 128-byte rows in both directions: K-major
 // for the forward (rows = output features), MN-major for the backward (rows =
 // the reduction index), so the producers write the same layout either way.
 #include <cudaTypedefs.h>
+
+#include <cstring>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -89,6 +93,7 @@ struct Params {
   void* out;
   int out_bf16;
   int accumulate;
+  int tma_store;     // bf16 output written through shared memory by bulk tensor stores
   NF4Table tab;
   uint32_t wait_limit;
 };
@@ -165,7 +170,7 @@ __device__ __forceinline__ uint64_t b_desc(uint32_t b_addr, int kk, bool bwd) {
 template <bool BWD>
 __global__ void __launch_bounds__(THREADS, 1)
     qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_codes,
-                      const Params p) {
+                      const __grid_constant__ CUtensorMap tmap_out, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   // the 16 fp32 levels, 256-byte aligned: an LDS address is the table base with
   // the level's byte offset (4 * code) in its low byte
@@ -195,6 +200,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_act);
     prefetch_tmap(&tmap_codes);
+    if (p.tma_store) prefetch_tmap(&tmap_out);
   }
   if (warp == 1) {
     tmem_alloc2(sm.tmem_addr, TMEM_COLS);
@@ -416,7 +422,50 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     // ------------------------------------------------------------ epilogue
     const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(sm.acc_full, 0, abort_flag, p.wait_limit) && !*abort_flag);
-    if (acc_ok) {
+    if (p.tma_store) {
+      // bf16 output through shared memory.  Once the accumulators are complete
+      // no MMA reads the rings any more, so the activation ring holds the
+      // CTA's 256 x 256 bf16 tile: group g (TMEM half g >> 1, columns
+      // (g & 1) * 128 ..) writes its 128 rows x 128 columns as two boxes of 64
+      // columns in the 128-byte swizzled layout of the output tensor map, and
+      // one thread of the group stores them with two bulk tensor copies (the
+      // copy skips rows and columns outside the output).
+      const int quad = warp & 3;
+      const int g = wp >> 2;
+      const int accn = g >> 1;
+      const int lrow = quad * 32 + lane;
+      uint8_t* box0 = sm.base + g * 2 * (BMH * 128);
+      if (acc_ok) {
+        tc_fence_after();
+        for (int cc = 0; cc < 8; ++cc) {
+          const int col = (g & 1) * 128 + cc * 16;
+          uint32_t r[16];
+          tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(accn * 256 + col), r);
+          tmem_ld_wait();
+          uint32_t pk[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) pk[q] = pack_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+          uint8_t* box = box0 + (cc >> 2) * (BMH * 128);
+          const int ch = (cc & 3) * 2;
+          *reinterpret_cast<uint4*>(box + sw128_offset(lrow, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(box + sw128_offset(lrow, ch + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        fence_proxy_async_smem();
+      }
+      // every warp of the group reaches this barrier, whatever its waits returned
+      __syncwarp();
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory");
+      if ((wp & 3) == 0 && lane == 0 && acc_ok && !*abort_flag) {
+        const int y = m0 + accn * BMH;
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          const int x = j0 + (g & 1) * 128 + b * 64;
+          if (x < p.n_out && y < p.M) tma_store_2d(&tmap_out, box0 + b * (BMH * 128), x, y);
+        }
+        bulk_commit();
+        bulk_wait_all();
+      }
+    } else if (acc_ok) {
       tc_fence_after();
       const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
       const int g = wp >> 2;                     // 0..3: half g>>1, columns (g&1)*128 ..
@@ -527,7 +576,7 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
     attr_set = true;
   }
   const int N = (int)w->rows, K = (int)w->cols;
-  CUtensorMap map_act, map_codes;
+  CUtensorMap map_act, map_codes, map_out;
   const int red = BWD ? N : K;   // reduction length = activation row length
   if (!make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, (uint64_t)red, (uint64_t)M, (uint64_t)red, BK,
                    BM, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -556,11 +605,17 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
   p.out = out;
   p.out_bf16 = out_dt == QL_BF16;
   p.accumulate = accumulate;
+  // bf16 output that is written, not accumulated: bulk tensor stores of
+  // 64-column boxes, 128 rows high
+  p.tma_store = out_dt == QL_BF16 && !accumulate && (reinterpret_cast<uintptr_t>(out) & 15) == 0 &&
+                make_map_2d(&map_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, (uint64_t)p.n_out, (uint64_t)M,
+                            (uint64_t)p.n_out, 64, BMH, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!p.tma_store) memset(&map_out, 0, sizeof(map_out));
   p.tab = nf4_table();
   p.wait_limit = 1u << 22;
   const dim3 grid(2u * (unsigned)((p.n_out + BN - 1) / BN), (unsigned)((M + 2 * BM - 1) / (2 * BM)));
   TraceScope ts(BWD ? TK_GEMM_BWD : TK_GEMM_FWD, st);
-  QL_CUDA_TRY(launch(qlora_gemm_kernel<BWD>, grid, dim3(THREADS), SMEM_BYTES, st, 2, 1, map_act, map_codes, p));
+  QL_CUDA_TRY(launch(qlora_gemm_kernel<BWD>, grid, dim3(THREADS), SMEM_BYTES, st, 2, 1, map_act, map_codes, map_out, p));
   return QL_OK;
 }
 

@@ -97,12 +97,16 @@ def test_fwd_bwd_fp32_outputs(q, N, K, M, r, s, dq):
         assert_fp_close(np64(got["dB"][:, :r]), ref["dB"], "dB")
 
 
-@pytest.mark.parametrize("N,K,M,r,s", SHAPES[:3])
+@pytest.mark.parametrize("N,K,M,r,s", SHAPES)
 def test_bf16_outputs_within_one_ulp(q, N, K, M, r, s):
     case = make_case(N, K, M, r, seed=11 + N + K + M + r)
     got = run_gpu(q, *case, r, s, out_dtype=torch.bfloat16)
     ref = run_oracle(*case, r, s)
-    assert_bf16_within_ulp(got["Y"], ref["Y"], "Y bf16")
+    # The adapter term enters the accumulator as U bf16(s B)^T: exact when s is a
+    # power of two; otherwise bf16(s B) carries one rounding (relative 2^-9), a
+    # bound of about 1e-4 * rms(Y) here, so near-zero outputs get 1e-3 * rms.
+    abs_y = 0.0 if float(np.log2(s)).is_integer() else 1e-3
+    assert_bf16_within_ulp(got["Y"], ref["Y"], "Y bf16", abs_rms=abs_y)
     assert_bf16_within_ulp(got["dX"], ref["dX"], "dX bf16", abs_rms=1e-3)
 
 
@@ -114,14 +118,19 @@ def test_accumulate_dx(q):
     assert_fp_close(np64(got["dX"]) - 0.5, ref["dX"], "dX accumulate")
 
 
-def test_projection_workload_full(q):
-    """The 4096 x 4096 projection with 4096 tokens, r = 16, alpha = 32, at full size."""
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_projection_workload_full(q, out_dtype):
+    """The 4096 x 4096 projection with 4096 tokens, r = 16, alpha = 32, at full size
+    (bf16 Y and dX are what the timed step writes)."""
     w = S.WORKLOADS["c2"]
     d = S.linear_inputs(w, 0)
-    got = run_gpu(q, d["W"], d["X"], d["A"], d["B"], d["dY"], w.r, w.s)
+    got = run_gpu(q, d["W"], d["X"], d["A"], d["B"], d["dY"], w.r, w.s, out_dtype=out_dtype)
     ref = run_oracle(d["W"], d["X"], d["A"], d["B"], d["dY"], w.r, w.s)
     for k in ("Y", "dX"):
-        assert_fp_close(np64(got[k]), ref[k], k)
+        if out_dtype == torch.bfloat16:
+            assert_bf16_within_ulp(got[k], ref[k], k + " bf16", abs_rms=1e-3)
+        else:
+            assert_fp_close(np64(got[k]), ref[k], k)
     assert_fp_close(np64(got["dA"]), ref["dA"], "dA")
     assert_fp_close(np64(got["dB"]), ref["dB"], "dB")
     assert_bf16_within_ulp(got["U"], ref["U"], "U", abs_rms=1e-4)
