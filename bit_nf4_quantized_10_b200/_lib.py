@@ -58,6 +58,7 @@ def _load() -> ctypes.CDLL:
         "qlora_get_status": (i32, [vp]),
         "qlora_status_string": (ctypes.c_char_p, [i32]),
         "qlora_selftest_wait_timeout": (i32, [i64, vp]),
+        "qlora_merge": (i32, [W, vp, vp, i32, f32, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -168,6 +169,14 @@ def qlora_linear_bwd(w: "NF4Weight", X, dY, A, B, r: int, s: float, U, dX, dA, d
     _check(LIB.qlora_linear_bwd(ctypes.byref(d), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B), int(r), float(s), _ptr(U),
                                 _ptr(dX), _dt(dX.dtype), 1 if accumulate_dx else 0, _ptr(dA), _ptr(dB),
                                 _dt(dA.dtype), _ptr(ws), ws_bytes, _stream(stream)), "qlora_linear_bwd")
+
+
+def qlora_merge(w: "NF4Weight", A, B, r: int, s: float, W_out=None, codes_out=None, absmax_out=None,
+                stream=None) -> None:
+    """W' = W_hat + s B A as bf16 (W_out) and/or quantized again (codes_out, absmax_out)."""
+    d = w.desc()
+    _check(LIB.qlora_merge(ctypes.byref(d), _ptr(A), _ptr(B), int(r), float(s), _ptr(W_out), _ptr(codes_out),
+                           _ptr(absmax_out), _stream(stream)), "qlora_merge")
 
 
 def qlora_silu_gate_fwd(g, u, h, stream=None) -> None:

@@ -13,6 +13,8 @@ ql_status launch_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q
                               void* ws, cudaStream_t st);
 ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStream_t st);
 unsigned status_word_codec(cudaStream_t st);
+ql_status launch_merge(const ql_nf4_weight* w, const void* A, const void* B, int r, float s, void* out,
+                       uint8_t* codes_out, float* absmax_out, cudaStream_t st);
 // gemm.cu
 ql_status launch_gemm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
                           float s, void* Y, ql_dtype y_dt, cudaStream_t st);
@@ -129,6 +131,22 @@ ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* 
   if (st != QL_OK) return st;
   if (!dtype_ok(out_dt) || !aligned16(out)) return QL_ERR_INVALID_ARG;
   return ql::launch_dequant(w, out, out_dt, as_stream(stream));
+}
+
+ql_status qlora_merge(const ql_nf4_weight* w, const void* A, const void* B, int r, float s, void* W_out,
+                      uint8_t* codes_out, float* absmax_out, void* stream) {
+  ql_status st = check_weight(w);
+  if (st != QL_OK) return st;
+  if (w->cols % 64 != 0) return QL_ERR_INVALID_ARG;
+  if (r < 0) return QL_ERR_INVALID_ARG;
+  if (r > QL_MAX_RANK) return QL_ERR_UNSUPPORTED;
+  if (r > 0 && (!aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
+  if ((codes_out == nullptr) != (absmax_out == nullptr)) return QL_ERR_INVALID_ARG;
+  if (!W_out && !codes_out) return QL_ERR_INVALID_ARG;
+  if ((W_out && !aligned16(W_out)) || (codes_out && (!aligned16(codes_out) || !aligned16(absmax_out))))
+    return QL_ERR_INVALID_ARG;
+  return ql::launch_merge(w, r > 0 ? A : nullptr, r > 0 ? B : nullptr, r, s, W_out, codes_out, absmax_out,
+                          as_stream(stream));
 }
 
 ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* A, const void* B, int r,

@@ -49,6 +49,36 @@ QuantBins build_bins(const NF4Table& t) {
   return b;
 }
 
+// The eight codes of v (elements 0..7 in nibbles 0..7) given the block's
+// absmax c.  `bins` is the QuantBins table in shared memory as (m bits, count
+// below) pairs.
+__device__ __forceinline__ uint32_t encode8(const float (&v)[8], float c, const uint2* bins, const NF4Table& tab) {
+  uint32_t word = 0;
+  if (c >= 1e-30f) {
+    // 16/c: c >= 1e-30 keeps it finite; its rounding moves y by < 1e-6
+    const float s16 = __fmul_rn(16.0f, __frcp_rn(c));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // 1.5 * 2^23 + 16: the sum's low bits are round(16 y + 16), in 0..32
+      const float t = __fmaf_rn(v[i], s16, 12582928.0f);
+      const uint2 e = bins[__float_as_uint(t) & 63u];
+      const float th = __fmul_rn(__uint_as_float(e.x), c);
+      word |= (e.y + (v[i] > th ? 1u : 0u)) << (4 * i);
+    }
+  } else {
+    // tiny (or NaN) absmax: count the thresholds directly
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t k = 0;
+#pragma unroll
+      for (int j = 0; j < 15; ++j) k += (v[i] > __fmul_rn(tab.m[j], c)) ? 1u : 0u;
+      word |= k << (4 * i);
+    }
+  }
+  if (c == 0.0f) word = 0x88888888u;
+  return word;
+}
+
 // Eight consecutive elements as loaded (raw words), and as fp32 values.
 template <typename T>
 struct Raw8;
@@ -145,29 +175,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, 
     for (int o = 1; o < 8; o <<= 1) abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
     if (abits >= 0x7F800000u && lane8 == 0 && b < nb) raise_status(ST_NONFINITE);
     const float c = __uint_as_float(abits);
-    uint32_t word = 0;
-    if (c >= 1e-30f) {
-      // 16/c: c >= 1e-30 keeps it finite; its rounding moves y by < 1e-6
-      const float s16 = __fmul_rn(16.0f, __frcp_rn(c));
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        // 1.5 * 2^23 + 16: the sum's low bits are round(16 y + 16), in 0..32
-        const float t = __fmaf_rn(v[i], s16, 12582928.0f);
-        const uint2 e = bins[__float_as_uint(t) & 63u];
-        const float th = __fmul_rn(__uint_as_float(e.x), c);
-        word |= (e.y + (v[i] > th ? 1u : 0u)) << (4 * i);
-      }
-    } else {
-      // tiny (or NaN) absmax: count the thresholds directly
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint32_t k = 0;
-#pragma unroll
-        for (int j = 0; j < 15; ++j) k += (v[i] > __fmul_rn(tab.m[j], c)) ? 1u : 0u;
-        word |= k << (4 * i);
-      }
-    }
-    if (c == 0.0f) word = 0x88888888u;
+    const uint32_t word = encode8(v, c, bins, tab);
     if (e0 + 8 <= n) {
       __stcs(reinterpret_cast<uint32_t*>(codes + (e0 >> 1)), word);
     } else if (e0 < n) {
@@ -317,6 +325,89 @@ __global__ void __launch_bounds__(256) dequant_f32_kernel(const uint8_t* __restr
   }
 }
 
+// ------------------------------------------------------------ adapter merge
+// W' = bf16(fl32(w_hat + fl32(s d))), d = sum over j = 0 .. r-1 in order of
+// B[n, j] A[j, k] in fp32 ("QLoRA: Quantize Base Weights to 4-Bit", FAQ on
+// inference latency: W = W_dequant + (alpha / r) B A in 16 bits; "QLoRA —
+// Fine-Tuning a 65B Model on One GPU", "Pitfalls": merge in 16 bits, then
+// quantize the merged weight if a quantized model is wanted).  A product of two
+// bf16 values is exact in fp32, so each fma is the rounded fp32 sum.
+// Optionally the merged values are quantized again (same code selection as
+// quantize_kernel), without a round trip of the bf16 weight through HBM.
+// Layout as in quantize_kernel: 8 threads per 64-block, 8 consecutive elements
+// each, a warp's four blocks iterate together.  K % 64 == 0, so a block lies in
+// one row and its A columns are 16-byte aligned.
+__global__ void __launch_bounds__(256) merge_kernel(const uint8_t* __restrict__ codes, WeightConsts wc, int64_t N,
+                                                    int64_t K, const __nv_bfloat16* __restrict__ A,
+                                                    const __nv_bfloat16* __restrict__ B, int r, float s,
+                                                    __nv_bfloat16* __restrict__ out, uint8_t* __restrict__ codes_out,
+                                                    float* __restrict__ absmax_out, NF4Table tab, QuantBins bins_in) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ uint2 bins[64];
+  __shared__ float q[16];
+  if (threadIdx.x < 64) bins[threadIdx.x] = make_uint2(__float_as_uint(bins_in.m[threadIdx.x]), bins_in.base[threadIdx.x]);
+  if (threadIdx.x < 16) q[threadIdx.x] = tab.q[threadIdx.x];
+  __syncthreads();
+  const int64_t nb = N * K / 64;
+  const float mu = wc.absmax ? 0.0f : *wc.offset;
+  const int lane8 = threadIdx.x & 7;
+  const int wib = threadIdx.x >> 5;
+  const int bq = (threadIdx.x >> 3) & 3;
+  const int64_t warps_per_grid = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t wb = ((int64_t)blockIdx.x * (blockDim.x >> 5) + wib) * 4; wb < nb; wb += warps_per_grid * 4) {
+    const int64_t b = wb + bq;
+    const bool live = b < nb;
+    const int64_t e0 = b * 64 + lane8 * 8;
+    float v[8];
+    if (live) {
+      const int64_t row = e0 / K, k0 = e0 - row * K;
+      const float c = block_const(wc, b, mu);
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + (e0 >> 1));
+      float d[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d[i] = 0.0f;
+      const __nv_bfloat16* brow = B + row * r;
+      for (int j = 0; j < r; ++j) {
+        const float bj = __bfloat162float(brow[j]);
+        const uint4 a = *reinterpret_cast<const uint4*>(A + (int64_t)j * K + k0);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          d[2 * h] = __fmaf_rn(bj, bf16_lo(aw[h]), d[2 * h]);
+          d[2 * h + 1] = __fmaf_rn(bj, bf16_hi(aw[h]), d[2 * h + 1]);
+        }
+      }
+      uint32_t pk[4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float wh = __bfloat162float(__float2bfloat16_rn(__fmul_rn(q[(w >> (4 * i)) & 0xFu], c)));
+        v[i] = __bfloat162float(__float2bfloat16_rn(__fadd_rn(wh, __fmul_rn(s, d[i]))));
+      }
+#pragma unroll
+      for (int h = 0; h < 4; ++h) pk[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
+      if (out) *reinterpret_cast<uint4*>(out + e0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    }
+    if (codes_out) {   // uniform over the grid: every lane takes part in the shuffles
+      uint32_t abits = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) abits = max(abits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
+      if (abits >= 0x7F800000u && lane8 == 0 && live) raise_status(ST_NONFINITE);
+      const float c2 = __uint_as_float(abits);
+      const uint32_t word = encode8(v, c2, bins, tab);
+      if (live) {
+        *reinterpret_cast<uint32_t*>(codes_out + (e0 >> 1)) = word;
+        if (lane8 == 0) absmax_out[b] = c2;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------- launch
 static int sm_count() {
   static int count = 0;
@@ -408,6 +499,27 @@ ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStr
     QL_CUDA_TRY(launch(dequant_f32_kernel, dim3(grid_for((n + 7) / 8, 256, 8)), dim3(256), 0, st, 1, 1, w->codes, wc, n, (float*)out,
                                                                      nf4_table()));
   }
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
+
+ql_status launch_merge(const ql_nf4_weight* w, const void* A, const void* B, int r, float s, void* out,
+                       uint8_t* codes_out, float* absmax_out, cudaStream_t st) {
+  const int64_t nb = w->rows * w->cols / 64;
+  WeightConsts wc{w->absmax, w->absmax_q, w->scale2, w->offset};
+  static int bps = 0;
+  if (!bps) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, merge_kernel, 256, 0) != cudaSuccess || bps < 1) {
+      cudaGetLastError();
+      bps = 4;
+    }
+  }
+  static const QuantBins bins = build_bins(nf4_table());
+  TraceScope ts(TK_MERGE, st);
+  QL_CUDA_TRY(launch(merge_kernel, dim3(grid_for(nb, 32, bps)), dim3(256), 0, st, 1, 1, w->codes, wc, w->rows, w->cols,
+                     (const __nv_bfloat16*)A, (const __nv_bfloat16*)B, r, s, (__nv_bfloat16*)out, codes_out, absmax_out,
+                     nf4_table(), bins));
   QL_LAUNCH_CHECK();
   return QL_OK;
 }

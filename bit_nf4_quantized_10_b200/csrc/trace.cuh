@@ -23,6 +23,7 @@ enum TraceKind : int {
   TK_SILU,
   TK_SMALLM,
   TK_TRANSPOSE,
+  TK_MERGE,
   TK_COUNT
 };
 

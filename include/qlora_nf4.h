@@ -7,7 +7,9 @@
  *   - double quantization of the fp32 block constants to 8-bit floats in
  *     groups of 256;
  *   - the frozen-4-bit + LoRA linear  Y = X * dequant(W)^T + s * (X A^T) B^T,
- *     s = alpha / r, forward and backward (dX, dA, dB; W is never written).
+ *     s = alpha / r, forward and backward (dX, dA, dB; W is never written);
+ *   - the adapter merge W' = dequant(W) + s B A after training, as a bf16
+ *     weight and/or quantized again.
  *
  * Sources (the web pages this library restates):
  *   [P2] "QLoRA: Quantize Base Weights to 4-Bit": §2.1 (NF4 quantile formula),
@@ -144,6 +146,35 @@ ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q,
 #define QL_NOALLOC_MAX_BLOCKS (1ll << 26)
 ql_status nf4_double_quant_noalloc(const float* absmax, int64_t nb, uint8_t* absmax_q,
                                    float* scale2, float* offset, void* stream);
+
+/*
+ * qlora_merge — fold a trained adapter into the base weight:
+ *   W' = W_hat + s B A  as a bf16 [N, K] weight, and/or that weight quantized
+ *   again to NF4.  [P2] FAQ "Does QLoRA introduce inference latency overhead
+ *   once the model is fine-tuned and deployed?": dequantize the base to 16 bits
+ *   and merge, W = W_dequant + (alpha / r) B A.  [P3] "Pitfalls": merge in 16
+ *   bits, then quantize the merged result if a quantized model is wanted
+ *   ("How it's used in practice": peft's merge_and_unload()).
+ * Arithmetic, per element (n, k), in this order:
+ *   d  = sum_{j = 0 .. r-1} B[n, j] A[j, k]   fp32, each partial sum rounded
+ *        (a bf16 x bf16 product is exact in fp32),
+ *   W' = bf16(fl32(w_hat + fl32(s d))),   w_hat = bf16(fl32(q_code c_hat)).
+ * Re-quantization codes W' exactly as nf4_quantize would code that bf16 tensor.
+ *   w          NF4 weight (either constant form); K = w->cols % 64 == 0.
+ *   A          device bf16 [r, K]; B device bf16 [N, r] (unused when r == 0).
+ *   r          0 <= r <= QL_MAX_RANK (no multiple-of-8 rule here).
+ *   s          alpha / r.
+ *   W_out      device bf16 [N, K], or NULL.
+ *   codes_out  device uint8 [N*K/2] and absmax_out device fp32 [N*K/64] (the
+ *              fp32 constants; nf4_double_quant compresses them), both or
+ *              neither.  At least one output must be given.  Outputs must not
+ *              overlap the inputs.
+ * A non-finite merged value sets QL_ERR_NONFINITE in the status word (when
+ * re-quantizing).  Errors: QL_ERR_INVALID_ARG (bad pointer, alignment, K % 64,
+ * output combination), QL_ERR_UNSUPPORTED (r > QL_MAX_RANK), QL_ERR_CUDA.
+ */
+ql_status qlora_merge(const ql_nf4_weight* w, const void* A, const void* B, int r, float s,
+                      void* W_out, uint8_t* codes_out, float* absmax_out, void* stream);
 
 /*
  * nf4_dequant — x_hat = bf16(fl32(q_code * c)) ([P3] "Quantization in one

@@ -25,7 +25,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .formats import F64, bf16
+from .formats import F64, bf16, fl32
 
 
 def _f64(t) -> np.ndarray:
@@ -69,6 +69,33 @@ def backward(X, W_hat, A, B, s: float, dY, U=None, materialize: bool = True):
     dA = s * (V.T @ X)
     dB = s * (dY.T @ U)
     return dict(dX=dX, dA=dA, dB=dB, V=V, U=U)
+
+
+def merge(W_hat, A, B, s: float) -> np.ndarray:
+    """Adapter merge: W' = W_hat + s B A as a bf16 weight.
+
+    [P2] FAQ "Does QLoRA introduce inference latency overhead once the model is
+    fine-tuned and deployed?": the base is dequantized to 16 bits and the
+    adapter folded in, W = W_dequant + (alpha / r) B A.  [P3] "Pitfalls" and
+    "How it's used in practice" (merge_and_unload): the merge happens in 16
+    bits; a quantized model is made by quantizing the merged weight again.
+
+    The pages fix no summation order.  This reading, in fp32 with one rounding
+    per step:
+      d  = sum over j = 0 .. r-1, in that order, of B[n, j] A[j, k]
+           (each product of two bf16 values is exact in fp32; each partial sum
+           is rounded to fp32),
+      t  = fl32(fl32(s) d),
+      W' = bf16(fl32(W_hat + t)).
+    The fp64 sums below are the fp32 additions themselves (formats.py: one
+    IEEE operation on fp32 operands, rounded through float64).
+    """
+    W_hat, A, B = _f64(W_hat), _f64(A), _f64(B)
+    d = np.zeros(W_hat.shape, dtype=F64)
+    for j in range(A.shape[0]):
+        d = fl32(d + np.outer(B[:, j], A[j, :]))
+    t = fl32(fl32(s) * d)
+    return bf16(fl32(W_hat + t))
 
 
 def adapter_param_count(d: int, k: int, r: int) -> int:

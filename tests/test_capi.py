@@ -81,6 +81,15 @@ def test_argument_errors_return_before_launch(lib):
     assert L.qlora_linear_bwd(ctypes.byref(w), fake, fake, 16, fake, fake, 8, 2.0, None, fake, lib.QL_F32, 0,
                               fake, fake, lib.QL_F32, fake, 0, s0) == lib.QL_ERR_WORKSPACE
     assert L.nf4_dequant(None, fake, lib.QL_BF16, s0) == lib.QL_ERR_INVALID_ARG
+    w = lib.ql_nf4_weight(fake, fake, None, None, None, 256, 500)                           # K % 64 != 0
+    assert L.qlora_merge(ctypes.byref(w), fake, fake, 8, 2.0, fake, None, None, s0) == lib.QL_ERR_INVALID_ARG
+    w = lib.ql_nf4_weight(fake, fake, None, None, None, 256, 512)
+    assert L.qlora_merge(ctypes.byref(w), fake, fake, 8, 2.0, None, None, None, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.qlora_merge(ctypes.byref(w), fake, fake, 8, 2.0, None, fake, None, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.qlora_merge(ctypes.byref(w), fake, fake, -1, 2.0, fake, None, None, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.qlora_merge(ctypes.byref(w), fake, fake, 65, 2.0, fake, None, None, s0) == lib.QL_ERR_UNSUPPORTED
+    assert L.qlora_merge(ctypes.byref(w), None, fake, 8, 2.0, fake, None, None, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.qlora_merge(ctypes.byref(w), fake, fake, 8, 2.0, fake + 8, None, None, s0) == lib.QL_ERR_INVALID_ARG
     assert lib.status_string(lib.QL_ERR_TIMEOUT) == "device wait timed out"
     for polls in (0, -1, (1 << 20) + 1):
         assert L.qlora_selftest_wait_timeout(polls, s0) == lib.QL_ERR_INVALID_ARG

@@ -8,6 +8,7 @@ adapter-count example are checked directly.
 import numpy as np
 import pytest
 
+from oracle import formats as F
 from oracle import lora, nf4
 
 
@@ -115,3 +116,80 @@ def test_dequant_then_linear_uses_table_values():
     assert cb[0] == c
     what = nf4.dequant(packed, 64, cb, out="f32")
     assert np.array_equal(what, w)
+
+
+# ------------------------------------------------------------ adapter merge
+def _bf16_inputs(rng, N, K, r, wstd=0.02):
+    """A dequantized NF4 weight (bf16 values), and bf16 A, B of the page's scales."""
+    import torch
+    W = torch.from_numpy((rng.standard_normal((N, K)) * wstd).astype(np.float32))
+    packed, c, _ = nf4.quantize(W)
+    W_hat = nf4.dequant(packed, N * K, c, out="bf16").reshape(N, K)
+    A = F.bf16(rng.uniform(-1.0, 1.0, (r, K)) / np.sqrt(K))
+    B = F.bf16(rng.standard_normal((N, r)) * 0.01)
+    return W, packed, c, W_hat, A, B
+
+
+def _ulps(a, b):
+    """Distance in bf16 steps between two arrays of bf16 values."""
+    def lin(v):
+        bits = F.bf16_bits(v).astype(np.int64)
+        return np.where(bits & 0x8000, -(bits & 0x7FFF), bits & 0x7FFF)
+    return np.abs(lin(a) - lin(b))
+
+
+def test_merge_zero_adapter_is_the_dequantized_weight():
+    rng = np.random.default_rng(11)
+    _, _, _, W_hat, A, B = _bf16_inputs(rng, 6, 128, 4)
+    assert np.array_equal(lora.merge(W_hat, A, B, 0.0), W_hat)
+    assert np.array_equal(lora.merge(W_hat, A, np.zeros_like(B), 2.0), W_hat)
+
+
+def test_merge_closed_form_on_exact_values():
+    # r = 1 and power-of-two entries: every step is exact, W' = W_hat + s b a
+    W_hat = np.array([[0.5, -0.25], [0.0, 1.0], [-0.75, 0.125]])
+    A = np.array([[0.25, -0.5]])
+    B = np.array([[0.125], [-1.0], [0.5]])
+    got = lora.merge(W_hat, A, B, 2.0)
+    want = W_hat + 2.0 * (B @ A)          # all representable in bf16
+    assert np.array_equal(got, want)
+    assert got[0, 0] == 0.5625 and got[1, 1] == 2.0
+
+
+@pytest.mark.parametrize("s", [2.0, 0.75, 0.25])
+@pytest.mark.parametrize("r", [1, 8, 16, 64])
+def test_merge_within_one_bf16_step_of_the_exact_sum(s, r):
+    # W_hat + s B A in exact float64 (errors ~1e-16), rounded once to bf16: the
+    # fp32 steps may move a value across a bf16 rounding boundary, nothing more
+    rng = np.random.default_rng(100 + r)
+    _, _, _, W_hat, A, B = _bf16_inputs(rng, 24, 192, r)
+    got = lora.merge(W_hat, A, B, s)
+    exact = F.bf16(W_hat + np.float64(np.float32(s)) * (B @ A))
+    d = _ulps(got, exact)
+    assert d.max() <= 1
+    assert (d == 0).mean() > 0.99
+    # the update is visible: the merged weight is not the base
+    assert (got != W_hat).mean() > 0.5
+
+
+def test_merge_sign_and_orientation():
+    # a mistake in the order of B A (A^T B^T, a transpose) or the sign shows here
+    W_hat = np.zeros((2, 3))
+    A = np.array([[1.0, 2.0, 4.0]])       # r x K
+    B = np.array([[0.5], [-0.25]])        # N x r
+    got = lora.merge(W_hat, A, B, 1.0)
+    assert np.array_equal(got, np.array([[0.5, 1.0, 2.0], [-0.25, -0.5, -1.0]]))
+
+
+def test_merge_zero_adapter_requantizes_to_the_original_codes():
+    # the merged weight with a zero adapter is the dequantized weight, whose
+    # nearest levels are the original codes: re-quantizing gives them back, with
+    # constants bf16(c) (the largest level is 1, so the block maximum is bf16(c))
+    rng = np.random.default_rng(12)
+    N, K = 5, 256
+    _, packed, c, W_hat, A, B = _bf16_inputs(rng, N, K, 8)
+    merged = lora.merge(W_hat, A, B, 0.0)
+    packed2, c2, finite = nf4.quantize(merged.reshape(-1))
+    assert finite
+    assert np.array_equal(nf4.unpack(packed2, N * K), nf4.unpack(packed, N * K))
+    assert np.array_equal(c2, F.bf16(c))
