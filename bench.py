@@ -298,7 +298,19 @@ def small_m_and_codec(q, dev, hbm_peak):
         t = statistics.median(times) / 1e3
         gbs = wbytes / t / 1e9
         out[f"M{M}"] = {"us": round(t * 1e6, 2), "weight_GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 3)}
-    del wq
+    # adapter merge of the same weight, bf16 output and re-quantized codes + fp32 constants
+    n5 = N * K
+    W_out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    codes_out = torch.empty(n5 // 2, dtype=torch.uint8, device=dev)
+    absmax_out = torch.empty(n5 // 64, dtype=torch.float32, device=dev)
+    t = _time_calls(lambda: q.qlora_merge(wq, A, B, r, s, W_out=W_out, codes_out=codes_out, absmax_out=absmax_out),
+                    flush, n_warm=3, n=10)
+    # read codes + E4M3 constants + scales + A, B; write bf16 W' + codes + fp32 constants
+    moved = n5 // 2 + n5 // 64 + 4 * (n5 // 16384) + 2 * r * (N + K) + 2 * n5 + n5 // 2 + 4 * (n5 // 64)
+    out[f"merge_{N}x{K}_r{r}"] = {"us": round(t * 1e6, 2), "GBps": round(moved / t / 1e9, 1),
+                                 "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3), "bytes": moved,
+                                 "fma_per_element": r}
+    del W_out, codes_out, absmax_out, wq
     torch.cuda.empty_cache()
     # codec over 4 Gi bf16 elements
     n = w5.codec_n
