@@ -8,6 +8,7 @@ Everything is numpy in float64, with every rounding the method prescribes
 written out explicitly (to fp32, bf16 or E4M3, round to nearest even).  Each
 function names the passage of the source pages it restates:
 
+  [P1] "Lesson 4 of the Finetuning Sessions"
   [P2] "QLoRA: Quantize Base Weights to 4-Bit"
   [P3] "QLoRA — Fine-Tuning a 65B Model on One GPU"
   [P4] "QLoRA fine-tuning on consumer GPUs" (FAQ)
@@ -17,4 +18,4 @@ function.  Parity status per function is in its docstring; every function here
 is pinned by a test under tests/ against something other than itself, except
 where a docstring says "parity unpinned".
 """
-from . import formats, nf4, lora  # noqa: F401
+from . import formats, nf4, lora, fp4  # noqa: F401

@@ -1,0 +1,130 @@
+"""4-bit float block formats with per-block scales: MXFP4 and NVFP4 (oracle).
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).  float64 numpy with the
+roundings written out.
+
+Sources:
+  [P1] "Lesson 4 of the Finetuning Sessions", "From FP32 to the 4-Bit Horizon":
+       MXFP4 (Open Compute Project microscaling): a block of 32 elements shares
+       one 8-bit E8M0 scale, always a power of two; NVFP4 (Blackwell): blocks
+       of 16 share an 8-bit E4M3 scale, whose 3 mantissa bits allow fractional
+       scales.  "From Turing to Blackwell": the 5th-generation tensor cores
+       execute these 4-bit tensors natively with the E4M3 scales.
+
+Both formats store E2M1 elements: 1 sign bit, 2 exponent bits (bias 1), 1
+mantissa bit; magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}; no infinities or NaN.
+
+Readings (the pages fix none of these steps):
+  - Element rounding: nearest E2M1 value, ties to even (mantissa bit 0),
+    magnitudes above 6 saturate to 6.
+  - MXFP4 scale: 2^(floor(log2 amax) - 2), the rule of the OCP microscaling
+    format: the block's largest magnitude lands in [4, 8), the top binade of
+    E2M1 (values in (6, 8) saturate).  An all-zero block takes 2^-127, the
+    smallest E8M0 scale.
+  - NVFP4 scale: E4M3(amax / 6) per block of 16, round to nearest even,
+    saturating at 448, so the largest element maps to about 6.  E4M3 spans
+    2^-9 .. 448; with `tensor_scale`, one fp32 scale per tensor, s_t =
+    fl32(amax_tensor / (6 * 448)), divides every block scale first
+    (E4M3(amax_b / (6 s_t))) and multiplies back on dequantization, so the
+    block scales of small weights use E4M3's normal range.  A block whose
+    scale rounds to 0 stores zeros.
+  - Element codes: the rounding of x / scale (the scale as decoded), computed
+    in float64 (the division is exact enough: one rounding to E2M1 follows).
+
+Parity: pinned by tests/test_oracle_fp4.py (E2M1 grid from the format's fields,
+brute-force nearest-even rounding, power-of-two scale invariance, exact blocks,
+error bounds).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .formats import F64, fl32, e4m3_round, round_to_precision
+
+E2M1_MAX = 6.0
+MX_BLOCK = 32       # [P1] "a block of 32 elements shares a single 8-bit scale"
+NV_BLOCK = 16       # [P1] "reducing the block size from 32 down to 16 elements"
+
+
+def e2m1_decode(code) -> np.ndarray:
+    """Value of each E2M1 code (0..15) from its fields."""
+    c = np.asarray(code, dtype=np.int64)
+    s = (c >> 3) & 1
+    e = (c >> 1) & 3
+    m = c & 1
+    v = np.where(e == 0, m * 0.5, np.ldexp(1.0 + m / 2.0, (e - 1).astype(np.int64)))
+    return np.where(s == 1, -v, v).astype(F64)
+
+
+def e2m1_round(v) -> np.ndarray:
+    """Nearest E2M1 value, ties to even, saturating at +-6 (2 significand bits,
+    smallest normal exponent 0, subnormal quantum 0.5)."""
+    return round_to_precision(v, 2, 0, E2M1_MAX, saturate=True)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """E2M1 code of e2m1_round(v); -0 keeps its sign bit."""
+    r = e2m1_round(v)
+    a = np.abs(r)
+    table = e2m1_decode(np.arange(8))
+    mag = np.searchsorted(table, a)            # exact: a is a table value
+    return (mag | (np.signbit(r).astype(np.int64) << 3)).astype(np.uint8)
+
+
+def _blocks(x, block):
+    x = np.asarray(x, dtype=F64).reshape(-1)
+    n = x.size
+    nb = -(-n // block)
+    xb = np.zeros(nb * block, dtype=F64)
+    xb[:n] = x
+    return xb.reshape(nb, block), n
+
+
+def mxfp4_quantize(x):
+    """(codes uint8 [n], scale exponents int [nb]) of MXFP4 with blocks of 32.
+
+    The scale of block b is 2^k_b, k_b = floor(log2 amax_b) - 2 (2^-127 for an
+    all-zero block); each element is e2m1_round(x / 2^k_b)."""
+    xb, n = _blocks(x, MX_BLOCK)
+    amax = np.abs(xb).max(axis=1)
+    with np.errstate(divide="ignore"):
+        _, e2 = np.frexp(amax)                  # amax = f 2^e2, f in [0.5, 1)
+    k = np.where(amax > 0, e2.astype(np.int64) - 1 - 2, -127)
+    k = np.clip(k, -127, 127)
+    y = xb / np.ldexp(1.0, k)[:, None]
+    codes = e2m1_encode(y).reshape(-1)[:n]
+    return codes, k
+
+
+def mxfp4_dequant(codes, k, n: int) -> np.ndarray:
+    v = e2m1_decode(codes)
+    return v * np.ldexp(1.0, np.asarray(k, dtype=np.int64)[np.arange(n) // MX_BLOCK])
+
+
+def nvfp4_quantize(x, tensor_scale: bool = True):
+    """(codes uint8 [n], E4M3 block scales as values [nb], fp32 tensor scale).
+
+    s_t = fl32(amax_tensor / 2688) with tensor_scale (2688 = 6 * 448), else 1;
+    block scale S_b = E4M3(amax_b / (6 s_t)); element = e2m1_round(x / (S_b s_t))
+    (0 where S_b = 0)."""
+    xb, n = _blocks(x, NV_BLOCK)
+    amax_t = float(np.abs(xb).max()) if xb.size else 0.0
+    s_t = float(fl32(amax_t / (E2M1_MAX * 448.0))) if tensor_scale and amax_t > 0 else 1.0
+    amax = np.abs(xb).max(axis=1)
+    S = e4m3_round(amax / (E2M1_MAX * s_t))
+    scale = S * s_t
+    safe = np.where(scale > 0, scale, 1.0)
+    y = np.where(scale[:, None] > 0, xb / safe[:, None], 0.0)
+    codes = e2m1_encode(y).reshape(-1)[:n]
+    return codes, S, s_t
+
+
+def nvfp4_dequant(codes, S, s_t: float, n: int) -> np.ndarray:
+    v = e2m1_decode(codes)
+    return v * (np.asarray(S, dtype=F64) * F64(s_t))[np.arange(n) // NV_BLOCK]
+
+
+def storage_bits_per_element(fmt: str) -> float:
+    """Bits per element including the block scales (MX: 8 per 32; NV: 8 per 16;
+    the single NVFP4 tensor scale is not counted)."""
+    return {"mxfp4": 4 + 8 / MX_BLOCK, "nvfp4": 4 + 8 / NV_BLOCK}[fmt]

@@ -1,0 +1,123 @@
+"""Pins for the oracle's MXFP4 / NVFP4 block formats (oracle/fp4.py): the E2M1
+grid from the format's fields, rounding checked by brute force over every
+candidate value, the MX scale rule, power-of-two invariance, exact blocks and
+the error bounds that follow from the grid spacing."""
+import numpy as np
+import pytest
+
+from oracle import fp4
+from oracle import formats as F
+
+GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def test_e2m1_values_from_fields():
+    assert np.array_equal(fp4.e2m1_decode(np.arange(8)), GRID)
+    assert np.array_equal(fp4.e2m1_decode(np.arange(8, 16)), -GRID)
+
+
+def _brute_round(v):
+    """Nearest of the 15 E2M1 values; a tie goes to the code whose mantissa bit
+    is 0; beyond 6 saturate."""
+    out = np.empty_like(v)
+    for i, x in enumerate(v):
+        a = min(abs(x), 6.0)
+        d = np.abs(GRID - a)
+        best = np.flatnonzero(d == d.min())
+        if best.size > 1:                              # a tie: the even code (mantissa bit 0)
+            best = [b for b in best if b % 2 == 0]
+        out[i] = np.copysign(GRID[best[0]], x)
+    return out
+
+
+def test_e2m1_round_bruteforce():
+    rng = np.random.default_rng(0)
+    mids = (GRID[1:] + GRID[:-1]) / 2
+    v = np.concatenate([rng.uniform(-9, 9, 4000), mids, -mids, GRID, -GRID, [6.5, 7.0, 7.9, 100.0, -7.0]])
+    assert np.array_equal(fp4.e2m1_round(v), _brute_round(v))
+
+
+def test_e2m1_encode_decode_roundtrip():
+    rng = np.random.default_rng(1)
+    v = rng.uniform(-8, 8, 2000)
+    assert np.array_equal(fp4.e2m1_decode(fp4.e2m1_encode(v)), fp4.e2m1_round(v))
+    assert fp4.e2m1_encode(np.array([-0.1]))[0] == 8      # -0 keeps its sign bit
+
+
+def test_mxfp4_scale_rule_and_bounds():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal(32 * 500) * np.repeat(np.exp(rng.uniform(-8, 8, 500)), 32)
+    codes, k = fp4.mxfp4_quantize(x)
+    amax = np.abs(x.reshape(-1, 32)).max(axis=1)
+    # the block maximum lands in [4, 8) after scaling
+    y = amax / np.ldexp(1.0, k)
+    assert np.all((y >= 4) & (y < 8))
+    xh = fp4.mxfp4_dequant(codes, k, x.size)
+    err = np.abs(xh - x).reshape(-1, 32)
+    sc = np.ldexp(1.0, k)[:, None]
+    ys = np.abs(x.reshape(-1, 32)) / sc
+    assert np.all(err[ys <= 6] <= (sc * np.ones_like(ys))[ys <= 6])      # half the widest step (4 -> 6)
+    assert np.all(err <= 2 * sc)                                         # (6, 8) saturates to 6
+
+
+def test_mxfp4_power_of_two_invariance():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(32 * 64)
+    c0, k0 = fp4.mxfp4_quantize(x)
+    for j in (-20, -3, 5, 17):
+        c, k = fp4.mxfp4_quantize(np.ldexp(x, j))
+        assert np.array_equal(c, c0) and np.array_equal(k, k0 + j)
+
+
+def test_mxfp4_exact_block_and_zero_block():
+    vals = np.array([6, -4, 3, 0.5, 0, -1.5, 2, 1] * 4) * 2.0 ** -5
+    codes, k = fp4.mxfp4_quantize(vals)
+    assert k[0] == -5
+    assert np.array_equal(fp4.mxfp4_dequant(codes, k, 32), vals)
+    codes, k = fp4.mxfp4_quantize(np.zeros(32))
+    assert k[0] == -127 and not codes.any()
+
+
+@pytest.mark.parametrize("tensor_scale", [False, True])
+def test_nvfp4_bounds(tensor_scale):
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal(16 * 800) * 0.02
+    codes, S, s_t = fp4.nvfp4_quantize(x, tensor_scale=tensor_scale)
+    # the block scales are E4M3 values
+    assert np.array_equal(F.e4m3_round(S), S)
+    xh = fp4.nvfp4_dequant(codes, S, s_t, x.size)
+    scale = (S * s_t)[:, None]
+    err = np.abs(xh - x).reshape(-1, 16)
+    amax = np.abs(x.reshape(-1, 16)).max(axis=1, keepdims=True)
+    # half the widest step is 1 scale unit; an element beyond 6 units (the scale
+    # rounded down) saturates, losing amax - 6 units at most
+    assert np.all(err <= np.maximum(scale, amax - 6 * scale) * (1 + 1e-12))
+    if tensor_scale:
+        # the tensor scale keeps every block scale in E4M3's normal range, where
+        # it rounds by at most 2^-4: the saturation loss stays below one unit
+        assert S.min() >= 2.0 ** -6 and S.max() <= 448
+        assert np.all(err <= scale * (1 + 1e-12))
+    else:
+        # 0.02-sigma weights put the block scales in E4M3's subnormal range
+        assert S.max() < 2.0 ** -6
+
+
+def test_nvfp4_exact_block():
+    S = 0.75 * 2.0 ** -3                         # an E4M3 value; amax = 6 S
+    vals = np.array([6, -4, 3, 0.5, 0, -1.5, 2, 1, -6, 4, -3, -0.5, 1.5, -2, -1, 0]) * S
+    codes, Sq, s_t = fp4.nvfp4_quantize(vals, tensor_scale=False)
+    assert s_t == 1.0 and Sq[0] == S
+    assert np.array_equal(fp4.nvfp4_dequant(codes, Sq, s_t, 16), vals)
+
+
+def test_nvfp4_tensor_scale_power_of_two_invariance():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(16 * 64)
+    c0, S0, t0 = fp4.nvfp4_quantize(x)
+    c1, S1, t1 = fp4.nvfp4_quantize(np.ldexp(x, -9))
+    assert np.array_equal(c0, c1) and np.array_equal(S0, S1) and t1 == np.ldexp(t0, -9)
+
+
+def test_storage_bits():
+    assert fp4.storage_bits_per_element("mxfp4") == 4.25
+    assert fp4.storage_bits_per_element("nvfp4") == 4.5

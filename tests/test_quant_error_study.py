@@ -22,7 +22,7 @@ Run with -s to print the table.
 """
 import numpy as np
 
-from oracle import nf4
+from oracle import fp4, nf4
 
 N_BLOCKS = 20000
 
@@ -42,8 +42,14 @@ def _study(seed=2024):
     y = xb / c
     e2m1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]) / 6.0
     packed, cc, _ = nf4.quantize(x.astype(np.float32))
+    e, s2, mu = nf4.double_quant(cc)
+    mx_codes, mx_k = fp4.mxfp4_quantize(x)
+    nv_codes, nv_S, nv_t = fp4.nvfp4_quantize(x)
     recon = {
         "nf4": nf4.dequant(packed, x.size, cc, out="f32").reshape(xb.shape),
+        "nf4_dq": nf4.dequant(packed, x.size, nf4.dq_constants(e, s2, mu), out="f32").reshape(xb.shape),
+        "mxfp4": fp4.mxfp4_dequant(mx_codes, mx_k, x.size).reshape(xb.shape),
+        "nvfp4": fp4.nvfp4_dequant(nv_codes, nv_S, nv_t, x.size).reshape(xb.shape),
         "int4_sym15": _nearest(np.arange(-7, 8) / 7.0, y) * c,
         "int4_16": _nearest(-1.0 + 2.0 * np.arange(16) / 15.0, y) * c,
         "fp4_e2m1": _nearest(np.concatenate([-e2m1[:0:-1], e2m1]), y) * c,
@@ -61,6 +67,22 @@ def test_nf4_has_the_lowest_error_on_normal_weights():
     # NF4 is worth about 1 dB of SQNR over the best of the others here
     best_other = min(nmse["int4_sym15"], nmse["int4_16"], nmse["fp4_e2m1"])
     assert -10 * np.log10(nmse["nf4"]) - (-10 * np.log10(best_other)) > 0.7
+
+
+def test_block_scaled_fp4_formats():
+    """MXFP4 (4.25 bits per element) and NVFP4 (4.5 bits, plus one fp32 tensor
+    scale) against NF4 with double-quantized constants (4.127 bits).  Measured
+    on normal data: NF4 has the lowest error, about 0.5 dB ahead of NVFP4 and
+    2 dB ahead of MXFP4.  NVFP4's blocks of 16 with fractional E4M3 scales
+    recover most of what E2M1's level spacing loses on a bell curve; MXFP4's
+    power-of-two scale leaves the block maximum anywhere in [4, 8) E2M1 units,
+    wasting part of the grid (and clipping (6, 8))."""
+    nmse = _study(seed=11)
+    for k in ("nf4_dq", "nvfp4", "mxfp4"):
+        print(f"{k:7s} NMSE {nmse[k]:.5f}  SQNR {-10 * np.log10(nmse[k]):.2f} dB")
+    assert nmse["nf4_dq"] < nmse["nvfp4"] < nmse["mxfp4"]
+    # double quantization of the constants costs NF4 almost nothing
+    assert nmse["nf4_dq"] < nmse["nf4"] * 1.01
 
 
 def test_nf4_error_in_the_expected_band():
