@@ -15,6 +15,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -62,6 +63,51 @@ bool pdl_enabled() {
     return !(e && e[0] == '0');
   }();
   return on;
+}
+
+namespace {
+struct PerDevice {
+  const void* key;
+  int tag, dev, val;
+};
+std::mutex g_pd_mu;
+std::vector<PerDevice> g_pd;
+}  // namespace
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) {
+    cudaGetLastError();
+    d = 0;
+  }
+  return d;
+}
+
+int per_device_impl(const void* key, int tag, const std::function<int()>& compute) {
+  const int dev = current_device();
+  {
+    std::lock_guard<std::mutex> g(g_pd_mu);
+    for (const PerDevice& e : g_pd)
+      if (e.key == key && e.tag == tag && e.dev == dev) return e.val;
+  }
+  const int v = compute();
+  if (v >= 0) {
+    std::lock_guard<std::mutex> g(g_pd_mu);
+    g_pd.push_back(PerDevice{key, tag, dev, v});   // two first calls may both add the same value
+  }
+  return v;
+}
+
+int device_sm_count() {
+  static const int key = 0;
+  return per_device(&key, 0, [] {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, current_device()) != cudaSuccess || c <= 0) {
+      cudaGetLastError();
+      return -1;
+    }
+    return c;
+  });
 }
 
 const NF4Table& nf4_table() {

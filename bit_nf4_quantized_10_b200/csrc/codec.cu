@@ -410,14 +410,23 @@ __global__ void __launch_bounds__(256) merge_kernel(const uint8_t* __restrict__ 
 
 // ------------------------------------------------------------------- launch
 static int sm_count() {
-  static int count = 0;
-  if (!count) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
-    if (count <= 0) count = 148;
-  }
-  return count;
+  const int c = device_sm_count();
+  return c > 0 ? c : 148;
+}
+
+// Resident 256-thread CTAs per SM of a streaming kernel (4 if the calculator
+// gives no answer).
+template <typename K>
+static int ctas_per_sm(K kernel) {
+  const int b = per_device(reinterpret_cast<const void*>(kernel), 1, [kernel] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      return -1;
+    }
+    return n;
+  });
+  return b > 0 ? b : 4;
 }
 
 static unsigned grid_for(int64_t work_items, int per_cta, int ctas_per_sm) {
@@ -431,14 +440,7 @@ ql_status launch_quantize(const void* x, ql_dtype dt, int64_t n, uint8_t* codes,
                           cudaStream_t st) {
   const int64_t nb = (n + 63) / 64;
   // one resident wave of CTAs (grid-stride loop), 32 blocks (8 warps x 4) per CTA iteration
-  static int per_sm[2] = {0, 0};
-  int& bps = per_sm[dt == QL_F32 ? 0 : 1];
-  if (!bps) {
-    const cudaError_t e = dt == QL_F32
-                              ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, quantize_kernel<float>, 256, 0)
-                              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, quantize_kernel<__nv_bfloat16>, 256, 0);
-    if (e != cudaSuccess || bps < 1) bps = 4;
-  }
+  const int bps = dt == QL_F32 ? ctas_per_sm(quantize_kernel<float>) : ctas_per_sm(quantize_kernel<__nv_bfloat16>);
   const unsigned grid = grid_for(nb, 32, bps);
   static const QuantBins bins = build_bins(nf4_table());
   TraceScope ts(TK_QUANTIZE, st);
@@ -508,13 +510,7 @@ ql_status launch_merge(const ql_nf4_weight* w, const void* A, const void* B, int
                        uint8_t* codes_out, float* absmax_out, cudaStream_t st) {
   const int64_t nb = w->rows * w->cols / 64;
   WeightConsts wc{w->absmax, w->absmax_q, w->scale2, w->offset};
-  static int bps = 0;
-  if (!bps) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, merge_kernel, 256, 0) != cudaSuccess || bps < 1) {
-      cudaGetLastError();
-      bps = 4;
-    }
-  }
+  const int bps = ctas_per_sm(merge_kernel);
   static const QuantBins bins = build_bins(nf4_table());
   TraceScope ts(TK_MERGE, st);
   QL_CUDA_TRY(launch(merge_kernel, dim3(grid_for(nb, 32, bps)), dim3(256), 0, st, 1, 1, w->codes, wc, w->rows, w->cols,

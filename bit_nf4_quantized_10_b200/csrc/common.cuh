@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cstdint>
+#include <functional>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -139,6 +141,19 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 bool pdl_enabled();
+
+// Host-side values of a (kernel, device) pair, such as a function attribute
+// that has been set or an occupancy answer, computed once per device: a process
+// may drive several devices, and host threads may launch concurrently.
+// `compute` runs outside the lock; its result is kept when it is >= 0 (a
+// negative result is an error and is computed again on the next call).
+int per_device_impl(const void* key, int tag, const std::function<int()>& compute);
+template <typename F>
+int per_device(const void* key, int tag, F&& compute) {
+  return per_device_impl(key, tag, std::function<int()>(std::forward<F>(compute)));
+}
+int current_device();
+int device_sm_count();
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, unsigned cluster_x,

@@ -569,12 +569,16 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
                                   const void* lora_b, int r, float s, void* out, ql_dtype out_dt, int accumulate,
                                   cudaStream_t st) {
   using namespace gemm;
-  static bool attr_set = false;
-  if (!attr_set) {
-    QL_CUDA_TRY(cudaFuncSetAttribute(qlora_gemm_kernel<BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)SMEM_BYTES));
-    attr_set = true;
-  }
+  // the shared-memory limit is a per-device attribute of the kernel
+  if (per_device(reinterpret_cast<const void*>(qlora_gemm_kernel<BWD>), 0, [] {
+        if (cudaFuncSetAttribute(qlora_gemm_kernel<BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)SMEM_BYTES) != cudaSuccess) {
+          cudaGetLastError();
+          return -1;
+        }
+        return 1;
+      }) < 0)
+    return QL_ERR_CUDA;
   const int N = (int)w->rows, K = (int)w->cols;
   CUtensorMap map_act, map_codes, map_out;
   const int red = BWD ? N : K;   // reduction length = activation row length

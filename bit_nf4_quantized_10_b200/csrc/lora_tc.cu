@@ -254,14 +254,8 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restri
 }  // namespace skinny
 
 static int sm_count_tc() {
-  static int count = 0;
-  if (!count) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
-    if (count <= 0) count = 148;
-  }
-  return count;
+  const int c = device_sm_count();
+  return c > 0 ? c : 148;
 }
 
 // One wave of clusters where the row tiles allow: the most splits (at most
@@ -299,25 +293,28 @@ static void split_plan_compute(bool a_mn, int rows, int64_t red, int& splits, in
   splits = (steps + per - 1) / per;
 }
 
-// The plan depends only on the shape; launches repeat the same few shapes.
+// The plan depends only on the shape and the device; launches repeat the same
+// few shapes.
 static void split_plan(bool a_mn, int rows, int64_t red, int& splits, int& per) {
   struct Entry {
     bool a_mn;
     int rows;
     int64_t red;
+    int dev;
     int splits, per;
   };
   static std::mutex mu;
   static std::vector<Entry> cache;
+  const int dev = current_device();
   std::lock_guard<std::mutex> lk(mu);
   for (const Entry& e : cache)
-    if (e.a_mn == a_mn && e.rows == rows && e.red == red) {
+    if (e.a_mn == a_mn && e.rows == rows && e.red == red && e.dev == dev) {
       splits = e.splits;
       per = e.per;
       return;
     }
   split_plan_compute(a_mn, rows, red, splits, per);
-  if (cache.size() < 256) cache.push_back(Entry{a_mn, rows, red, splits, per});
+  if (cache.size() < 256) cache.push_back(Entry{a_mn, rows, red, dev, splits, per});
 }
 
 // C = scale * Z_op G, see the file comment.  a_mn: Z_op is the transpose of a
@@ -328,14 +325,17 @@ static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, 
                                float scale, void* out_row, ql_dtype row_dt, void* out_t, int64_t ld_t, ql_dtype t_dt,
                                int kind, cudaStream_t st) {
   using namespace skinny;
-  static bool attr[2] = {false, false};
-  if (!attr[a_mn]) {
-    // two CTAs per SM need the largest shared-memory carveout
-    auto k = a_mn ? skinny_kernel<true> : skinny_kernel<false>;
-    QL_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES));
-    QL_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
-    attr[a_mn] = true;
-  }
+  // two CTAs per SM need the largest shared-memory carveout (per-device attributes)
+  auto k = a_mn ? skinny_kernel<true> : skinny_kernel<false>;
+  if (per_device(reinterpret_cast<const void*>(k), 0, [k] {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) {
+          cudaGetLastError();
+          return -1;
+        }
+        return 1;
+      }) < 0)
+    return QL_ERR_CUDA;
   const int rp = (r + 15) / 16 * 16;
   CUtensorMap ma, mb;
   if (a_mn) {

@@ -58,9 +58,8 @@ __global__ void __launch_bounds__(256) silu_gate_bwd_kernel(const uint4* __restr
 }
 
 static unsigned elem_grid(int64_t n8) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int c = device_sm_count();
+  const int sms = c > 0 ? c : 148;
   int64_t need = (n8 + 255) / 256;
   int64_t cap = (int64_t)sms * 8;
   return (unsigned)(need < 1 ? 1 : (need < cap ? need : cap));

@@ -26,6 +26,8 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -444,14 +446,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 }  // namespace smallm
 
 static int sm_count_sm() {
-  static int count = 0;
-  if (!count) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
-    if (count <= 0) count = 148;
-  }
-  return count;
+  const int c = device_sm_count();
+  return c > 0 ? c : 148;
 }
 
 struct SmallmPlan {
@@ -483,17 +479,16 @@ static bool smallm_layout(int per, SmallmPlan& pl) {
 }
 
 static bool smallm_attr() {
-  static bool set = false;
-  if (!set) {
-    if (cudaFuncSetAttribute(smallm::smallm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(227 * 1024 - smallm_static_smem())) != cudaSuccess)
-      return false;
-    if (cudaFuncSetAttribute(smallm::smallm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
-        cudaSuccess)
-      return false;
-    set = true;
-  }
-  return true;
+  return per_device(reinterpret_cast<const void*>(smallm::smallm_kernel), 0, [] {
+           if (cudaFuncSetAttribute(smallm::smallm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)(227 * 1024 - smallm_static_smem())) != cudaSuccess ||
+               cudaFuncSetAttribute(smallm::smallm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+                   cudaSuccess) {
+             cudaGetLastError();
+             return -1;
+           }
+           return 1;
+         }) > 0;
 }
 
 // Cluster size (CTAs sharing K) and cluster count: the tiles are handed out in
@@ -558,15 +553,32 @@ ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, co
   if (M < 1 || M > TN || r > MAX_R) return QL_ERR_UNSUPPORTED;
   const int N = (int)w->rows, K = (int)w->cols;
   if (!smallm_attr()) return QL_ERR_CUDA;
-  // the plan for a weight shape is fixed, so it is computed once per shape
-  static int64_t cached_N = -1, cached_K = -1;
-  static SmallmPlan cached;
-  if (N != cached_N || K != cached_K) {
-    if (!smallm_plan(N, K, cached, true)) return QL_ERR_UNSUPPORTED;
-    cached_N = N;
-    cached_K = K;
+  // the plan for a weight shape is fixed: computed once per shape and device
+  // (the layers of a model alternate a few shapes)
+  struct Entry {
+    int64_t N, K;
+    int dev;
+    SmallmPlan pl;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  const int dev = current_device();
+  SmallmPlan pl;
+  bool have = false;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (const Entry& e : cache)
+      if (e.N == N && e.K == K && e.dev == dev) {
+        pl = e.pl;
+        have = true;
+        break;
+      }
   }
-  const SmallmPlan pl = cached;
+  if (!have) {
+    if (!smallm_plan(N, K, pl, true)) return QL_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache.size() < 256) cache.push_back(Entry{N, K, dev, pl});
+  }
   CUtensorMap map_x, map_codes;
   if (!make_map_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, TN,
                    CU_TENSOR_MAP_SWIZZLE_128B))
