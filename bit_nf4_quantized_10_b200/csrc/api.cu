@@ -3,6 +3,8 @@
 #include <algorithm>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace ql {
@@ -109,9 +111,20 @@ size_t ws_bwd(int64_t M, int64_t N, int64_t K, int r) { return ws_bwd_layout(M, 
 
 }  // namespace
 
+// An NVTX range around each public call ("qlora_nf4/<call>"), so a timeline
+// profiler shows which library call launched which kernels.  Without a tool
+// attached the push and pop do nothing.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 extern "C" {
 
 ql_status nf4_quantize(const void* x, ql_dtype x_dt, int64_t n, uint8_t* codes, float* absmax, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/nf4_quantize");
   if (n <= 0 || !dtype_ok(x_dt)) return QL_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(absmax)) return QL_ERR_INVALID_ARG;
   return ql::launch_quantize(x, x_dt, n, codes, absmax, as_stream(stream));
@@ -119,6 +132,7 @@ ql_status nf4_quantize(const void* x, ql_dtype x_dt, int64_t n, uint8_t* codes, 
 
 ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q, float* scale2, float* offset,
                            void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/nf4_double_quant");
   if (nb <= 0) return QL_ERR_INVALID_ARG;
   if (!aligned16(absmax) || !aligned16(absmax_q) || !aligned16(scale2) || !aligned16(offset) || !aligned16(ws))
     return QL_ERR_INVALID_ARG;
@@ -127,6 +141,7 @@ ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q, f
 }
 
 ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/nf4_dequant");
   ql_status st = check_weight(w);
   if (st != QL_OK) return st;
   if (!dtype_ok(out_dt) || !aligned16(out)) return QL_ERR_INVALID_ARG;
@@ -135,6 +150,7 @@ ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* 
 
 ql_status qlora_merge(const ql_nf4_weight* w, const void* A, const void* B, int r, float s, void* W_out,
                       uint8_t* codes_out, float* absmax_out, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/qlora_merge");
   ql_status st = check_weight(w);
   if (st != QL_OK) return st;
   if (w->cols % 64 != 0) return QL_ERR_INVALID_ARG;
@@ -151,6 +167,7 @@ ql_status qlora_merge(const ql_nf4_weight* w, const void* A, const void* B, int 
 
 ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* A, const void* B, int r,
                            float s, void* Y, ql_dtype y_dt, void* U_out, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/qlora_linear_fwd");
   ql_status st = check_gemm_shape(w, M, r);
   if (st != QL_OK) return st;
   if (!dtype_ok(y_dt) || !aligned16(X) || !aligned16(Y)) return QL_ERR_INVALID_ARG;
@@ -175,6 +192,7 @@ ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, con
 ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
                            const void* B, int r, float s, const void* U, void* dX, ql_dtype dx_dt, int accumulate_dx,
                            void* dA, void* dB, ql_dtype grad_dt, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/qlora_linear_bwd");
   ql_status st = check_gemm_shape(w, M, r);
   if (st != QL_OK) return st;
   if (!dtype_ok(dx_dt) || !dtype_ok(grad_dt) || !aligned16(dY) || !aligned16(dX)) return QL_ERR_INVALID_ARG;
@@ -225,12 +243,14 @@ ql_status qlora_selftest_wait_timeout(int64_t polls, void* stream) {
 }
 
 ql_status qlora_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/qlora_silu_gate_fwd");
   if (n <= 0 || !aligned16(g) || !aligned16(u) || !aligned16(h)) return QL_ERR_INVALID_ARG;
   return ql::launch_silu_gate_fwd(g, u, h, n, as_stream(stream));
 }
 
 ql_status qlora_silu_gate_bwd(const void* dh, const void* g, const void* u, void* dg, void* du, int64_t n,
                               void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/qlora_silu_gate_bwd");
   if (n <= 0 || !aligned16(dh) || !aligned16(g) || !aligned16(u) || !aligned16(dg) || !aligned16(du))
     return QL_ERR_INVALID_ARG;
   return ql::launch_silu_gate_bwd(dh, g, u, dg, du, n, as_stream(stream));
