@@ -24,12 +24,14 @@ Readings (the pages fix none of these steps):
   - NVFP4 scale: E4M3(amax / 6) per block of 16, round to nearest even,
     saturating at 448, so the largest element maps to about 6.  E4M3 spans
     2^-9 .. 448; with `tensor_scale`, one fp32 scale per tensor, s_t =
-    fl32(amax_tensor / (6 * 448)), divides every block scale first
-    (E4M3(amax_b / (6 s_t))) and multiplies back on dequantization, so the
-    block scales of small weights use E4M3's normal range.  A block whose
-    scale rounds to 0 stores zeros.
-  - Element codes: the rounding of x / scale (the scale as decoded), computed
-    in float64 (the division is exact enough: one rounding to E2M1 follows).
+    fl32(amax_tensor / (6 * 448)), divides every block scale first and
+    multiplies back on dequantization, so the block scales of small weights
+    use E4M3's normal range.  A block whose scale rounds to 0 stores zeros.
+  - The scale steps are fp32 operations, each rounded once, in this order (a
+    kernel takes the same integer decisions):
+      denom = fl32(6 s_t),  S = E4M3(fl32(amax_b / denom)),
+      scale = fl32(S s_t),  code = E2M1(fl32(x / scale)),
+      x_hat = fl32(E2M1(code) scale).
 
 Parity: pinned by tests/test_oracle_fp4.py (E2M1 grid from the format's fields,
 brute-force nearest-even rounding, power-of-two scale invariance, exact blocks,
@@ -105,23 +107,26 @@ def nvfp4_quantize(x, tensor_scale: bool = True):
     """(codes uint8 [n], E4M3 block scales as values [nb], fp32 tensor scale).
 
     s_t = fl32(amax_tensor / 2688) with tensor_scale (2688 = 6 * 448), else 1;
-    block scale S_b = E4M3(amax_b / (6 s_t)); element = e2m1_round(x / (S_b s_t))
-    (0 where S_b = 0)."""
+    then the fp32 steps of the module docstring; an element of a block whose
+    scale is 0 codes as 0."""
     xb, n = _blocks(x, NV_BLOCK)
     amax_t = float(np.abs(xb).max()) if xb.size else 0.0
     s_t = float(fl32(amax_t / (E2M1_MAX * 448.0))) if tensor_scale and amax_t > 0 else 1.0
     amax = np.abs(xb).max(axis=1)
-    S = e4m3_round(amax / (E2M1_MAX * s_t))
-    scale = S * s_t
+    denom = fl32(E2M1_MAX * s_t)
+    S = e4m3_round(fl32(amax / denom))
+    scale = fl32(S * s_t)
     safe = np.where(scale > 0, scale, 1.0)
-    y = np.where(scale[:, None] > 0, xb / safe[:, None], 0.0)
+    y = np.where(scale[:, None] > 0, fl32(xb / safe[:, None]), 0.0)
     codes = e2m1_encode(y).reshape(-1)[:n]
     return codes, S, s_t
 
 
 def nvfp4_dequant(codes, S, s_t: float, n: int) -> np.ndarray:
+    """x_hat = fl32(E2M1(code) fl32(S s_t))."""
     v = e2m1_decode(codes)
-    return v * (np.asarray(S, dtype=F64) * F64(s_t))[np.arange(n) // NV_BLOCK]
+    scale = fl32(np.asarray(S, dtype=F64) * F64(s_t))
+    return fl32(v * scale[np.arange(n) // NV_BLOCK])
 
 
 def storage_bits_per_element(fmt: str) -> float:
