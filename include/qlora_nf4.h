@@ -120,6 +120,8 @@ ql_status nf4_quantize(const void* x, ql_dtype x_dt, int64_t n,
  * (zero padded to a power of two).  Per group of 256: d = fl32(c - mu),
  * s_2 = fl32(max|d| / 448), code = E4M3_rne_satfinite(fl32(d / s_2)); a group
  * with s_2 == 0 stores code 0x00.
+ * Errors: QL_ERR_INVALID_ARG (nb <= 0, a NULL or misaligned pointer),
+ * QL_ERR_WORKSPACE (ws_bytes too small), QL_ERR_CUDA.
  */
 ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q,
                            float* scale2, float* offset, void* ws, size_t ws_bytes,
@@ -181,6 +183,8 @@ ql_status qlora_merge(const ql_nf4_weight* w, const void* A, const void* B, int 
  * paragraph"; [P2] §3 dequantize to BF16), c = absmax[b] or the double-quant
  * reconstruction when w->absmax is NULL.  out: device, rows*cols elements of
  * out_dt (QL_F32 skips the bf16 rounding).
+ * Errors: QL_ERR_INVALID_ARG (NULL w, rows or cols <= 0, a misaligned weight
+ * buffer or output, an unknown dtype), QL_ERR_CUDA.
  */
 ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* stream);
 
@@ -199,6 +203,11 @@ ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* 
  * bf16 W_hat.  U is accumulated in fp32 (split over K, summed in a fixed
  * order) and rounded to bf16; the adapter term U (s B)^T enters the main fp32
  * accumulator with s B rounded to bf16 (exact when s is a power of two).
+ * M == 0 launches nothing.  Errors: QL_ERR_INVALID_ARG (bad weight
+ * descriptor, M < 0, K % 64 or N % 8 != 0, r < 0 or r % 8 != 0, a NULL or
+ * misaligned pointer, an unknown dtype), QL_ERR_UNSUPPORTED (r > QL_MAX_RANK,
+ * M, N or K >= 2^31), QL_ERR_WORKSPACE (ws_bytes too small), QL_ERR_CUDA; a
+ * bounded device wait that ran out sets QL_ERR_TIMEOUT in the status word.
  */
 ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M,
                            const void* A, const void* B, int r, float s,
@@ -216,6 +225,8 @@ ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M,
  *   X, dY, A, B: device bf16;  U: device bf16 [M, r] from the forward, or NULL
  *   to recompute it.  dX of dx_dt; dA, dB of grad_dt (overwritten).
  *   ws >= qlora_workspace_size(QL_OP_BWD, M, N, K, r).
+ * M == 0 only zeroes dA and dB.  Errors: as qlora_linear_fwd; U may be NULL
+ * (it is then recomputed) but must be 16-byte aligned when given.
  */
 ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY, int64_t M,
                            const void* A, const void* B, int r, float s, const void* U,
@@ -229,7 +240,8 @@ ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY
  *   qlora_silu_gate_fwd: h = bf16(silu(g) * u), silu(x) = x * sigmoid(x)
  *   qlora_silu_gate_bwd: dg = bf16(dh * u * sig(g) * (1 + g (1 - sig(g)))),
  *                        du = bf16(dh * silu(g))
- * All device bf16 [n].
+ * All device bf16 [n], n % 8 == 0.  Errors: QL_ERR_INVALID_ARG (n <= 0, a
+ * NULL or misaligned pointer), QL_ERR_UNSUPPORTED (n % 8 != 0), QL_ERR_CUDA.
  */
 ql_status qlora_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, void* stream);
 ql_status qlora_silu_gate_bwd(const void* dh, const void* g, const void* u,
