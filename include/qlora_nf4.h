@@ -104,6 +104,8 @@ typedef struct {
  * every element as the zero level (8).  An odd n pads the last high nibble
  * with 8.  NaN/Inf in a block sets QL_ERR_NONFINITE in the status word
  * (that block's outputs are then unspecified).  n may exceed 2^32.
+ * Errors: QL_ERR_INVALID_ARG (n <= 0, a NULL or misaligned pointer, an
+ * unknown dtype), QL_ERR_CUDA.
  */
 ql_status nf4_quantize(const void* x, ql_dtype x_dt, int64_t n,
                        uint8_t* codes, float* absmax, void* stream);
@@ -225,8 +227,10 @@ ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M,
  *   X, dY, A, B: device bf16;  U: device bf16 [M, r] from the forward, or NULL
  *   to recompute it.  dX of dx_dt; dA, dB of grad_dt (overwritten).
  *   ws >= qlora_workspace_size(QL_OP_BWD, M, N, K, r).
- * M == 0 only zeroes dA and dB.  Errors: as qlora_linear_fwd; U may be NULL
- * (it is then recomputed) but must be 16-byte aligned when given.
+ * M == 0 only zeroes dA and dB.  Errors: those of qlora_linear_fwd
+ * (QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_WORKSPACE, QL_ERR_CUDA;
+ * QL_ERR_TIMEOUT in the status word); U may be NULL (it is then recomputed)
+ * but must be 16-byte aligned when given.
  */
 ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY, int64_t M,
                            const void* A, const void* B, int r, float s, const void* U,

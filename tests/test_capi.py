@@ -93,3 +93,16 @@ def test_argument_errors_return_before_launch(lib):
     assert lib.status_string(lib.QL_ERR_TIMEOUT) == "device wait timed out"
     for polls in (0, -1, (1 << 20) + 1):
         assert L.qlora_selftest_wait_timeout(polls, s0) == lib.QL_ERR_INVALID_ARG
+
+
+def test_boundary_calls_document_source_and_errors():
+    """Each call of the hot path's boundary cites the passage it restates and
+    states its error behaviour in the header comment right above it."""
+    text = open(os.path.join(ROOT, "include", "qlora_nf4.h")).read()
+    for name in ("nf4_quantize", "nf4_double_quant", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
+                 "qlora_merge"):
+        m = re.search(r"/\*((?:(?!\*/).)*?)\*/\s*(?:#define[^\n]*\n\s*)?ql_status\s+" + name + r"\s*\(", text, flags=re.S)
+        assert m, name
+        comment = m.group(1)
+        assert re.search(r"\[P[1-5]\]", comment), f"{name}: no source citation"
+        assert "QL_ERR" in comment, f"{name}: no error behaviour"
