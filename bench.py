@@ -528,8 +528,11 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.warmup):
         wl.step(allreduce)
     torch.cuda.synchronize()
-    while not args.profile and time.time() - t_warm < 0.5:   # clock samples under load
-        wl.step(allreduce)
+    # clock samples under load: a wall-clock bound, so the step count differs
+    # between ranks; these steps therefore skip the collective (every rank must
+    # issue the same all-reduces in the same order)
+    while not args.profile and time.time() - t_warm < 0.5:
+        wl.step(None)
         torch.cuda.synchronize()
     st = q.qlora_get_status()
     if st != q.QL_OK:
