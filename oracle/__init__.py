@@ -18,4 +18,4 @@ function.  Parity status per function is in its docstring; every function here
 is pinned by a test under tests/ against something other than itself, except
 where a docstring says "parity unpinned".
 """
-from . import formats, nf4, lora, fp4  # noqa: F401
+from . import formats, nf4, lora, fp4, adamw  # noqa: F401
