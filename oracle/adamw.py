@@ -47,3 +47,33 @@ def adamw_step(p, g, m, v, t: int, lr: float, b1: float = 0.9, b2: float = 0.999
     vhat = v / (1.0 - b2 ** t)
     p = p - lr * mhat / (np.sqrt(vhat) + eps)
     return p, m, v
+
+
+def adamw_step_fp32(p, g, m, v, t: int, lr: float, b1: float = 0.9, b2: float = 0.999, eps: float = 1e-8,
+                    wd: float = 0.0):
+    """The same step as single fp32 operations in a fixed order (what a kernel
+    with fp32 states computes; "paged_adamw_32bit").  Constants are fp32, the
+    bias corrections from the fp32 betas (so 1 - b1 and the t = 1 correction
+    are the same number):
+        b1, b2, lr, eps = fl32(.);  keep = fl32(1 - lr wd)
+        c1 = fl32(1 - b1^t), c2 = fl32(1 - b2^t)   (power in float64)
+        p  = fl32(p keep)
+        m  = fl32(fl32(b1 m) + fl32((1 - b1) g))
+        v  = fl32(fl32(b2 v) + fl32(fl32((1 - b2) g) g))
+        d  = fl32(fl32(sqrt(fl32(v / c2))) + eps)
+        p  = fl32(p - fl32(lr fl32(fl32(m / c1) / d)))
+    Each line's float64 operation followed by fl32 is the fp32 operation itself
+    (formats.py; the same holds for sqrt).  Returns (p, m, v) as fp32 values."""
+    from .formats import fl32
+    f = lambda x: fl32(np.asarray(x, dtype=F64))
+    p, g, m, v = f(p), f(g), f(m), f(v)
+    lr_, b1_, b2_, eps_ = (float(f(x)) for x in (lr, b1, b2, eps))
+    keep = float(f(1.0 - lr * wd))
+    c1, c2 = float(f(1.0 - b1_ ** t)), float(f(1.0 - b2_ ** t))
+    omb1, omb2 = float(f(1.0 - b1_)), float(f(1.0 - b2_))
+    p = f(p * keep)
+    m = f(f(b1_ * m) + f(omb1 * g))
+    v = f(f(b2_ * v) + f(f(omb2 * g) * g))
+    d = f(f(np.sqrt(f(v / c2))) + eps_)
+    p = f(p - f(lr_ * f(f(m / c1) / d)))
+    return p, m, v

@@ -38,3 +38,31 @@ def test_matches_torch_adamw_over_steps():
         opt.step()
         p, m, v = adamw.adamw_step(p, g, m, v, t, lr=lr, b1=b1, b2=b2, eps=eps, wd=wd)
     assert np.allclose(p, tp.detach().numpy(), rtol=0, atol=1e-14)
+
+
+def test_fp32_form_tracks_the_float64_update():
+    # the fp32 step differs from the float64 one only by fp32 roundings
+    rng = np.random.default_rng(2)
+    p0 = rng.standard_normal(4096).astype(np.float32).astype(np.float64)
+    p, m, v = p0.copy(), np.zeros(4096), np.zeros(4096)
+    q, mq, vq = p0.copy(), np.zeros(4096), np.zeros(4096)
+    for t in range(1, 6):
+        g = rng.standard_normal(4096).astype(np.float32).astype(np.float64)
+        p, m, v = adamw.adamw_step(p, g, m, v, t, lr=1e-3, wd=0.01)
+        q, mq, vq = adamw.adamw_step_fp32(q, g, mq, vq, t, lr=1e-3, wd=0.01)
+    assert np.all(q == q.astype(np.float32).astype(np.float64))      # fp32 values
+    assert np.max(np.abs(q - p)) < 5 * 2.0 ** -24 * np.max(np.abs(p))
+    # the fp32 betas differ from the float64 ones by ~1e-8; m can cancel to near
+    # zero, so its error is measured against its scale
+    assert np.max(np.abs(mq - m)) < 1e-6 * np.max(np.abs(m))
+
+
+def test_fp32_form_first_step_is_plus_minus_lr_when_eps_is_zero():
+    rng = np.random.default_rng(3)
+    p = np.zeros(256)
+    g = rng.standard_normal(256).astype(np.float32).astype(np.float64)
+    q, _, _ = adamw.adamw_step_fp32(p, g, np.zeros(256), np.zeros(256), 1, lr=0.5, eps=0.0)
+    # m / c1 = g (1 - b1 and 1 - b1^1 are the same fp32 number) and sqrt(v / c2) = |g|
+    # up to a few roundings, so the step is 0.5 to within a few fp32 ulps
+    assert np.allclose(np.abs(q), 0.5, rtol=8 * 2.0 ** -24, atol=0)
+    assert np.array_equal(np.sign(q), -np.sign(g))
