@@ -55,7 +55,7 @@ def adamw_step_fp32(p, g, m, v, t: int, lr: float, b1: float = 0.9, b2: float = 
     with fp32 states computes; "paged_adamw_32bit").  Constants are fp32, the
     bias corrections from the fp32 betas (so 1 - b1 and the t = 1 correction
     are the same number):
-        b1, b2, lr, eps = fl32(.);  keep = fl32(1 - lr wd)
+        b1, b2, lr, eps, wd = fl32(.);  keep = fl32(1 - lr wd)  (product in float64)
         c1 = fl32(1 - b1^t), c2 = fl32(1 - b2^t)   (power in float64)
         p  = fl32(p keep)
         m  = fl32(fl32(b1 m) + fl32((1 - b1) g))
@@ -68,7 +68,7 @@ def adamw_step_fp32(p, g, m, v, t: int, lr: float, b1: float = 0.9, b2: float = 
     f = lambda x: fl32(np.asarray(x, dtype=F64))
     p, g, m, v = f(p), f(g), f(m), f(v)
     lr_, b1_, b2_, eps_ = (float(f(x)) for x in (lr, b1, b2, eps))
-    keep = float(f(1.0 - lr * wd))
+    keep = float(f(1.0 - lr_ * float(f(wd))))   # from the fp32 lr and wd, product in float64
     c1, c2 = float(f(1.0 - b1_ ** t)), float(f(1.0 - b2_ ** t))
     omb1, omb2 = float(f(1.0 - b1_)), float(f(1.0 - b2_))
     p = f(p * keep)
