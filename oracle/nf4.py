@@ -198,8 +198,20 @@ def double_quant(c: np.ndarray):
     """
     c = fl32(np.asarray(c, dtype=F64))
     nb = c.size
-    ng = -(-nb // DQ_GROUP)
     mu = float(fl32(tree_sum_f64(c) / nb)) if nb else 0.0
+    e, s2 = dq_encode(c, mu)
+    return e, s2, mu
+
+
+def dq_encode(c: np.ndarray, mu: float):
+    """The per-group part of double_quant for a given mean: (codes, s2).
+
+    A tensor quantized in shards aligned to groups of 256 constants gets the
+    whole tensor's codes when every shard is encoded with the whole tensor's
+    mean."""
+    c = fl32(np.asarray(c, dtype=F64))
+    nb = c.size
+    ng = -(-nb // DQ_GROUP)
     d = fl32(c - mu)
     pad = np.zeros(ng * DQ_GROUP, dtype=F64)
     pad[:nb] = np.abs(d)
@@ -210,7 +222,7 @@ def double_quant(c: np.ndarray):
         ratio = fl32(np.where(s2_b != 0.0, d / np.where(s2_b != 0.0, s2_b, 1.0), 0.0))
     e = e4m3_encode(ratio)
     e = np.where(s2_b == 0.0, 0, e).astype(np.uint8)
-    return e, s2, mu
+    return e, s2
 
 
 def dq_constants(e: np.ndarray, s2: np.ndarray, mu: float) -> np.ndarray:

@@ -13,6 +13,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 from bit_nf4_quantized_10_b200.dp import token_shard, allreduce_adapter_grads
+from oracle import formats as F
 from oracle import lora, nf4
 from synthetic import inputs as S
 
@@ -72,3 +73,51 @@ def test_token_shards_partition_the_batch(m, world):
         assert b0 == a1
     sizes = [b - a for a, b in spans]
     assert max(sizes) - min(sizes) <= 1
+
+
+# ------------------------------------------------ quantization sharded by rows
+# Each rank quantizes a slab of weight rows whose block constants start on a
+# multiple of 2048 (a subtree of the double-quant mean's fixed adjacent-pair
+# tree).  It reduces its constants to level-1 tree nodes (one float64 sum per
+# 2048 constants), the ranks all-gather the nodes in rank order, and each
+# finishes the tree: the mean is the single-process mean bit for bit, so every
+# rank's E4M3 codes and group scales are the matching slice of the
+# single-process ones (groups of 256 never straddle a slab).
+KQ = 4096                       # 64 constants per row, 32 rows per 2048 constants
+CHUNK = 2048
+
+
+def _quant_shard_worker(rank, world, port, n_rows, rows_split):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        W = S.custom_weight(n_rows, KQ, 0.02, 21)
+        r0, r1 = rows_split[rank], rows_split[rank + 1]
+        _, c_r, _ = nf4.quantize(W[r0:r1])
+        nodes = np.array([nf4.tree_sum_f64(c_r[i:i + CHUNK]) for i in range(0, c_r.size, CHUNK)])
+        counts = [torch.zeros(1, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(counts, torch.tensor([nodes.size], dtype=torch.int64))
+        most = max(int(c.item()) for c in counts)
+        mine = torch.zeros(most, dtype=torch.float64)
+        mine[:nodes.size] = torch.from_numpy(nodes)
+        gathered = [torch.zeros(most, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(gathered, mine)
+        all_nodes = np.concatenate([g.numpy()[:int(c.item())] for g, c in zip(gathered, counts)])
+        nb_total = n_rows * KQ // 64
+        mu = float(F.fl32(nf4.tree_sum_f64(all_nodes) / nb_total))
+        e_r, s2_r = nf4.dq_encode(c_r, mu)
+        # the single-process result
+        _, c, _ = nf4.quantize(W)
+        e, s2, mu_ref = nf4.double_quant(c)
+        assert np.float32(mu).view(np.uint32) == np.float32(mu_ref).view(np.uint32), (rank, mu, mu_ref)
+        b0, b1 = r0 * KQ // 64, r1 * KQ // 64
+        assert np.array_equal(e_r, e[b0:b1])
+        assert np.array_equal(s2_r, s2[b0 // 256:-(-b1 // 256)])
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("n_rows,rows_split", [(128, [0, 64, 128]), (100, [0, 64, 100])])
+def test_double_quant_sharded_by_rows_gloo(n_rows, rows_split):
+    mp.spawn(_quant_shard_worker, args=(2, _free_port(), n_rows, rows_split), nprocs=2, join=True)
