@@ -106,3 +106,16 @@ def test_boundary_calls_document_source_and_errors():
         comment = m.group(1)
         assert re.search(r"\[P[1-5]\]", comment), f"{name}: no source citation"
         assert "QL_ERR" in comment, f"{name}: no error behaviour"
+
+
+@pytest.mark.parametrize("M,N,K,r", [(4096, 4096, 4096, 16), (130, 512, 1024, 16), (1, 28672, 8192, 64),
+                                     (600, 384, 320, 8), (16, 256, 512, 8)])
+def test_workspace_sizes_follow_the_documented_layout(lib, M, N, K, r):
+    """Forward: U [M, r] bf16.  Backward: B^T [r, N], U^T [r, Mp], V [M, r],
+    V^T [r, Mp] bf16 (Mp = M rounded up to 8), each piece 256-byte aligned."""
+    a256 = lambda b: (b + 255) // 256 * 256
+    Mp = (M + 7) // 8 * 8
+    assert lib.qlora_workspace_size(lib.QL_OP_FWD, M, N, K, r) == a256(M * r * 2)
+    want = a256(r * N * 2) + a256(r * Mp * 2) + a256(M * r * 2) + a256(r * Mp * 2)
+    assert lib.qlora_workspace_size(lib.QL_OP_BWD, M, N, K, r) == want
+    assert lib.qlora_workspace_size(lib.QL_OP_BWD, M, N, K, 0) == 0
