@@ -114,8 +114,9 @@ def test_projection_sized_weight_full(q):
 
 def test_codec_4gi_bf16_sampled(q):
     """4 Gi bf16 elements (64-bit indexing): every absmax, E4M3 code, scale and
-    the mean bit-exact; packed codes on sampled blocks, including blocks past
-    element 2^32 and the last block."""
+    the mean bit-exact; packed codes on sampled blocks, including the blocks on
+    both sides of element 2^31 (where 32-bit signed indexing would overflow)
+    and the last block."""
     n = 4 * 2 ** 30
     x = S.codec_tensor(n, 0.02, S.seed_of(5, 9, "W"), device="cuda")
     w, absmax = gpu_codec(q, x)
@@ -134,12 +135,13 @@ def test_codec_4gi_bf16_sampled(q):
     assert np.array_equal(f32_bits_t(w.scale2), F.f32_bits(s2))
     assert np.array_equal(np_u8(w.absmax_q), e)
     rng = np.random.default_rng(0)
-    blocks = np.unique(np.concatenate([rng.integers(0, nb, 200), [0, nb - 1, 2 ** 26 - 1, (2 ** 32) // 64,
-                                                                    (2 ** 32) // 64 + 1]]))
+    blocks = np.unique(np.concatenate([rng.integers(0, nb, 200), [0, nb - 1, 2 ** 25 - 1, 2 ** 25, 2 ** 25 + 1]]))
+    assert blocks.max() < nb
     codes_dev = w.codes
     for b in blocks:
         b = int(b)
         xb = x[b * 64:(b + 1) * 64].cpu()
+        assert xb.numel() == 64
         packed, cb, _ = nf4.quantize(xb)
         assert np.array_equal(np_u8(codes_dev[b * 32:(b + 1) * 32]), packed), b
 

@@ -104,39 +104,31 @@ def test_mlp_chain_reduced_tokens(q):
         assert_chain_close(np64(got), b[name], np.inf, name)
 
 
-def mlp_x(c):
-    return c["X"]
+def _rows_of(d, rows, keys):
+    return {k: (v[rows] if k in keys else v) for k, v in d.items()}
 
 
-def dy_of(c):
-    return c["dy"]
-
-
-def test_mlp_chain_full_size_sampled_tokens(q):
-    """The 7B MLP workload at full size (8192 tokens); forward output and dX are
-    per-token, so sampled token rows are checked against the oracle row by row;
-    the adapter gradients are checked through <dA, A> = <dB, B> relations."""
+def test_mlp_chain_full_size(q):
+    """The 7B MLP workload at full size (8192 tokens, r = 64).  The oracle runs
+    the whole chain on every token; the six adapter gradients are compared
+    element by element in full, and y and dX (per token) on sampled token rows
+    with the bound of a one-ulp flip in every bf16 intermediate."""
     w = S.WORKLOADS["c3"]
     D, H, M, r, s = 4096, 11008, w.M, w.r, w.s
     c = _mlp_case(D, H, M, r, seed=3000)
     mlp, y = _run_gpu_mlp(q, c, r, s)
+    Wg, Wu, Wd = _oracle_weight(c["Wg"]), _oracle_weight(c["Wu"]), _oracle_weight(c["Wd"])
+    args = (c["X"], Wg, c["Ag"], c["Bg"], Wu, c["Au"], c["Bu"], Wd, c["Ad"], c["Bd"], s)
+    f = lora.mlp_forward(*args)
+    b = lora.mlp_backward(*args, c["dy"], f)
+    for name, got in (("dAg", mlp.dAg), ("dBg", mlp.dBg), ("dAu", mlp.dAu), ("dBu", mlp.dBu),
+                      ("dAd", mlp.dAd), ("dBd", mlp.dBd)):
+        assert_fp_close(np64(got), b[name], name)
     rows = np.array([0, 1, 77, 1000, 4095, 4096, 6000, M - 1])
     sub = dict(c)
     sub["X"], sub["dy"] = c["X"][rows], c["dy"][rows]
-    Wg, Wu, Wd = _oracle_weight(c["Wg"]), _oracle_weight(c["Wu"]), _oracle_weight(c["Wd"])
-    args = (sub["X"], Wg, c["Ag"], c["Bg"], Wu, c["Au"], c["Bu"], Wd, c["Ad"], c["Bd"], s)
-    f = lora.mlp_forward(*args)
-    b = lora.mlp_backward(*args, sub["dy"], f)
-    yb, dxb = chain_bounds(sub, f, b, Wg, Wu, Wd, s)
-    assert_chain_close(np64(y[rows]), f["y"], yb, "y rows")
-    assert_chain_close(np64(mlp.dX[rows]), b["dX"], dxb, "dX rows")
-    # s <V, U> appears in both <dA, A> and <dB, B> for each linear (U from the
-    # linear's input, V from its output gradient as the device materialized them)
-    for dA, A, dB, B, xin, dout in ((mlp.dAg, c["Ag"], mlp.dBg, c["Bg"], mlp_x(c), mlp.dg),
-                                    (mlp.dAu, c["Au"], mlp.dBu, c["Bu"], mlp_x(c), mlp.du),
-                                    (mlp.dAd, c["Ad"], mlp.dBd, c["Bd"], mlp.h, dy_of(c))):
-        U = np64(xin) @ np64(A).T
-        V = np64(dout) @ np64(B)
-        a, b = (np64(dA), np64(A)), (np64(dB), np64(B))
-        lhs, rhs = float((a[0] * a[1]).sum()), float((b[0] * b[1]).sum())
-        assert abs(lhs - rhs) <= adjoint_bound(s, U, V, a, b), (lhs, rhs)
+    fr = _rows_of(f, rows, ("y", "g", "u", "h", "Ug", "Uu", "Ud"))
+    br = _rows_of(b, rows, ("dX", "dh", "dg", "du"))
+    yb, dxb = chain_bounds(sub, fr, br, Wg, Wu, Wd, s)
+    assert_chain_close(np64(y[rows]), fr["y"], yb, "y rows")
+    assert_chain_close(np64(mlp.dX[rows]), br["dX"], dxb, "dX rows")

@@ -193,3 +193,50 @@ def test_merge_zero_adapter_requantizes_to_the_original_codes():
     assert finite
     assert np.array_equal(nf4.unpack(packed2, N * K), nf4.unpack(packed, N * K))
     assert np.array_equal(c2, F.bf16(c))
+
+
+def _bf16_rne(x: float) -> float:
+    """Round a Python float to the nearest bf16 value (8 significant bits), ties
+    to even: the textbook rule, written out independently of the oracle."""
+    import math
+    if x == 0.0:
+        return x
+    m, e = math.frexp(x)            # x = m 2^e, 0.5 <= |m| < 1
+    return round(m * 256.0) * 2.0 ** (e - 8)   # Python's round() is ties-to-even
+
+
+def test_mlp_materialization_points_hand_case():
+    """One token, one feature, one hidden unit, zero adapters: every bf16
+    materialization point of the gated MLP (g, u, h, dh, dg, du) is checked
+    against values worked out by hand from the definition, with weights chosen
+    so that leaving out any one rounding (or rounding in a different place)
+    changes the value checked."""
+    import math
+    s = 2.0
+    one = np.ones((1, 1))
+    zA, zB = np.full((1, 1), 0.5), np.zeros((1, 1))
+    wg, wu, wd = 1 + 2.0 ** -9, 3 + 2.0 ** -8, 1 + 3 * 2.0 ** -9
+    X, dy = one, one
+    args = (X, wg * one, zA, zB, wu * one, zA, zB, wd * one, zA, zB, s)
+    f = lora.mlp_forward(*args)
+    b = lora.mlp_backward(*args, dy, f)
+    sig = lambda t: 1.0 / (1.0 + math.exp(-t))
+    g = _bf16_rne(wg)                       # 1 + 2^-9 rounds to 1
+    u = _bf16_rne(wu)                       # 3 + 2^-8 rounds to 3
+    h = _bf16_rne(g * sig(g) * u)
+    dh = _bf16_rne(wd)                      # dy = 1
+    dg = _bf16_rne(dh * u * sig(g) * (1 + g * (1 - sig(g))))
+    du = _bf16_rne(dh * g * sig(g))
+    assert (g, u, h) == (1.0, 3.0, 2.1875)
+    assert (dh, du) == (1.0078125, 0.73828125)
+    for name, got, want in (("g", f["g"], g), ("u", f["u"], u), ("h", f["h"], h), ("y", f["y"], h * wd),
+                            ("dh", b["dh"], dh), ("dg", b["dg"], dg), ("du", b["du"], du),
+                            ("dX", b["dX"], dg * wg + du * wu)):
+        assert float(np.asarray(got).ravel()[0]) == want, name
+    # each rounding matters in this case: without it the checked value moves
+    unrounded = {"g": wg, "u": wu, "h": g * sig(g) * u, "dh": wd,
+                 "dg": dh * u * sig(g) * (1 + g * (1 - sig(g))), "du": dh * g * sig(g)}
+    for name, v in unrounded.items():
+        assert v != {"g": g, "u": u, "h": h, "dh": dh, "dg": dg, "du": du}[name], name
+    assert _bf16_rne(wg * sig(wg) * u) != h          # silu of the unrounded g
+    assert _bf16_rne(wd * u * sig(g) * (1 + g * (1 - sig(g)))) != dg   # the unrounded dh
