@@ -15,6 +15,8 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import formats as F
+from oracle import nf4
 from synthetic import inputs as S
 
 pytestmark = pytest.mark.gpu
@@ -51,6 +53,39 @@ def test_noalloc_matches_workspace_entry_two_calls(nb):
         assert np.array_equal(a1, a2), (nb, call)
         assert np.array_equal(s1, s2), (nb, call)
         assert np.array_equal(m1, m2), (nb, call)
+    assert q.qlora_get_status() == q.QL_OK
+
+
+@pytest.mark.parametrize("nb", [2049, 300_000])
+def test_noalloc_matches_oracle(nb):
+    """The no-allocation entry point against the oracle's double quantization
+    directly (mean, E4M3 codes, second-level scales), bit for bit."""
+    import bit_nf4_quantized_10_b200._lib as q
+    W = S.normal((nb * 64,), 0.02, 31 + nb, device="cuda")
+    codes = torch.empty(nb * 32, dtype=torch.uint8, device="cuda")
+    absmax = torch.empty(nb, dtype=torch.float32, device="cuda")
+    q.nf4_quantize(W, codes, absmax)
+    ng = -(-nb // 256)
+    aq = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    s2 = torch.empty(ng, dtype=torch.float32, device="cuda")
+    mu = torch.empty(1, dtype=torch.float32, device="cuda")
+    q.nf4_double_quant_noalloc(absmax, aq, s2, mu)
+    torch.cuda.synchronize()
+    e, s2_ref, mu_ref = nf4.double_quant(absmax.cpu().double().numpy())
+    assert np.array_equal(aq.cpu().numpy(), e)
+    assert np.array_equal(s2.cpu().view(torch.int32).numpy().view(np.uint32), F.f32_bits(s2_ref))
+    assert mu.cpu().view(torch.int32).numpy().view(np.uint32)[0] == F.f32_bits(np.array([mu_ref]))[0]
+    assert q.qlora_get_status() == q.QL_OK
+
+
+def test_noalloc_at_the_maximum_size():
+    """nb = QL_NOALLOC_MAX_BLOCKS (64 Mi constants, a 4 Gi-element weight): the
+    fixed scratch holds the deepest tree; equal to the workspace entry point."""
+    import bit_nf4_quantized_10_b200._lib as q
+    nb = 1 << 26
+    absmax = S.normal((nb,), 0.02, 77, device="cuda").abs_()
+    (a1, s1, m1), (a2, s2, m2) = _run_both(q, absmax)
+    assert np.array_equal(a1, a2) and np.array_equal(s1, s2) and np.array_equal(m1, m2)
     assert q.qlora_get_status() == q.QL_OK
 
 
