@@ -18,11 +18,14 @@ LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
 
 QL_OK, QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_WORKSPACE, QL_ERR_CUDA, QL_ERR_NONFINITE, QL_ERR_TIMEOUT = range(7)
 QL_F32, QL_BF16 = 0, 1
-QL_OP_DOUBLE_QUANT, QL_OP_FWD, QL_OP_BWD = 0, 1, 2
+QL_OP_DOUBLE_QUANT, QL_OP_FWD, QL_OP_BWD, QL_OP_NVFP4 = 0, 1, 2, 3
+QL_PAGE_DEVICE, QL_PAGE_HOST = 0, 1
 
 EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_double_quant_noalloc", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
            "qlora_silu_gate_fwd", "qlora_silu_gate_bwd", "qlora_workspace_size", "nf4_storage_bytes",
-           "nf4_codebook", "qlora_get_status", "qlora_status_string", "qlora_selftest_wait_timeout")
+           "nf4_codebook", "qlora_get_status", "qlora_status_string", "qlora_selftest_wait_timeout",
+           "qlora_merge", "nf4_double_quant_level1", "nf4_double_quant_finish", "nvfp4_quantize", "mxfp4_quantize",
+           "nvfp4_dequant", "mxfp4_dequant", "qlora_adamw_step", "qlora_paged_prefetch")
 
 
 class QLoraError(RuntimeError):
@@ -59,6 +62,14 @@ def _load() -> ctypes.CDLL:
         "qlora_status_string": (ctypes.c_char_p, [i32]),
         "qlora_selftest_wait_timeout": (i32, [i64, vp]),
         "qlora_merge": (i32, [W, vp, vp, i32, f32, vp, vp, vp, vp]),
+        "nf4_double_quant_level1": (i32, [vp, i64, vp, vp]),
+        "nf4_double_quant_finish": (i32, [vp, i64, i64, vp, i64, vp, vp, vp, vp, sz, vp]),
+        "nvfp4_quantize": (i32, [vp, i32, i64, i32, vp, vp, vp, vp, sz, vp]),
+        "mxfp4_quantize": (i32, [vp, i32, i64, vp, vp, vp]),
+        "nvfp4_dequant": (i32, [vp, vp, vp, i64, vp, vp]),
+        "mxfp4_dequant": (i32, [vp, vp, i64, vp, vp]),
+        "qlora_adamw_step": (i32, [vp, vp, vp, vp, vp, i64, i64, f32, f32, f32, f32, f32, vp]),
+        "qlora_paged_prefetch": (i32, [vp, sz, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -146,6 +157,52 @@ def nf4_double_quant_noalloc(absmax: torch.Tensor, absmax_q: torch.Tensor, scale
     device memory; the library uses a fixed internal scratch array instead."""
     _check(LIB.nf4_double_quant_noalloc(_ptr(absmax), absmax.numel(), _ptr(absmax_q), _ptr(scale2), _ptr(offset),
                                         _stream(stream)), "nf4_double_quant_noalloc")
+
+
+def nf4_double_quant_level1(absmax: torch.Tensor, nodes: torch.Tensor, stream=None) -> None:
+    _check(LIB.nf4_double_quant_level1(_ptr(absmax), absmax.numel(), _ptr(nodes), _stream(stream)),
+           "nf4_double_quant_level1")
+
+
+def nf4_double_quant_finish(nodes: torch.Tensor, nb_total: int, absmax: torch.Tensor, absmax_q: torch.Tensor,
+                            scale2: torch.Tensor, offset: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    _check(LIB.nf4_double_quant_finish(_ptr(nodes), nodes.numel(), int(nb_total), _ptr(absmax), absmax.numel(),
+                                       _ptr(absmax_q), _ptr(scale2), _ptr(offset), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)), "nf4_double_quant_finish")
+
+
+def nvfp4_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, tensor_scale: torch.Tensor,
+                   ws: torch.Tensor, use_tensor_scale: bool = True, stream=None) -> None:
+    _check(LIB.nvfp4_quantize(_ptr(x), _dt(x.dtype), x.numel(), 1 if use_tensor_scale else 0, _ptr(codes),
+                              _ptr(scales), _ptr(tensor_scale), _ptr(ws), ws.numel() * ws.element_size(),
+                              _stream(stream)), "nvfp4_quantize")
+
+
+def mxfp4_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None) -> None:
+    _check(LIB.mxfp4_quantize(_ptr(x), _dt(x.dtype), x.numel(), _ptr(codes), _ptr(scales), _stream(stream)),
+           "mxfp4_quantize")
+
+
+def nvfp4_dequant(codes: torch.Tensor, scales: torch.Tensor, tensor_scale: torch.Tensor, n: int, out: torch.Tensor,
+                  stream=None) -> None:
+    _check(LIB.nvfp4_dequant(_ptr(codes), _ptr(scales), _ptr(tensor_scale), int(n), _ptr(out), _stream(stream)),
+           "nvfp4_dequant")
+
+
+def mxfp4_dequant(codes: torch.Tensor, scales: torch.Tensor, n: int, out: torch.Tensor, stream=None) -> None:
+    _check(LIB.mxfp4_dequant(_ptr(codes), _ptr(scales), int(n), _ptr(out), _stream(stream)), "mxfp4_dequant")
+
+
+def qlora_adamw_step(p, g, m, v, n: int, t: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+                     eps: float = 1e-8, weight_decay: float = 0.0, p_bf16=None, stream=None) -> None:
+    """p, g, m, v: fp32 tensors or raw device / managed-memory addresses (ints)."""
+    _check(LIB.qlora_adamw_step(_ptr(p), _ptr(g), _ptr(m), _ptr(v), _ptr(p_bf16), int(n), int(t), float(lr),
+                                float(beta1), float(beta2), float(eps), float(weight_decay), _stream(stream)),
+           "qlora_adamw_step")
+
+
+def qlora_paged_prefetch(ptr, nbytes: int, where: int, stream=None) -> None:
+    _check(LIB.qlora_paged_prefetch(_ptr(ptr), int(nbytes), int(where), _stream(stream)), "qlora_paged_prefetch")
 
 
 def nf4_dequant(w: "NF4Weight", out: torch.Tensor, stream=None) -> None:

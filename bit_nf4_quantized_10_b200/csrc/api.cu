@@ -15,6 +15,9 @@ ql_status launch_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q
                               void* ws, cudaStream_t st);
 ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStream_t st);
 unsigned status_word_codec(cudaStream_t st);
+ql_status launch_dq_level1(const float* absmax, int64_t nb, double* nodes, cudaStream_t st);
+ql_status launch_dq_finish(const double* nodes, int64_t n_nodes, int64_t nb_total, const float* absmax, int64_t nb,
+                           uint8_t* absmax_q, float* scale2, float* offset, void* ws, cudaStream_t st);
 ql_status launch_merge(const ql_nf4_weight* w, const void* A, const void* B, int r, float s, void* out,
                        uint8_t* codes_out, float* absmax_out, cudaStream_t st);
 // gemm.cu
@@ -37,8 +40,21 @@ ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t
 ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st);
 // smallm.cu
 bool smallm_supported(int64_t N, int64_t K);
-ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
-                            float s, void* Y, ql_dtype y_dt, cudaStream_t st);
+size_t smallm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* A, const void* B, int r,
+                            float s, void* Y, ql_dtype y_dt, void* U_out, void* ws, cudaStream_t st);
+// fp4.cu
+ql_status launch_nvfp4_quantize(const void* x, ql_dtype dt, int64_t n, int use_ts, uint8_t* codes, uint8_t* scales,
+                                float* ts, void* ws, cudaStream_t st);
+ql_status launch_mxfp4_quantize(const void* x, ql_dtype dt, int64_t n, uint8_t* codes, uint8_t* scales,
+                                cudaStream_t st);
+ql_status launch_fp4_dequant(const uint8_t* codes, const uint8_t* scales, const float* ts, int64_t n, int fmt,
+                             float* out, cudaStream_t st);
+unsigned status_word_fp4(cudaStream_t st);
+// adamw.cu
+ql_status launch_adamw(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int64_t t, float lr,
+                       float b1, float b2, float eps, float wd, cudaStream_t st);
+ql_status paged_prefetch(const void* ptr, size_t bytes, int where, cudaStream_t st);
 // mlp.cu
 ql_status launch_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, cudaStream_t st);
 ql_status launch_silu_gate_bwd(const void* dh, const void* g, const void* u, void* dg, void* du, int64_t n,
@@ -75,16 +91,15 @@ ql_status check_gemm_shape(const ql_nf4_weight* w, int64_t M, int r) {
   return QL_OK;
 }
 
-// Tokens up to this count take the small-M (HBM-bound) forward kernel, for
-// K up to 40960 (its K slice of X must fit in shared memory).
+// Tokens up to this count take the small-token (HBM-bound) forward kernels.
 constexpr int64_t kSmallM = 16;
 
-bool use_smallm(int64_t M, int64_t N, int64_t K) { return M <= kSmallM && ql::smallm_supported(N, K); }
+bool use_smallm(int64_t M, int64_t N, int64_t K) { return M >= 1 && M <= kSmallM && ql::smallm_supported(N, K); }
 
-// Forward workspace: U [M, r] (when U_out is not given).
+// Forward workspace: U [M, r] (when U_out is not given); for the small-token
+// path also the fp32 part sums of Y and U (smallm.cu).
 size_t ws_fwd(int64_t M, int64_t N, int64_t K, int r) {
-  (void)N;
-  (void)K;
+  if (use_smallm(M, N, K)) return ql::smallm_workspace_bytes(M, N, K, r);
   return align256((size_t)M * r * 2);
 }
 
@@ -140,6 +155,24 @@ ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q, f
   return ql::launch_double_quant(absmax, nb, absmax_q, scale2, offset, ws, as_stream(stream));
 }
 
+ql_status nf4_double_quant_level1(const float* absmax, int64_t nb, double* nodes, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/nf4_double_quant_level1");
+  if (nb <= 0 || !aligned16(absmax) || !aligned16(nodes)) return QL_ERR_INVALID_ARG;
+  return ql::launch_dq_level1(absmax, nb, nodes, as_stream(stream));
+}
+
+ql_status nf4_double_quant_finish(const double* nodes, int64_t n_nodes, int64_t nb_total, const float* absmax,
+                                  int64_t nb, uint8_t* absmax_q, float* scale2, float* offset, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/nf4_double_quant_finish");
+  if (n_nodes <= 0 || nb <= 0 || nb_total < nb || n_nodes != (nb_total + 2047) / 2048) return QL_ERR_INVALID_ARG;
+  if (!aligned16(nodes) || !aligned16(absmax) || !aligned16(absmax_q) || !aligned16(scale2) || !aligned16(offset) ||
+      !aligned16(ws))
+    return QL_ERR_INVALID_ARG;
+  if (ws_bytes < ql::dq_workspace_bytes(nb_total)) return QL_ERR_WORKSPACE;
+  return ql::launch_dq_finish(nodes, n_nodes, nb_total, absmax, nb, absmax_q, scale2, offset, ws, as_stream(stream));
+}
+
 ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* stream) {
   NvtxRange nvtx_range("qlora_nf4/nf4_dequant");
   ql_status st = check_weight(w);
@@ -180,12 +213,11 @@ ql_status qlora_linear_fwd(const ql_nf4_weight* w, const void* X, int64_t M, con
   if (r == 0 && !small) return ql::launch_gemm_fwd(w, X, M, nullptr, nullptr, 0, s, Y, y_dt, cs);
   if (ws_bytes < ws_fwd(M, N, K, r)) return QL_ERR_WORKSPACE;
   if (!aligned16(ws)) return QL_ERR_INVALID_ARG;
+  // small token counts: U = bf16(X A^T) comes out of the same pass over K
+  if (small) return ql::launch_smallm_fwd(w, X, M, A, B, r, s, Y, y_dt, U_out, ws, cs);
   void* U = U_out ? U_out : ws;
-  if (r > 0) {
-    st = ql::launch_proj(X, M, K, A, K, r, U, nullptr, 0, cs);    // U = bf16(X A^T)
-    if (st != QL_OK) return st;
-  }
-  if (small) return ql::launch_smallm_fwd(w, X, M, U, B, r, s, Y, y_dt, cs);
+  st = ql::launch_proj(X, M, K, A, K, r, U, nullptr, 0, cs);      // U = bf16(X A^T)
+  if (st != QL_OK) return st;
   return ql::launch_gemm_fwd(w, X, M, U, B, r, s, Y, y_dt, cs);
 }
 
@@ -237,6 +269,54 @@ ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY
   return ql::launch_grad_a(X, M, (int)K, Vt, Mp, r, s, dA, grad_dt, cs);   // dA = s V^T X
 }
 
+ql_status nvfp4_quantize(const void* x, ql_dtype x_dt, int64_t n, int use_tensor_scale, uint8_t* codes,
+                         uint8_t* scales, float* tensor_scale, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/nvfp4_quantize");
+  if (n <= 0 || !dtype_ok(x_dt)) return QL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(tensor_scale) || !aligned16(ws))
+    return QL_ERR_INVALID_ARG;
+  if (ws_bytes < qlora_workspace_size(QL_OP_NVFP4, n, 0, 0, 0)) return QL_ERR_WORKSPACE;
+  return ql::launch_nvfp4_quantize(x, x_dt, n, use_tensor_scale ? 1 : 0, codes, scales, tensor_scale, ws,
+                                   as_stream(stream));
+}
+
+ql_status mxfp4_quantize(const void* x, ql_dtype x_dt, int64_t n, uint8_t* codes, uint8_t* scales, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/mxfp4_quantize");
+  if (n <= 0 || !dtype_ok(x_dt)) return QL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return QL_ERR_INVALID_ARG;
+  return ql::launch_mxfp4_quantize(x, x_dt, n, codes, scales, as_stream(stream));
+}
+
+ql_status nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale, int64_t n,
+                        float* out, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/nvfp4_dequant");
+  if (n <= 0 || !aligned16(codes) || !aligned16(scales) || !aligned16(tensor_scale) || !aligned16(out))
+    return QL_ERR_INVALID_ARG;
+  return ql::launch_fp4_dequant(codes, scales, tensor_scale, n, 0, out, as_stream(stream));
+}
+
+ql_status mxfp4_dequant(const uint8_t* codes, const uint8_t* scales, int64_t n, float* out, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/mxfp4_dequant");
+  if (n <= 0 || !aligned16(codes) || !aligned16(scales) || !aligned16(out)) return QL_ERR_INVALID_ARG;
+  return ql::launch_fp4_dequant(codes, scales, nullptr, n, 1, out, as_stream(stream));
+}
+
+ql_status qlora_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int64_t t, float lr,
+                           float beta1, float beta2, float eps, float weight_decay, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/qlora_adamw_step");
+  if (n <= 0 || t < 1) return QL_ERR_INVALID_ARG;
+  if (!aligned16(p) || !aligned16(g) || !aligned16(m) || !aligned16(v) || (p_bf16 && !aligned16(p_bf16)))
+    return QL_ERR_INVALID_ARG;
+  if (!(beta1 >= 0.0f && beta1 < 1.0f) || !(beta2 >= 0.0f && beta2 < 1.0f) || !(eps >= 0.0f)) return QL_ERR_INVALID_ARG;
+  return ql::launch_adamw(p, g, m, v, p_bf16, n, t, lr, beta1, beta2, eps, weight_decay, as_stream(stream));
+}
+
+ql_status qlora_paged_prefetch(const void* ptr, size_t bytes, int where, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/qlora_paged_prefetch");
+  if (!ptr || bytes == 0 || (where != QL_PAGE_DEVICE && where != QL_PAGE_HOST)) return QL_ERR_INVALID_ARG;
+  return ql::paged_prefetch(ptr, bytes, where, as_stream(stream));
+}
+
 ql_status qlora_selftest_wait_timeout(int64_t polls, void* stream) {
   if (polls < 1 || polls > (1 << 20)) return QL_ERR_INVALID_ARG;
   return ql::launch_wait_timeout((uint32_t)polls, as_stream(stream));
@@ -261,6 +341,7 @@ size_t qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r) {
     case QL_OP_DOUBLE_QUANT: return M > 0 ? ql::dq_workspace_bytes(M) : 0;
     case QL_OP_FWD: return ws_fwd(M, N, K, r);
     case QL_OP_BWD: return ws_bwd(M, N, K, r);
+    case QL_OP_NVFP4: return M > 0 ? 256 : 0;
     default: return 0;
   }
 }
@@ -282,7 +363,7 @@ ql_status qlora_get_status(void* stream) {
   // one status word per translation unit that raises status bits
   unsigned v = 0;
   for (unsigned (*word)(cudaStream_t) : {ql::status_word_codec, ql::status_word_gemm, ql::status_word_lora,
-                                         ql::status_word_smallm, ql::status_word_diag}) {
+                                         ql::status_word_smallm, ql::status_word_diag, ql::status_word_fp4}) {
     const unsigned w = word(cs);
     if (w == ~0u) return QL_ERR_CUDA;
     v |= w;

@@ -489,6 +489,44 @@ ql_status launch_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q
   return QL_OK;
 }
 
+// Quantization sharded by rows: the level-1 nodes of the mean's tree (one
+// float64 sum per 2048 constants) of this slab ...
+ql_status launch_dq_level1(const float* absmax, int64_t nb, double* nodes, cudaStream_t st) {
+  const int64_t cnt = (nb + 2047) / 2048;
+  TraceScope ts(TK_DQ_MEAN, st);
+  QL_CUDA_TRY(launch(tree_sum_pass<float>, dim3((unsigned)cnt), dim3(256), 0, st, 1, 1, absmax, nb, nodes, nb,
+                     (float*)nullptr));
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
+// ... and, from every slab's nodes in order, the mean (the remaining levels of
+// the same tree) and this slab's E4M3 codes and group scales.
+ql_status launch_dq_finish(const double* nodes, int64_t n_nodes, int64_t nb_total, const float* absmax, int64_t nb,
+                           uint8_t* absmax_q, float* scale2, float* offset, void* ws, cudaStream_t st) {
+  double* dst = reinterpret_cast<double*>(ws);
+  const double* prev = nodes;
+  int64_t cnt = n_nodes;
+  {
+    TraceScope ts(TK_DQ_MEAN, st);
+    do {
+      const int64_t next = (cnt + 2047) / 2048;
+      QL_CUDA_TRY(launch(tree_sum_pass<double>, dim3((unsigned)next), dim3(256), 0, st, 1, 1, prev, cnt, dst, nb_total,
+                         next == 1 ? offset : nullptr));
+      QL_LAUNCH_CHECK();
+      prev = dst;
+      dst += next;
+      cnt = next;
+    } while (cnt > 1);
+  }
+  const int64_t ng = (nb + 255) / 256;
+  TraceScope ts(TK_DQ_ENCODE, st);
+  QL_CUDA_TRY(launch(dq_encode_kernel, dim3(grid_for(ng, 8, 8)), dim3(256), 0, st, 1, 1, absmax, nb, offset, absmax_q,
+                     scale2));
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
 ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStream_t st) {
   const int64_t n = w->rows * w->cols;
   WeightConsts wc{w->absmax, w->absmax_q, w->scale2, w->offset};

@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int gt = ((wp % GROUP_WARPS) << 5) | lane;   // thread within the group, 0..127
     const int kblocks = p.K / 64;            // 64-blocks per weight row
     const float mu = p.wc.absmax ? 0.0f : *p.wc.offset;
-    const uint32_t qbase = smem_u32(qlev);   // low byte 0
+    const uint32_t qbase = opaque_after_barrier(smem_u32(qlev));   // low byte 0
     int row_in_tile, col_chunk;
     if (!BWD) { row_in_tile = gt; col_chunk = 0; }
     else { row_in_tile = gt & 63; col_chunk = gt >> 6; }
@@ -357,8 +357,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t o[4];
 #pragma unroll
           for (int bb = 0; bb < 4; ++bb) {
-            const float fe = lds_f32(__byte_perm(e4, qbase, 0x7650u | bb));
-            const float fo = lds_f32(__byte_perm(o4, qbase, 0x7650u | bb));
+            const float fe = lds_f32_const(__byte_perm(e4, qbase, 0x7650u | bb));
+            const float fo = lds_f32_const(__byte_perm(o4, qbase, 0x7650u | bb));
             float pe, po;
             mul2_rn(fe, fo, c, pe, po);
             o[bb] = pack_bf16x2(pe, po);

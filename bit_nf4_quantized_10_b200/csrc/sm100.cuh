@@ -294,5 +294,21 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return v;
 }
 
+// The same load as a pure function of its address, which the compiler may
+// schedule freely (also across volatile asm such as mma.sync), for reads of a
+// table that is written once before a barrier and never again.  The address
+// must come from opaque_after_barrier() so that no read moves above the
+// barrier that publishes the table.
+__device__ __forceinline__ float lds_f32_const(uint32_t addr) {
+  float v;
+  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t opaque_after_barrier(uint32_t x) {
+  uint32_t y;
+  asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x) : "memory");
+  return y;
+}
+
 }  // namespace sm100
 }  // namespace ql

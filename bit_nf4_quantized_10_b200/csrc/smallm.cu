@@ -1,33 +1,36 @@
-// Small-token forward: Y = X * W_hat^T + s * U * B^T for M <= 16 tokens.
+// Small-token forward: Y = X * W_hat^T + s * U * B^T, U = bf16(X * A^T), for
+// M <= 16 tokens.
 //
 // With a handful of tokens each dequantized weight element meets at most 16
 // activations, so the layer is bound by reading the packed 4-bit weight from
 // HBM ("QLoRA — Fine-Tuning a 65B Model on One GPU", "Pitfalls":
 // memory-bandwidth-bound generation has less to read with 4-bit weights) and
-// by the integer work of expanding it, which must keep pace with HBM.
-//   * Operands are swapped: the expanded weight tile is the MMA's A operand
-//     (M = 128 weight rows) and lives in TMEM, written with tcgen05.st from the
-//     producer registers; the tokens are the N = 16 operand (zero-padded).
-//   * Expansion: the 16 fp32 levels sit in a shared-memory table (one
-//     conflict-free LDS per element), times the block constant in fp32, pairs
-//     packed to bf16: bf16(fl32(q * c)), as everywhere else.
-//   * Persistent clusters: the CTAs of a cluster (up to 8) split K, so each
-//     CTA owns one fixed K slice and keeps the tokens' slice of X in shared
-//     memory for the whole kernel; the clusters walk over 128-row weight
-//     tiles.  Each TMA stage brings 128 contiguous bytes (256 codes) of every
-//     row of the tile.
-//   * The split-K partials meet in shared memory: each CTA drains its 128 x 16
-//     fp32 partial (TMEM, double-buffered) into shared memory, and CTA q of the
-//     cluster adds the slices of its share of the tile's outputs in slice
-//     order through distributed shared memory, adds s * U * B^T in fp32 and
-//     writes Y.  Hand-offs between the CTAs go through mbarriers with remote
-//     arrivals (release/acquire at cluster scope), so the expansion of the
-//     next tile overlaps the reduction of the last.
-#include <cudaTypedefs.h>
-
+// by the work of expanding it, which must keep pace with HBM.  On this part
+// the expansion's floor is the shared-memory read of one fp32 NF4 level per
+// element (128 bytes per clock per SM), so everything else is kept off the
+// shared-memory and issue budget:
+//   * No staging of the expanded weight: each thread expands its codes straight
+//     into the A-operand registers of warp-level tensor-core MMAs
+//     (mma.sync m16n8k16, bf16 in, fp32 accumulate), weight rows as M = 16 and
+//     tokens as N = 8 (one or two token tiles).
+//   * The reduction dimension is permuted so that each thread reads 8
+//     contiguous code bytes (16 codes) of a 64-block per row: for k-step u of
+//     block j, thread quad-index t's MMA slots {2t, 2t+1} and {2t+8, 2t+9} hold
+//     the elements at k = 64 j + 16 t + 4 u + {0, 1} and {2, 3}.  The
+//     activation fragments use the same permutation, so every k is summed once.
+//   * K is split over the 16 warps of a CTA (KV codes per row each) and over
+//     parts of K handled by different CTAs; each warp keeps the activation
+//     fragments of its K range in registers for the whole kernel and walks the
+//     CTA's row blocks, loading the next row block's codes into registers while
+//     it expands the current one.  The 16 warps' partial sums meet in shared
+//     memory in warp order; each part's sums go to the workspace.
+//   * The CTA that owns the last row block of each part also computes that
+//     part's share of U = X A^T with the same fragments (A rows as M).
+//   * A second kernel sums the parts in order, rounds U to bf16, adds
+//     s * (U B^T) in fp32 and writes Y (and U).
+// Every sum has a fixed order, so results do not depend on scheduling.  There
+// are no inter-CTA waits: the kernels only use __syncthreads.
 #include <algorithm>
-#include <mutex>
-#include <vector>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -38,575 +41,400 @@ using namespace sm100;
 
 QL_DEFINE_STATUS_ACCESSOR(status_word_smallm)
 
-bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
-                 uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
-
 namespace smallm {
 
-constexpr int TM = 128;           // weight rows per tile (MMA M)
-constexpr int TN = 16;            // token slots (MMA N)
-constexpr int BK = 64;            // reduction elements per MMA sub-step (one 64-block per row)
-constexpr int SUB = 4;            // sub-steps per code stage: 256 codes = 128 contiguous bytes per row
-constexpr int C_STAGE_BYTES = TM * BK * SUB / 2;   // 16 KB packed codes
-constexpr int MAX_C_STAGES = 8;
-constexpr int X_SUB_BYTES = TN * BK * 2;           // 2 KB activation sub-tile
-constexpr int MAX_PER = 80;       // sub-steps per K slice (bounded by shared memory)
-constexpr int MAX_CS = 8;         // CTAs per cluster (portable cluster size)
-constexpr int A_STAGES = 3;       // TMEM ring of expanded A stages (128 rows x 256 codes each)
-constexpr int GROUP_WARPS = 8;    // producer warps per group; two groups take alternate sub-steps
-constexpr int PRODUCER_WARPS = 2 * GROUP_WARPS;
-constexpr int DRAIN_WARP0 = 2 + PRODUCER_WARPS;
-constexpr int DRAIN_WARPS = 4;
-constexpr int THREADS = (DRAIN_WARP0 + DRAIN_WARPS) * 32;
-constexpr int TMEM_COLS = 512;    // D[b] at columns 16 b; A stage s at 128 + 128 s (32 per sub-step)
-constexpr int A_COL0 = 128;
-constexpr int A_STAGE_COLS = 128;
-constexpr int RED_LD = 18;        // floats per row of a reduction buffer (conflict-free float2 reads)
-constexpr int RED_BYTES = TM * RED_LD * 4;
+constexpr int WARPS = 16;
+constexpr int THREADS = WARPS * 32;
+constexpr int MAX_M = 16;
 constexpr int MAX_R = 64;
 
 struct Params {
   int M, N, K, r;
-  int kb_total;       // K / 64
-  int per;            // sub-steps per K slice (the last slice may be shorter)
-  int tiles;          // ceil(N / 128)
-  int c_stages;       // code ring depth (a power of two)
-  int c_log;          // log2(c_stages)
-  float s;
+  int kb;            // K / 64 (blocks per weight row)
+  int parts;         // CTAs' K parts
+  int part_k;        // reduction elements per part (WARPS * KV)
+  int row_blocks;    // ceil(N / (16 T))
   WeightConsts wc;
   NF4Table tab;
-  const __nv_bfloat16* U;   // [M, r]
-  const __nv_bfloat16* B;   // [N, r]
-  void* Y;
-  int y_bf16;
-  uint32_t wait_limit;
+  const uint8_t* codes;
+  const __nv_bfloat16* X;    // [M, K]
+  const __nv_bfloat16* A;    // [r, K]
+  float* part_y;             // [parts][N][M] fp32
+  float* part_u;             // [parts][M][r] fp32
 };
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Arrive on the barrier at this offset in CTA `rank`, release at cluster
-// scope: publishes this thread's (and, through a preceding warp barrier, its
-// warp's) shared-memory accesses to the other CTA.
-__device__ __forceinline__ void arrive_remote_release(uint64_t* bar, uint32_t rank) {
-  asm volatile(
-      "{\n .reg .b32 ra;\n"
-      " mapa.shared::cluster.u32 ra, %0, %1;\n"
-      " mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n}" ::"r"(smem_u32(bar)),
-      "r"(rank)
-      : "memory");
+// Two codes (the low and high nibble of byte b of `w`) -> bf16x2 of
+// bf16(fl32(q * c)), the low code in the low half.  e4 / o4 hold 4 * low / high
+// nibble of each byte; the level table's low address byte is replaced by it.
+__device__ __forceinline__ uint32_t expand_pair(uint32_t e4, uint32_t o4, uint32_t qbase, uint32_t sel, float c) {
+  const float lo = lds_f32_const(__byte_perm(e4, qbase, sel));
+  const float hi = lds_f32_const(__byte_perm(o4, qbase, sel));
+  float pl, ph;
+  mul2_rn(lo, hi, c, pl, ph);
+  return pack_bf16x2(pl, ph);
 }
 
-__device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
-  return v;
+// One row's 16 codes of each of this warp's blocks (8 bytes each) for this
+// thread.  Rows past N read nothing and expand to zero (constant 0).
+template <int KV>
+__device__ __forceinline__ void load_codes(const Params& p, int row, int kb0, int nbw, int tq, uint2 (&w)[KV / 64]) {
+#pragma unroll
+  for (int j = 0; j < KV / 64; ++j) {
+    w[j] = make_uint2(0u, 0u);
+    if (row < p.N && j < nbw)
+      w[j] = __ldcs(reinterpret_cast<const uint2*>(p.codes + (size_t)row * (p.K / 2) + (size_t)(kb0 + j) * 32 + tq * 8));
+  }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    smallm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
-                  const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ float us[TN * MAX_R];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int cs = (int)gridDim.x;                 // CTAs per cluster = K slices
-  const int q = (int)blockIdx.x;                 // this CTA's slice (its cluster rank)
-  const int kb0 = q * p.per;
-  const int per_q = min(p.per, p.kb_total - kb0);
-  const int nst = (per_q + SUB - 1) / SUB;       // code stages per tile
-  const int nt = (p.tiles - (int)blockIdx.y + (int)gridDim.y - 1) / (int)gridDim.y;   // tiles of this cluster
-  const int C = p.c_stages;
-  uint8_t* xs = base;                                            // per_q x 2 KB
-  uint8_t* cring = xs + p.per * X_SUB_BYTES;                     // C x 16 KB
-  float* red = reinterpret_cast<float*>(cring + C * C_STAGE_BYTES);   // 2 x 128 x RED_LD
-  // the 16 fp32 levels, 256-byte aligned: an LDS address is the table base
-  // with the level's byte offset (4 * code) in its low byte
-  float* qtab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(red) + 2 * RED_BYTES);
-  uint64_t* full_x = reinterpret_cast<uint64_t*>(qtab + 64);
-  uint64_t* full_c = full_x + 1;
-  uint64_t* empty_c = full_c + MAX_C_STAGES;
-  uint64_t* a_full = empty_c + MAX_C_STAGES;
-  uint64_t* a_empty = a_full + A_STAGES;
-  uint64_t* acc_full = a_empty + A_STAGES;
-  uint64_t* tmem_free = acc_full + 2;
-  uint64_t* ready = tmem_free + 2;
-  uint64_t* freed = ready + 2;
-  uint32_t* tmem_addr = reinterpret_cast<uint32_t*>(freed + 2);
-  volatile int* abort_flag = reinterpret_cast<int*>(tmem_addr + 1);
+// Raw block constants of one row's blocks: the E4M3 byte (or the fp32 bits of
+// a plain constant) per block, and the group scales s_2 of the first and the
+// last block (blocks of a row chunk span at most two groups of 256).  Only
+// loads here: the decode waits until the row block is expanded, so the loads
+// of the next row block stay in flight while this one computes.
+template <int KV>
+__device__ __forceinline__ void load_consts(const Params& p, int row, int kb0, int nbw, uint32_t (&q)[KV / 64],
+                                            float (&s2)[2]) {
+  s2[0] = s2[1] = 0.0f;
+#pragma unroll
+  for (int j = 0; j < KV / 64; ++j) {
+    q[j] = 0u;
+    if (row < p.N && j < nbw) {
+      const int64_t b = (int64_t)row * p.kb + kb0 + j;
+      q[j] = p.wc.absmax ? __float_as_uint(__ldg(p.wc.absmax + b)) : (uint32_t)__ldg(p.wc.absmax_q + b);
+    }
+  }
+  if (!p.wc.absmax && row < p.N && nbw > 0) {
+    const int64_t b0 = (int64_t)row * p.kb + kb0;
+    s2[0] = __ldg(p.wc.scale2 + (b0 >> 8));
+    s2[1] = __ldg(p.wc.scale2 + ((b0 + nbw - 1) >> 8));
+  }
+}
+
+// The reconstructed constant of block j of a row chunk starting at block b0:
+// c_hat = fl32(fl32(E4M3(q) s_2) + mu) (double quant) or the plain fp32 value.
+__device__ __forceinline__ float decode_const(const WeightConsts& wc, uint32_t q, const float (&s2)[2], int64_t b0,
+                                              int j, float mu) {
+  if (wc.absmax) return __uint_as_float(q);
+  const float s = ((b0 + j) >> 8) == (b0 >> 8) ? s2[0] : s2[1];
+  return __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)q), s), mu);
+}
+
+// Per row block of 16 T rows: the codes and raw constants a thread expands.
+template <int NT, int KV, int T>
+struct Frag {
+  uint2 w[T][2][KV / 64];     // [tile][row g / g+8][block]
+  uint32_t q[T][2][KV / 64];
+  float s2[T][2][2];
+};
+
+template <int NT, int KV, int T>
+__device__ __forceinline__ void load_frag(const Params& p, int rb, int kb0, int nbw, int g, int tq,
+                                          Frag<NT, KV, T>& f) {
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = rb * 16 * T + 16 * t + g + 8 * h;
+      load_codes<KV>(p, row, kb0, nbw, tq, f.w[t][h]);
+      load_consts<KV>(p, row, kb0, nbw, f.q[t][h], f.s2[t][h]);
+    }
+  }
+}
+
+template <int NT, int KV, int T>
+__device__ __forceinline__ void compute_frag(const Params& p, const Frag<NT, KV, T>& f, int rb, int kb0, float mu,
+                                             const uint32_t (&xb)[KV / 16][NT][2], uint32_t qbase, int nbw,
+                                             int g, float (&acc)[T][NT][4]) {
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[t][n][i] = 0.0f;
+#pragma unroll
+  for (int j = 0; j < KV / 64; ++j) {
+    if (j < nbw) {
+#pragma unroll
+      for (int t = 0; t < T; ++t) {
+        const int row = rb * 16 * T + 16 * t + g;
+        const float cg = decode_const(p.wc, f.q[t][0][j], f.s2[t][0], (int64_t)row * p.kb + kb0, j, mu);
+        const float c8 = decode_const(p.wc, f.q[t][1][j], f.s2[t][1], (int64_t)(row + 8) * p.kb + kb0, j, mu);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {        // word .x: k-steps 0, 1; word .y: k-steps 2, 3
+          const uint32_t wg = half ? f.w[t][0][j].y : f.w[t][0][j].x;
+          const uint32_t w8 = half ? f.w[t][1][j].y : f.w[t][1][j].x;
+          const uint32_t eg = (wg << 2) & 0x3C3C3C3Cu, og = (wg >> 2) & 0x3C3C3C3Cu;
+          const uint32_t e8 = (w8 << 2) & 0x3C3C3C3Cu, o8 = (w8 >> 2) & 0x3C3C3C3Cu;
+#pragma unroll
+          for (int s = 0; s < 2; ++s) {               // k-step u = 2 half + s: bytes 2s (slots 2t..) and 2s+1 (slots 2t+8..)
+            const uint32_t a0 = expand_pair(eg, og, qbase, 0x7650u | (2 * s), cg);
+            const uint32_t a1 = expand_pair(e8, o8, qbase, 0x7650u | (2 * s), c8);
+            const uint32_t a2 = expand_pair(eg, og, qbase, 0x7650u | (2 * s + 1), cg);
+            const uint32_t a3 = expand_pair(e8, o8, qbase, 0x7650u | (2 * s + 1), c8);
+            const int ks = 4 * j + 2 * half + s;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) mma_bf16(acc[t][n], a0, a1, a2, a3, xb[ks][n][0], xb[ks][n][1]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// Partials of a row block (16 T rows x M tokens): warp w's C fragments into
+// red, then the CTA sums the 16 warps in order and writes part_y.
+template <int NT, int T>
+__device__ __forceinline__ void stash(float* red, const float (&acc)[T][NT][4], int warp, int g, int tq) {
+  // red layout: [warp][16 T rows][8 NT tokens]
+  constexpr int TOK = 8 * NT;
+  float* base = red + warp * (16 * T * TOK);
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int tok = 8 * n + 2 * tq;
+      *reinterpret_cast<float2*>(base + (16 * t + g) * TOK + tok) = make_float2(acc[t][n][0], acc[t][n][1]);
+      *reinterpret_cast<float2*>(base + (16 * t + g + 8) * TOK + tok) = make_float2(acc[t][n][2], acc[t][n][3]);
+    }
+}
+
+// Dynamic shared memory of the main kernel: two reduction buffers.
+template <int NT, int T>
+__host__ __device__ constexpr size_t red_floats() { return (size_t)WARPS * 16 * T * 8 * NT; }
+
+template <int NT, int KV, int T>
+__global__ void __launch_bounds__(THREADS, 1) smallm_kernel(Params p) {
+  constexpr int ROWS = 16 * T;
+  constexpr int TOK = 8 * NT;
+  __shared__ __align__(256) float qlev[64];
+  extern __shared__ __align__(16) float red_dyn[];   // two reduction buffers of red_floats<NT, T>()
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  auto tile_of = [&](int ti) { return (int)blockIdx.y + ti * (int)gridDim.y; };
-
-  if (threadIdx.x < 16) qtab[threadIdx.x] = p.tab.q[threadIdx.x];
-  if (threadIdx.x == 0) {
-    mbar_init(full_x, 1);
-    for (int i = 0; i < MAX_C_STAGES; ++i) {
-      mbar_init(&full_c[i], 1);
-      mbar_init(&empty_c[i], 1);
-    }
-    for (int i = 0; i < A_STAGES; ++i) {
-      mbar_init(&a_full[i], GROUP_WARPS);
-      mbar_init(&a_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&tmem_free[i], DRAIN_WARPS);
-      mbar_init(&ready[i], cs * DRAIN_WARPS);
-      mbar_init(&freed[i], cs * DRAIN_WARPS);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_addr, TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  cluster_sync();   // every CTA's barriers are initialised before any remote arrival
-  tc_fence_after();
-  const uint32_t tmem = *tmem_addr;
+  const int g = lane >> 2, tq = lane & 3;
+  if (threadIdx.x < 16) qlev[threadIdx.x] = p.tab.q[threadIdx.x];
   pdl_wait();
   pdl_trigger();
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA warp
-    if (lane == 0) {
-      prefetch_tmap(&tmap_x);
-      prefetch_tmap(&tmap_codes);
-      mbar_arrive_expect_tx(full_x, per_q * X_SUB_BYTES);
-      for (int j = 0; j < per_q; ++j) tma_load_2d(xs + j * X_SUB_BYTES, &tmap_x, full_x, (kb0 + j) * BK, 0);
-      int issued = 0;
-      bool ok = true;
-      for (int ti = 0; ti < nt && ok; ++ti) {
-        for (int st = 0; st < nst; ++st) {
-          const int g = ti * nst + st, cslot = g % C;
-          if (g >= C && !mbar_wait(&empty_c[cslot], ((g / C) - 1) & 1, abort_flag, p.wait_limit)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full_c[cslot], C_STAGE_BYTES);
-          tma_load_2d(cring + cslot * C_STAGE_BYTES, &tmap_codes, &full_c[cslot], (kb0 + st * SUB) * (BK / 2),
-                      tile_of(ti) * TM);
-          issued = g + 1;
-        }
+  const int part = blockIdx.x;
+  // this warp's K range: blocks [kb0, kb0 + nbw) of every row
+  const int k0 = part * p.part_k + warp * KV;
+  const int kb0 = k0 / 64;
+  const int nbw = max(0, min(KV, p.K - k0)) / 64;
+  const float mu = p.wc.absmax ? 0.0f : __ldg(p.wc.offset);
+  // activation fragments of the K range, in the permuted order (0 past M or K)
+  uint32_t xb[KV / 16][NT][2];
+#pragma unroll
+  for (int j = 0; j < KV / 64; ++j)
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int tok = 8 * n + g;
+        uint2 v = make_uint2(0u, 0u);
+        if (tok < p.M && j < nbw)
+          v = __ldg(reinterpret_cast<const uint2*>(p.X + (size_t)tok * p.K + k0 + 64 * j + 16 * tq + 4 * u));
+        xb[4 * j + u][n][0] = v.x;
+        xb[4 * j + u][n][1] = v.y;
       }
-      // before leaving, make sure no copy is still landing in shared memory
-      mbar_wait(full_x, 0, abort_flag, p.wait_limit);
-      for (int g = (issued > C ? issued - C : 0); g < issued; ++g)
-        mbar_wait(&full_c[g % C], (g / C) & 1, abort_flag, p.wait_limit);
+  __syncthreads();
+  const uint32_t qbase = opaque_after_barrier(smem_u32(qlev));   // table reads stay below the barrier
+  const int rb_first = blockIdx.y, rb_step = gridDim.y;
+  Frag<NT, KV, T> f[2];
+  int it = 0;
+  if (rb_first < p.row_blocks) load_frag<NT, KV, T>(p, rb_first, kb0, nbw, g, tq, f[0]);
+  for (int rb = rb_first; rb < p.row_blocks; rb += rb_step, ++it) {
+    const int nxt = rb + rb_step;
+    float acc[T][NT][4];
+    if ((it & 1) == 0) {
+      if (nxt < p.row_blocks) load_frag<NT, KV, T>(p, nxt, kb0, nbw, g, tq, f[1]);
+      compute_frag<NT, KV, T>(p, f[0], rb, kb0, mu, xb, qbase, nbw, g, acc);
+    } else {
+      if (nxt < p.row_blocks) load_frag<NT, KV, T>(p, nxt, kb0, nbw, g, tq, f[0]);
+      compute_frag<NT, KV, T>(p, f[1], rb, kb0, mu, xb, qbase, nbw, g, acc);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(TM, TN, false, false);
-      bool ok = mbar_wait(full_x, 0, abort_flag, p.wait_limit);
-      for (int ti = 0; ti < nt && ok; ++ti) {
-        const int b = ti & 1;
-        if (ti >= 2) ok = mbar_wait(&tmem_free[b], ((ti >> 1) - 1) & 1, abort_flag, p.wait_limit);
-        // one A stage = one code stage: up to four 64-deep sub-steps, 16 MMAs
-        for (int st = 0; st < nst && ok; ++st) {
-          const int G = ti * nst + st, aslot = G % A_STAGES;
-          ok = mbar_wait(&a_full[aslot], (G / A_STAGES) & 1, abort_flag, p.wait_limit);
-          if (!ok) break;
-          tc_fence_after();
-          const int nsub = min(SUB, per_q - st * SUB);
-          for (int u = 0; u < nsub; ++u) {
-            const int j = st * SUB + u;
-            const uint32_t x_addr = smem_u32(xs + j * X_SUB_BYTES);
-            const uint32_t a_col = A_COL0 + aslot * A_STAGE_COLS + u * 32;
+    float* rbuf = red_dyn + (it & 1) * red_floats<NT, T>();
+    stash<NT, T>(rbuf, acc, warp, g, tq);
+    __syncthreads();
+    // thread -> (row, token) of the row block; the 16 warps summed in order
+    const int row_l = threadIdx.x / TOK, tok = threadIdx.x % TOK;
+    const int row = rb * ROWS + row_l;
+    if (row_l < ROWS && tok < p.M && row < p.N) {
+      float sum = 0.0f;
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              mma_ts(tmem + 16 * b, tmem + a_col + kk * 8, sdesc_sw128(x_addr + kk * 32, 16, 1024), idesc,
-                     (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&a_empty[aslot]);
-          mma_commit(&empty_c[G % C]);
-        }
-        if (ok) mma_commit(&acc_full[b]);
-      }
-    }
-  } else if (warp < DRAIN_WARP0) {
-    // ------------------------------------------------------ dequant producers
-    // group grp expands the A stages G = grp, grp+2, ... of this CTA's
-    // sequence (tile by tile; one A stage = the up to four 64-deep sub-steps
-    // of one code stage); warp: TMEM lanes 32*(warp&3) (weight rows) and half
-    // of the 64 codes of each sub-step
-    const int grp = (warp - 2) / GROUP_WARPS;
-    const int half = ((warp - 2) >> 2) & 1;
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const float mu = p.wc.absmax ? 0.0f : *p.wc.offset;
-    const uint32_t qbase = smem_u32(qtab);   // low byte 0
-    // block constants of the sub-steps of stage st of tile ti (raw: absmax, or
-    // scale2 and the E4M3 code)
-    auto load_c = [&](int ti, int st, float2 (&r)[SUB]) {
-#pragma unroll
-      for (int u = 0; u < SUB; ++u) r[u] = make_float2(0.0f, 0.0f);
-      if (ti >= nt) return;
-      const int n = tile_of(ti) * TM + row;
-      if (n >= p.N) return;
-#pragma unroll
-      for (int u = 0; u < SUB; ++u) {
-        const int j = st * SUB + u;
-        if (j >= per_q) break;
-        const int64_t b = (int64_t)n * p.kb_total + kb0 + j;
-        if (p.wc.absmax) r[u].x = __ldg(p.wc.absmax + b);
-        else { r[u].x = __ldg(p.wc.scale2 + (b >> 8)); r[u].y = __uint_as_float((uint32_t)__ldg(p.wc.absmax_q + b)); }
-      }
-    };
-    // (tile, stage) two stages further on: this group's next stage
-    auto advance2 = [&](int& ti, int& st) {
-      st += 2;
-      while (st >= nst) { st -= nst; ++ti; }
-    };
-    int ti = 0, st = grp;
-    while (st >= nst) { st -= nst; ++ti; }
-    int nti = ti, nst2 = st;
-    advance2(nti, nst2);
-    float2 cur[SUB], nxt[SUB];
-    load_c(ti, st, cur);
-    bool ok = true;
-    for (int G = grp; ti < nt && ok; G += 2) {
-      const int cslot = G & (C - 1);
-      const int aslot = G % A_STAGES;
-      const bool valid = tile_of(ti) * TM + row < p.N;
-      const int nsub = min(SUB, per_q - st * SUB);
-      load_c(nti, nst2, nxt);
-      ok = __all_sync(0xffffffffu, mbar_wait(&full_c[cslot], (G >> p.c_log) & 1, abort_flag, p.wait_limit) &&
-                                       (G < A_STAGES ||
-                                        mbar_wait(&a_empty[aslot], ((G / A_STAGES) - 1) & 1, abort_flag, p.wait_limit)));
-      if (!ok) break;
-      tc_fence_after();
-      const uint8_t* cst = cring + cslot * C_STAGE_BYTES;
-#pragma unroll
-      for (int u = 0; u < SUB; ++u) {
-        if (u >= nsub) break;
-        uint32_t out[16];
-        if (valid) {
-          const float c = p.wc.absmax ? cur[u].x
-                                      : __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)__float_as_uint(cur[u].y)), cur[u].x), mu);
-          // 128-byte code rows with the 128B swizzle: 16-byte chunk ^= row mod 8
-          const uint32_t coff = row * 128 + (((2 * u + half) ^ (row & 7)) << 4);
-          const uint4 cw = *reinterpret_cast<const uint4*>(cst + coff);
-          const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            // element i of the word is nibble i; its level sits at qbase + 4 * nibble
-            const uint32_t e4 = (w[q4] << 2) & 0x3C3C3C3Cu;   // 4 * low nibble of each byte
-            const uint32_t o4 = (w[q4] >> 2) & 0x3C3C3C3Cu;   // 4 * high nibble of each byte
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-              // byte bb of e4 / o4 under the table base's upper three bytes
-              const float fe = lds_f32(__byte_perm(e4, qbase, 0x7650u | bb));
-              const float fo = lds_f32(__byte_perm(o4, qbase, 0x7650u | bb));
-              float pe, po;
-              mul2_rn(fe, fo, c, pe, po);
-              out[4 * q4 + bb] = pack_bf16x2(pe, po);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int t = 0; t < 16; ++t) out[t] = 0u;
-        }
-        tmem_st16(tmem + ((uint32_t)(quad * 32) << 16) +
-                      (uint32_t)(A_COL0 + aslot * A_STAGE_COLS + u * 32 + half * 16),
-                  out);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[aslot]);
-#pragma unroll
-      for (int u = 0; u < SUB; ++u) cur[u] = nxt[u];
-      ti = nti;
-      st = nst2;
-      advance2(nti, nst2);
-    }
-  } else {
-    // ---------------------------------------- drain, cluster reduction, output
-    const int t = threadIdx.x - DRAIN_WARP0 * 32;   // 0..127
-    const int quad = warp & 3;
-    const int drow = quad * 32 + lane;              // the TMEM lane this thread drains
-    for (int i = t; i < p.M * p.r; i += DRAIN_WARPS * 32) us[i] = __bfloat162float(p.U[i]);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    // this CTA's share of the tile's (row, token pair) outputs, token pair fastest
-    const int items = TM * (TN / 2);
-    const int i0 = items * q / cs, i1 = items * (q + 1) / cs;
-    // adapter row of an item, 16-byte loads issued together
-    uint4 bv[MAX_R / 8];
-    auto load_brow = [&](int n) {
-#pragma unroll
-      for (int c8 = 0; c8 < MAX_R / 8; ++c8)
-        if (c8 * 8 < p.r && n < p.N) bv[c8] = *reinterpret_cast<const uint4*>(p.B + (size_t)n * p.r + c8 * 8);
-    };
-    bool ok = true;
-    for (int ti = 0; ti < nt && ok; ++ti) {
-      const int b = ti & 1;
-      const int n0 = tile_of(ti) * TM;
-      float* rb = red + b * (TM * RED_LD);
-      // the first item's adapter row is fetched while the tile is still being computed
-      if (p.r > 0 && i0 + t < i1) load_brow(n0 + ((i0 + t) >> 3));
-      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], (ti >> 1) & 1, abort_flag, p.wait_limit));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t v[16];
-      tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(16 * b), v);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tmem_free[b]);
-      // the other CTAs are done reading this buffer's previous tile
-      if (ti >= 2) ok = __all_sync(0xffffffffu, mbar_wait_cluster(&freed[b], ((ti >> 1) - 1) & 1, abort_flag, p.wait_limit));
-      if (!ok) break;
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        *reinterpret_cast<float2*>(rb + drow * RED_LD + 2 * k) =
-            make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-      __syncwarp();
-      if (lane == 0)
-        for (int pr = 0; pr < cs; ++pr) arrive_remote_release(&ready[b], (uint32_t)pr);
-      ok = __all_sync(0xffffffffu, mbar_wait_cluster(&ready[b], (ti >> 1) & 1, abort_flag, p.wait_limit));
-      if (!ok) break;
-      const uint32_t rb_addr = smem_u32(rb);
-      for (int it = i0 + t; it < i1; it += DRAIN_WARPS * 32) {
-        const int r_in = it >> 3, tp = it & 7;
-        const int n = n0 + r_in, m0 = 2 * tp;
-        if (p.r > 0 && it != i0 + t) load_brow(n);
-        if (n >= p.N || m0 >= p.M) continue;
-        const uint32_t off = rb_addr + (uint32_t)((r_in * RED_LD + m0) * 4);
-        // every slice's partial in flight at once, added in slice order
-        float2 x[MAX_CS];
-#pragma unroll
-        for (int pr = 0; pr < MAX_CS; ++pr)
-          if (pr < cs) x[pr] = ld_cluster_f2(cluster_map(off, (uint32_t)pr));
-        float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int pr = 0; pr < MAX_CS; ++pr)
-          if (pr < cs) {
-            acc.x = __fadd_rn(acc.x, x[pr].x);
-            acc.y = __fadd_rn(acc.y, x[pr].y);
-          }
-        float o[2] = {acc.x, acc.y};
-        if (p.r > 0) {
-#pragma unroll
-          for (int mm = 0; mm < 2; ++mm) {
-            if (m0 + mm >= p.M) break;
-            const float* um = us + (m0 + mm) * p.r;
-            float l = 0.0f;
-#pragma unroll
-            for (int c8 = 0; c8 < MAX_R / 8; ++c8) {
-              if (c8 * 8 >= p.r) break;
-              const uint32_t bw[4] = {bv[c8].x, bv[c8].y, bv[c8].z, bv[c8].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                l = fmaf(um[c8 * 8 + 2 * e], bf16_lo(bw[e]), l);
-                l = fmaf(um[c8 * 8 + 2 * e + 1], bf16_hi(bw[e]), l);
-              }
-            }
-            o[mm] = __fadd_rn(o[mm], __fmul_rn(p.s, l));
-          }
-        }
-#pragma unroll
-        for (int mm = 0; mm < 2; ++mm) {
-          if (m0 + mm >= p.M) break;
-          const size_t yo = (size_t)(m0 + mm) * p.N + n;
-          if (p.y_bf16) reinterpret_cast<__nv_bfloat16*>(p.Y)[yo] = __float2bfloat16_rn(o[mm]);
-          else reinterpret_cast<float*>(p.Y)[yo] = o[mm];
-        }
-      }
-      __syncwarp();
-      if (lane == 0)
-        for (int pr = 0; pr < cs; ++pr) arrive_remote_release(&freed[b], (uint32_t)pr);
+      for (int w = 0; w < WARPS; ++w) sum = __fadd_rn(sum, rbuf[w * (ROWS * TOK) + row_l * TOK + tok]);
+      p.part_y[((size_t)part * p.N + row) * p.M + tok] = sum;
     }
   }
-  tc_fence_before();
-  cluster_sync();   // no CTA leaves while another may still read its shared memory or arrive on its barriers
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+  // this part's share of U = X A^T: the CTA with the last row block of the part
+  if (blockIdx.y == (p.row_blocks - 1) % gridDim.y && p.r > 0) {
+    __syncthreads();
+    float* ubuf = red_dyn;                      // [warp][16 adapter rows][TOK tokens] fits in one buffer
+    for (int rt = 0; rt < (p.r + 15) / 16; ++rt) {
+      float acc[NT][4];
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
+      const int ja = 16 * rt + g, jb = ja + 8;
+#pragma unroll
+      for (int j = 0; j < KV / 64; ++j) {
+        if (j < nbw) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const size_t off = (size_t)k0 + 64 * j + 16 * tq + 4 * u;
+            uint2 va = make_uint2(0u, 0u), vb = make_uint2(0u, 0u);
+            if (ja < p.r) va = __ldg(reinterpret_cast<const uint2*>(p.A + (size_t)ja * p.K + off));
+            if (jb < p.r) vb = __ldg(reinterpret_cast<const uint2*>(p.A + (size_t)jb * p.K + off));
+#pragma unroll
+            for (int n = 0; n < NT; ++n) mma_bf16(acc[n], va.x, vb.x, va.y, vb.y, xb[4 * j + u][n][0], xb[4 * j + u][n][1]);
+          }
+        }
+      }
+      float* base = ubuf + warp * (16 * TOK);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int tok = 8 * n + 2 * tq;
+        *reinterpret_cast<float2*>(base + g * TOK + tok) = make_float2(acc[n][0], acc[n][1]);
+        *reinterpret_cast<float2*>(base + (g + 8) * TOK + tok) = make_float2(acc[n][2], acc[n][3]);
+      }
+      __syncthreads();
+      const int jl = threadIdx.x / TOK, tok = threadIdx.x % TOK;
+      const int jr = 16 * rt + jl;
+      if (jl < 16 && jr < p.r && tok < p.M) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) sum = __fadd_rn(sum, ubuf[w * (16 * TOK) + jl * TOK + tok]);
+        p.part_u[((size_t)part * p.M + tok) * p.r + jr] = sum;
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Y[m, n] = (sum over parts, in order) + fl32(s * sum_j U[m, j] B[n, j]),
+// U = bf16(sum over parts of the U shares, in order); U_out gets U.
+__global__ void __launch_bounds__(256) smallm_finish_kernel(const float* __restrict__ part_y,
+                                                            const float* __restrict__ part_u, int parts, int M, int N,
+                                                            int r, float s, const __nv_bfloat16* __restrict__ B,
+                                                            void* Y, int y_bf16, __nv_bfloat16* U_out) {
+  __shared__ float u_s[MAX_M * MAX_R];
+  pdl_wait();
+  pdl_trigger();
+  for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+    float sum = 0.0f;
+    for (int q = 0; q < parts; ++q) sum = __fadd_rn(sum, part_u[(size_t)q * M * r + i]);
+    const __nv_bfloat16 ub = __float2bfloat16_rn(sum);
+    u_s[i] = __bfloat162float(ub);
+    if (blockIdx.x == 0 && U_out) U_out[i] = ub;
+  }
+  __syncthreads();
+  const int64_t total = (int64_t)N * M;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int n = (int)(i / M), m = (int)(i % M);
+    float y = 0.0f;
+    for (int q = 0; q < parts; ++q) y = __fadd_rn(y, part_y[(size_t)q * total + i]);
+    if (r > 0) {
+      float l = 0.0f;
+      const __nv_bfloat16* brow = B + (size_t)n * r;
+      for (int j = 0; j < r; ++j) l = __fadd_rn(l, __fmul_rn(u_s[m * r + j], __bfloat162float(brow[j])));
+      y = __fadd_rn(y, __fmul_rn(s, l));
+    }
+    const int64_t o = (int64_t)m * N + n;
+    if (y_bf16) reinterpret_cast<__nv_bfloat16*>(Y)[o] = __float2bfloat16_rn(y);
+    else reinterpret_cast<float*>(Y)[o] = y;
   }
 }
 
 }  // namespace smallm
 
-static int sm_count_sm() {
-  const int c = device_sm_count();
-  return c > 0 ? c : 148;
-}
-
-struct SmallmPlan {
-  int cs, per, c_stages, c_log, clusters;
-  size_t smem;
+// Tile shape per token count: one token tile of 8 (KV = 256 reduction
+// elements per warp) or two (KV = 128), one 16-row tile per row block: the
+// activation fragments take 32 registers either way.
+struct SmallmShape {
+  int nt, kv, t;
 };
+static SmallmShape smallm_shape(int64_t M) { return M <= 8 ? SmallmShape{1, 256, 1} : SmallmShape{2, 128, 1}; }
 
-static size_t smallm_static_smem() { return sizeof(float) * (smallm::TN * smallm::MAX_R); }
+static int smallm_parts(int64_t M, int64_t K) {
+  const SmallmShape sh = smallm_shape(M);
+  const int64_t part_k = (int64_t)smallm::WARPS * sh.kv;
+  return (int)((K + part_k - 1) / part_k);
+}
 
-// Shared memory for a K slice of `per` sub-steps; false if it cannot fit.
-static bool smallm_layout(int per, SmallmPlan& pl) {
+// Workspace of the small-token forward: part sums of Y [parts][N][M] and of U
+// [parts][M][r] (fp32), then U [M, r] bf16 when the caller does not take it.
+size_t smallm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  const size_t parts = (size_t)smallm_parts(M, K);
+  auto a256 = [](size_t b) { return (b + 255) & ~(size_t)255; };
+  return a256(parts * N * M * 4) + a256(parts * M * std::max(r, 1) * 4) + a256((size_t)M * std::max(r, 1) * 2);
+}
+
+bool smallm_supported(int64_t N, int64_t K) { return N >= 1 && K >= 64 && K % 64 == 0; }
+
+ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* A, const void* B, int r,
+                            float s, void* Y, ql_dtype y_dt, void* U_out, void* ws, cudaStream_t st) {
   using namespace smallm;
-  if (per > MAX_PER) return false;
-  // alignment slack, the X slice, two reduction buffers, the level table,
-  // 33 mbarriers + TMEM address + abort flag
-  const size_t fixed = 1024 + (size_t)per * X_SUB_BYTES + 2 * RED_BYTES + 256 + 512;
-  const size_t limit = 227 * 1024 - smallm_static_smem();
-  if (fixed + 2 * C_STAGE_BYTES > limit) return false;
-  int c = 2, lg = 1;
-  while (c * 2 <= MAX_C_STAGES && fixed + (size_t)(c * 2) * C_STAGE_BYTES <= limit) {
-    c *= 2;
-    ++lg;
-  }
-  pl.per = per;
-  pl.c_stages = c;
-  pl.c_log = lg;
-  pl.smem = fixed + (size_t)c * C_STAGE_BYTES;
-  return true;
-}
-
-static bool smallm_attr() {
-  return per_device(reinterpret_cast<const void*>(smallm::smallm_kernel), 0, [] {
-           if (cudaFuncSetAttribute(smallm::smallm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)(227 * 1024 - smallm_static_smem())) != cudaSuccess ||
-               cudaFuncSetAttribute(smallm::smallm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
-                   cudaSuccess) {
-             cudaGetLastError();
-             return -1;
-           }
-           return 1;
-         }) > 0;
-}
-
-// Cluster size (CTAs sharing K) and cluster count: the tiles are handed out in
-// rounds of `clusters`, each round costing about `per` sub-steps, scaled up
-// when the code ring is shallower than 8 stages; pick the cheapest among the
-// cluster sizes that fit (the cluster count comes from the occupancy
-// calculator: a cluster's CTAs must share a GPC, which caps it below SMs / cs).
-static bool smallm_plan(int64_t N, int64_t K, SmallmPlan& best, bool query) {
-  using namespace smallm;
-  const int kb = (int)(K / BK);
-  if (kb < 1) return false;
-  const int tiles = (int)((N + TM - 1) / TM);
-  bool found = false;
-  long best_cost = 0;
-  for (int cs0 = std::min(MAX_CS, kb); cs0 >= 1; --cs0) {
-    SmallmPlan pl;
-    const int per = (kb + cs0 - 1) / cs0;
-    if (!smallm_layout(per, pl)) continue;
-    pl.cs = (kb + per - 1) / per;
-    int maxc = sm_count_sm() / pl.cs;
-    if (query) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)pl.cs, (unsigned)std::max(1, maxc));
-      cfg.blockDim = dim3(THREADS);
-      cfg.dynamicSmemBytes = pl.smem;
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = (unsigned)pl.cs;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      cfg.attrs = at;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, smallm_kernel, &cfg) == cudaSuccess && n > 0) maxc = std::min(maxc, n);
-      else cudaGetLastError();
-    }
-    pl.clusters = std::max(1, std::min(tiles, maxc));
-    const long rounds = (tiles + pl.clusters - 1) / pl.clusters;
-    // a CTA streams its codes at a rate that grows with the bytes it has in
-    // flight, up to about 8 stages (128 KB): shallower rings cost in proportion
-    const long cost = rounds * per * (MAX_C_STAGES / pl.c_stages);
-    if (!found || cost < best_cost) {
-      best = pl;
-      best_cost = cost;
-      found = true;
-    }
-  }
-  return found;
-}
-
-// Whether the small-token kernel handles this shape (its K slice of X must fit
-// in shared memory: K <= 40960 with eight slices).
-bool smallm_supported(int64_t N, int64_t K) {
-  SmallmPlan pl;
-  return smallm_plan(N, K, pl, false);
-}
-
-// Y = X W_hat^T + s U B^T for M <= 16; U [M, r] given (bf16).
-ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, const void* U, const void* B, int r,
-                            float s, void* Y, ql_dtype y_dt, cudaStream_t st) {
-  using namespace smallm;
-  if (M < 1 || M > TN || r > MAX_R) return QL_ERR_UNSUPPORTED;
+  if (M < 1 || M > MAX_M || r > MAX_R) return QL_ERR_UNSUPPORTED;
   const int N = (int)w->rows, K = (int)w->cols;
-  if (!smallm_attr()) return QL_ERR_CUDA;
-  // the plan for a weight shape is fixed: computed once per shape and device
-  // (the layers of a model alternate a few shapes)
-  struct Entry {
-    int64_t N, K;
-    int dev;
-    SmallmPlan pl;
-  };
-  static std::mutex mu;
-  static std::vector<Entry> cache;
-  const int dev = current_device();
-  SmallmPlan pl;
-  bool have = false;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    for (const Entry& e : cache)
-      if (e.N == N && e.K == K && e.dev == dev) {
-        pl = e.pl;
-        have = true;
-        break;
-      }
-  }
-  if (!have) {
-    if (!smallm_plan(N, K, pl, true)) return QL_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lk(mu);
-    if (cache.size() < 256) cache.push_back(Entry{N, K, dev, pl});
-  }
-  CUtensorMap map_x, map_codes;
-  if (!make_map_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, TN,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
-    return QL_ERR_CUDA;
-  if (!make_map_2d(&map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, (uint64_t)K / 2, (uint64_t)N,
-                   (uint64_t)K / 2, SUB * BK / 2, TM, CU_TENSOR_MAP_SWIZZLE_128B))
-    return QL_ERR_CUDA;
+  const SmallmShape sh = smallm_shape(M);
+  const int parts = smallm_parts(M, K);
+  auto a256 = [](size_t b) { return (b + 255) & ~(size_t)255; };
+  uint8_t* wp = reinterpret_cast<uint8_t*>(ws);
+  float* part_y = reinterpret_cast<float*>(wp);
+  float* part_u = reinterpret_cast<float*>(wp + a256((size_t)parts * N * M * 4));
+  __nv_bfloat16* U = U_out ? reinterpret_cast<__nv_bfloat16*>(U_out)
+                           : reinterpret_cast<__nv_bfloat16*>(wp + a256((size_t)parts * N * M * 4) +
+                                                              a256((size_t)parts * M * std::max(r, 1) * 4));
   Params p;
   p.M = (int)M;
   p.N = N;
   p.K = K;
   p.r = r;
-  p.kb_total = K / BK;
-  p.per = pl.per;
-  p.tiles = (N + TM - 1) / TM;
-  p.c_stages = pl.c_stages;
-  p.c_log = pl.c_log;
-  p.s = s;
+  p.kb = K / 64;
+  p.parts = parts;
+  p.part_k = WARPS * sh.kv;
+  p.row_blocks = (N + 16 * sh.t - 1) / (16 * sh.t);
   p.wc = WeightConsts{w->absmax, w->absmax_q, w->scale2, w->offset};
   p.tab = nf4_table();
-  p.U = (const __nv_bfloat16*)U;
-  p.B = (const __nv_bfloat16*)B;
-  p.Y = Y;
-  p.y_bf16 = y_dt == QL_BF16;
-  p.wait_limit = 1u << 22;
+  p.codes = w->codes;
+  p.X = reinterpret_cast<const __nv_bfloat16*>(X);
+  p.A = reinterpret_cast<const __nv_bfloat16*>(A);
+  p.part_y = part_y;
+  p.part_u = part_u;
+  const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+  const int gy = std::max(1, std::min(p.row_blocks, std::max(1, sms / parts)));
+  const dim3 grid((unsigned)parts, (unsigned)gy);
+  const size_t smem = sizeof(float) * 2 * (sh.nt == 1 ? red_floats<1, 1>() : red_floats<2, 1>());
+  auto set_smem = [smem](const void* k) {
+    return per_device(k, 0, [k, smem] {
+             if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+               cudaGetLastError();
+               return -1;
+             }
+             return 1;
+           }) > 0;
+  };
   TraceScope ts(TK_SMALLM, st);
-  QL_CUDA_TRY(launch(smallm_kernel, dim3((unsigned)pl.cs, (unsigned)pl.clusters), dim3(THREADS), pl.smem, st,
-                     (unsigned)pl.cs, 1, map_x, map_codes, p));
+  if (sh.nt == 1) {
+    if (!set_smem(reinterpret_cast<const void*>(smallm_kernel<1, 256, 1>))) return QL_ERR_CUDA;
+    QL_CUDA_TRY(launch(smallm_kernel<1, 256, 1>, grid, dim3(THREADS), smem, st, 1, 1, p));
+  } else {
+    if (!set_smem(reinterpret_cast<const void*>(smallm_kernel<2, 128, 1>))) return QL_ERR_CUDA;
+    QL_CUDA_TRY(launch(smallm_kernel<2, 128, 1>, grid, dim3(THREADS), smem, st, 1, 1, p));
+  }
+  const int64_t total = (int64_t)N * M;
+  const unsigned fgrid = (unsigned)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, (int64_t)sms * 4));
+  QL_CUDA_TRY(launch(smallm_finish_kernel, dim3(fgrid), dim3(256), 0, st, 1, 1, (const float*)part_y,
+                     (const float*)part_u, parts, (int)M, N, r, s, reinterpret_cast<const __nv_bfloat16*>(B), Y,
+                     y_dt == QL_BF16 ? 1 : 0, U));
+  QL_LAUNCH_CHECK();
   return QL_OK;
 }
 

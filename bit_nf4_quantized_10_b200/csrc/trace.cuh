@@ -24,6 +24,8 @@ enum TraceKind : int {
   TK_SMALLM,
   TK_TRANSPOSE,
   TK_MERGE,
+  TK_FP4,
+  TK_ADAMW,
   TK_COUNT
 };
 

@@ -130,6 +130,30 @@ ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q,
                            void* stream);
 
 /*
+ * Double quantization of a weight quantized in row slabs on several ranks
+ * (data parallelism, each rank holding one slab).  The result is the double
+ * quantization of [P2] §2.2 and [P3] "Double quantization: the constants are
+ * not free" for the whole tensor; the split is this library's data-parallel
+ * layout (the pages quantize on one GPU).  The mean is a sum over a
+ * fixed adjacent-pair tree whose level-1 nodes are float64 sums of 2048
+ * consecutive constants, so a slab whose constants start on a multiple of 2048
+ * owns whole nodes:
+ *   nf4_double_quant_level1  this slab's nodes: nodes[ceil(nb/2048)] (float64)
+ *   nf4_double_quant_finish  given every slab's nodes in slab order
+ *                            (n_nodes = ceil(nb_total/2048)), the mean of the
+ *                            whole tensor and this slab's codes and scales
+ * The concatenated results equal nf4_double_quant of the whole tensor bit for
+ * bit.  The caller moves the nodes between ranks (an all-gather).  ws as for
+ * nf4_double_quant with nb_total.  Errors: QL_ERR_INVALID_ARG (counts, a NULL
+ * or misaligned pointer, n_nodes inconsistent with nb_total),
+ * QL_ERR_WORKSPACE, QL_ERR_CUDA.
+ */
+ql_status nf4_double_quant_level1(const float* absmax, int64_t nb, double* nodes, void* stream);
+ql_status nf4_double_quant_finish(const double* nodes, int64_t n_nodes, int64_t nb_total, const float* absmax,
+                                  int64_t nb, uint8_t* absmax_q, float* scale2, float* offset, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/*
  * nf4_double_quant_noalloc — nf4_double_quant for callers that cannot
  * allocate device memory (no workspace argument).  The pages have no
  * counterpart; this is a library convenience.  Callers such as a plugin or
@@ -140,12 +164,14 @@ ql_status nf4_double_quant(const float* absmax, int64_t nb, uint8_t* absmax_q,
  *   nb must be <= QL_NOALLOC_MAX_BLOCKS (64 Mi constants, i.e. weights of up
  *   to 4 Gi elements); larger nb returns QL_ERR_UNSUPPORTED.
  *   The scratch is a fixed 256.5 KiB array of device memory inside the
- *   library, held by every GPU that loads it until the process exits.  The
- *   first call on a device looks its address up (cudaGetSymbolAddress), so
- *   make that first call before any stream capture.  All calls on a device
- *   share the array: calls whose kernels may overlap on the GPU (different
- *   streams with no ordering) race and must not be issued.  The library never
- *   calls cudaMalloc, cudaFree or an allocating routine here.
+ *   library, held by every GPU that loads it until the process exits (one
+ *   copy per CUDA context, since the library's module is loaded per context).
+ *   The first call in a context looks its address up (cudaGetSymbolAddress)
+ *   and caches it under the context's unique ID, so make that first call
+ *   before any stream capture.  All calls in a context share the array: calls
+ *   whose kernels may overlap on the GPU (different streams with no ordering)
+ *   race and must not be issued.  The library never calls cudaMalloc, cudaFree
+ *   or an allocating routine here.
  */
 #define QL_NOALLOC_MAX_BLOCKS (1ll << 26)
 ql_status nf4_double_quant_noalloc(const float* absmax, int64_t nb, uint8_t* absmax_q,
@@ -200,7 +226,8 @@ ql_status nf4_dequant(const ql_nf4_weight* w, void* out, ql_dtype out_dt, void* 
  *   Y      device out [M, N] of y_dt
  *   U_out  device out bf16 [M, r] (the tensor the backward reuses) or NULL
  *   ws     workspace >= qlora_workspace_size(QL_OP_FWD, M, N, K, r) (0 when
- *          r == 0; ws may then be NULL)
+ *          r == 0 and M > 16; ws may then be NULL).  For 1 <= M <= 16 the
+ *          small-token kernels keep fp32 part sums of Y and U there.
  * The main product accumulates in fp32 on the tensor cores from the exact
  * bf16 W_hat.  U is accumulated in fp32 (split over K, summed in a fixed
  * order) and rounded to bf16; the adapter term U (s B)^T enters the main fp32
@@ -251,10 +278,76 @@ ql_status qlora_silu_gate_fwd(const void* g, const void* u, void* h, int64_t n, 
 ql_status qlora_silu_gate_bwd(const void* dh, const void* g, const void* u,
                               void* dg, void* du, int64_t n, void* stream);
 
+/*
+ * 4-bit float block formats ([P1] "Lesson 4 of the Finetuning Sessions",
+ * "From FP32 to the 4-Bit Horizon": MXFP4 shares one 8-bit power-of-two (E8M0)
+ * scale over 32 elements; NVFP4 shares one E4M3 scale over 16; "From Turing to
+ * Blackwell": the 5th-generation tensor cores execute them natively).
+ * Elements are E2M1 (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), rounded to
+ * nearest even and saturated at +-6; elements 2j, 2j+1 share byte j (low
+ * nibble first); an odd n pads the last high nibble with +0.
+ *
+ * nvfp4_quantize: x device (x_dt) [n]; codes out uint8 [ceil(n/2)]; scales
+ *   out uint8 [ceil(n/16)] E4M3 codes S_b; tensor_scale out fp32 [1]: s_t =
+ *   fl32(amax / 2688) when use_tensor_scale (1 otherwise; 2688 = 6 * 448).
+ *   Steps (fp32, one rounding each): denom = fl32(6 s_t), S_b =
+ *   E4M3_rne_satfinite(fl32(amax_b / denom)), scale = fl32(S_b s_t), code =
+ *   E2M1(fl32(x / scale)), 0 where scale == 0.  ws >=
+ *   qlora_workspace_size(QL_OP_NVFP4, n, 0, 0, 0) (the tensor maximum).
+ * mxfp4_quantize: scales out uint8 [ceil(n/32)] E8M0 codes k_b + 127, k_b =
+ *   floor(log2 amax_b) - 2 clamped to [-127, 127] (-127 for an all-zero
+ *   block); code = E2M1(x 2^-k_b).
+ * nvfp4_dequant / mxfp4_dequant: out fp32 [n], x_hat = fl32(E2M1(code)
+ *   fl32(S_b s_t)) / E2M1(code) 2^k_b (exact).
+ * NaN/Inf in the input sets QL_ERR_NONFINITE in the status word (outputs are
+ * then unspecified).  Errors: QL_ERR_INVALID_ARG (n <= 0, a NULL or misaligned
+ * pointer, an unknown dtype), QL_ERR_WORKSPACE, QL_ERR_CUDA.
+ */
+ql_status nvfp4_quantize(const void* x, ql_dtype x_dt, int64_t n, int use_tensor_scale, uint8_t* codes,
+                         uint8_t* scales, float* tensor_scale, void* ws, size_t ws_bytes, void* stream);
+ql_status mxfp4_quantize(const void* x, ql_dtype x_dt, int64_t n, uint8_t* codes, uint8_t* scales, void* stream);
+ql_status nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale, int64_t n,
+                        float* out, void* stream);
+ql_status mxfp4_dequant(const uint8_t* codes, const uint8_t* scales, int64_t n, float* out, void* stream);
+
+/*
+ * qlora_adamw_step — one AdamW update of adapter parameters with fp32 states
+ * (the paged optimizer: [P2] §2.3 and [P3] "Paged optimizers: surviving the
+ * spikes" keep the states in unified memory, paged to host RAM under memory
+ * pressure and back for the next update; [P3] "How it's used in practice"
+ * names the 32-bit variant).  The pages give no update formula; paging leaves
+ * the arithmetic alone, so this is AdamW with decoupled weight decay.  Per
+ * element, each operation one fp32 IEEE operation in this order, with keep =
+ * fl32(1 - lr wd), c1 = fl32(1 - beta1^t), c2 = fl32(1 - beta2^t) computed on
+ * the host in float64 from the fp32 arguments:
+ *   p = fl32(p keep);  m = fl32(fl32(beta1 m) + fl32((1 - beta1) g));
+ *   v = fl32(fl32(beta2 v) + fl32(fl32((1 - beta2) g) g));
+ *   d = fl32(fl32(sqrt(fl32(v / c2))) + eps);
+ *   p = fl32(p - fl32(lr fl32(fl32(m / c1) / d))).
+ *   p, m, v  fp32 [n], updated in place; g fp32 [n].  Device memory or CUDA
+ *            managed memory (wherever its pages currently are).
+ *   p_bf16   bf16 [n] copy of the updated p (the adapter the linear reads), or
+ *            NULL.   t: step number, >= 1.
+ * Errors: QL_ERR_INVALID_ARG (n <= 0, t < 1, a beta outside [0, 1), eps < 0,
+ * a NULL or misaligned pointer), QL_ERR_CUDA.
+ *
+ * qlora_paged_prefetch — move a managed range (cudaMallocManaged memory owned
+ * by the caller) to the current device (QL_PAGE_DEVICE), before an update, or
+ * to host memory (QL_PAGE_HOST), to free device memory after one; stream
+ * ordered.  Errors: QL_ERR_INVALID_ARG (NULL, bytes == 0, an unknown `where`,
+ * memory that is not managed), QL_ERR_CUDA.
+ */
+#define QL_PAGE_DEVICE 0
+#define QL_PAGE_HOST 1
+ql_status qlora_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int64_t t,
+                           float lr, float beta1, float beta2, float eps, float weight_decay, void* stream);
+ql_status qlora_paged_prefetch(const void* ptr, size_t bytes, int where, void* stream);
+
 /* Workspace query.  op: one of the QL_OP_* values; unused sizes are ignored. */
 #define QL_OP_DOUBLE_QUANT 0   /* M = nb */
 #define QL_OP_FWD 1
 #define QL_OP_BWD 2
+#define QL_OP_NVFP4 3          /* M = n */
 size_t qlora_workspace_size(int op, int64_t M, int64_t N, int64_t K, int r);
 
 /* Bytes needed for n parameters: ceil(n/2) codes + (dq ? nb + 4*ng + 4 : 4*nb)

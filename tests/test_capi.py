@@ -56,6 +56,7 @@ def test_workspace_sizes(lib):
     assert lib.qlora_workspace_size(lib.QL_OP_FWD, 4096, 4096, 4096, 16) >= 4096 * 16 * 2
     assert lib.qlora_workspace_size(lib.QL_OP_FWD, 4096, 4096, 4096, 0) == 0
     assert lib.qlora_workspace_size(lib.QL_OP_BWD, 4096, 4096, 4096, 16) >= 2 * 4096 * 16 * 2
+    assert lib.qlora_workspace_size(lib.QL_OP_NVFP4, 100) >= 4
 
 
 def test_argument_errors_return_before_launch(lib):
@@ -90,6 +91,28 @@ def test_argument_errors_return_before_launch(lib):
     assert L.qlora_merge(ctypes.byref(w), fake, fake, 65, 2.0, fake, None, None, s0) == lib.QL_ERR_UNSUPPORTED
     assert L.qlora_merge(ctypes.byref(w), None, fake, 8, 2.0, fake, None, None, s0) == lib.QL_ERR_INVALID_ARG
     assert L.qlora_merge(ctypes.byref(w), fake, fake, 8, 2.0, fake + 8, None, None, s0) == lib.QL_ERR_INVALID_ARG
+    # 4-bit float formats, the AdamW step and the paging helper
+    assert L.nvfp4_quantize(fake, lib.QL_BF16, 0, 1, fake, fake, fake, fake, 256, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.nvfp4_quantize(fake, lib.QL_BF16, 64, 1, fake, fake, fake, fake, 0, s0) == lib.QL_ERR_WORKSPACE
+    assert L.nvfp4_quantize(fake, lib.QL_BF16, 64, 1, fake + 4, fake, fake, fake, 256, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.mxfp4_quantize(fake, 9, 64, fake, fake, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.mxfp4_quantize(None, lib.QL_F32, 64, fake, fake, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.nvfp4_dequant(fake, fake, None, 64, fake, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.mxfp4_dequant(fake, fake, -1, fake, s0) == lib.QL_ERR_INVALID_ARG
+    adam = lambda n, t, b1, b2, eps, g=fake: L.qlora_adamw_step(fake, g, fake, fake, None, n, t, 1e-3, b1, b2, eps,
+                                                                 0.0, s0)
+    assert adam(0, 1, 0.9, 0.999, 1e-8) == lib.QL_ERR_INVALID_ARG
+    assert adam(16, 0, 0.9, 0.999, 1e-8) == lib.QL_ERR_INVALID_ARG
+    assert adam(16, 1, 1.0, 0.999, 1e-8) == lib.QL_ERR_INVALID_ARG
+    assert adam(16, 1, 0.9, -0.5, 1e-8) == lib.QL_ERR_INVALID_ARG
+    assert adam(16, 1, 0.9, 0.999, -1.0) == lib.QL_ERR_INVALID_ARG
+    assert adam(16, 1, 0.9, 0.999, 1e-8, g=fake + 4) == lib.QL_ERR_INVALID_ARG
+    assert L.qlora_paged_prefetch(None, 64, lib.QL_PAGE_HOST, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.qlora_paged_prefetch(fake, 0, lib.QL_PAGE_HOST, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.qlora_paged_prefetch(fake, 64, 5, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.nf4_double_quant_finish(fake, 2, 2048, fake, 2048, fake, fake, fake, fake, 1 << 20,
+                                     s0) == lib.QL_ERR_INVALID_ARG     # 2 nodes for 2048 constants
+    assert L.nf4_double_quant_level1(fake, 0, fake, s0) == lib.QL_ERR_INVALID_ARG
     assert lib.status_string(lib.QL_ERR_TIMEOUT) == "device wait timed out"
     for polls in (0, -1, (1 << 20) + 1):
         assert L.qlora_selftest_wait_timeout(polls, s0) == lib.QL_ERR_INVALID_ARG
@@ -100,8 +123,8 @@ def test_boundary_calls_document_source_and_errors():
     states its error behaviour in the header comment right above it."""
     text = open(os.path.join(ROOT, "include", "qlora_nf4.h")).read()
     for name in ("nf4_quantize", "nf4_double_quant", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
-                 "qlora_merge"):
-        m = re.search(r"/\*((?:(?!\*/).)*?)\*/\s*(?:#define[^\n]*\n\s*)?ql_status\s+" + name + r"\s*\(", text, flags=re.S)
+                 "qlora_merge", "nvfp4_quantize", "qlora_adamw_step", "nf4_double_quant_level1"):
+        m = re.search(r"/\*((?:(?!\*/).)*?)\*/\s*(?:#define[^\n]*\n\s*)*ql_status\s+" + name + r"\s*\(", text, flags=re.S)
         assert m, name
         comment = m.group(1)
         assert re.search(r"\[P[1-5]\]", comment), f"{name}: no source citation"
@@ -109,13 +132,21 @@ def test_boundary_calls_document_source_and_errors():
 
 
 @pytest.mark.parametrize("M,N,K,r", [(4096, 4096, 4096, 16), (130, 512, 1024, 16), (1, 28672, 8192, 64),
-                                     (600, 384, 320, 8), (16, 256, 512, 8)])
+                                     (600, 384, 320, 8), (16, 256, 512, 8), (9, 28672, 8192, 16), (8, 1024, 4160, 0)])
 def test_workspace_sizes_follow_the_documented_layout(lib, M, N, K, r):
-    """Forward: U [M, r] bf16.  Backward: B^T [r, N], U^T [r, Mp], V [M, r],
-    V^T [r, Mp] bf16 (Mp = M rounded up to 8), each piece 256-byte aligned."""
+    """Forward: U [M, r] bf16; for 1 <= M <= 16 (the small-token kernels)
+    first the fp32 part sums of Y [parts, N, M] and of U [parts, M, r], parts =
+    ceil(K / 4096) for M <= 8 and ceil(K / 2048) above.  Backward: B^T [r, N],
+    U^T [r, Mp], V [M, r], V^T [r, Mp] bf16 (Mp = M rounded up to 8), each
+    piece 256-byte aligned."""
     a256 = lambda b: (b + 255) // 256 * 256
     Mp = (M + 7) // 8 * 8
-    assert lib.qlora_workspace_size(lib.QL_OP_FWD, M, N, K, r) == a256(M * r * 2)
+    if M <= 16:
+        parts = -(-K // (4096 if M <= 8 else 2048))
+        want_fwd = a256(parts * N * M * 4) + a256(parts * M * max(r, 1) * 4) + a256(M * max(r, 1) * 2)
+    else:
+        want_fwd = a256(M * r * 2)
+    assert lib.qlora_workspace_size(lib.QL_OP_FWD, M, N, K, r) == want_fwd
     want = a256(r * N * 2) + a256(r * Mp * 2) + a256(M * r * 2) + a256(r * Mp * 2)
     assert lib.qlora_workspace_size(lib.QL_OP_BWD, M, N, K, r) == want
     assert lib.qlora_workspace_size(lib.QL_OP_BWD, M, N, K, 0) == 0

@@ -12,7 +12,7 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from bit_nf4_quantized_10_b200.dp import token_shard, allreduce_adapter_grads
+from bit_nf4_quantized_10_b200.dp import token_shard, allreduce_adapter_grads, GradBucket
 from oracle import formats as F
 from oracle import lora, nf4
 from synthetic import inputs as S
@@ -121,3 +121,36 @@ def _quant_shard_worker(rank, world, port, n_rows, rows_split):
 @pytest.mark.parametrize("n_rows,rows_split", [(128, [0, 64, 128]), (100, [0, 64, 100])])
 def test_double_quant_sharded_by_rows_gloo(n_rows, rows_split):
     mp.spawn(_quant_shard_worker, args=(2, _free_port(), n_rows, rows_split), nprocs=2, join=True)
+
+
+# ------------------------------------------- one all-reduce for every gradient
+def _bucket_worker(rank, world, port):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        shapes = [(8, 24), (40, 8), (8, 136), (3, 8), (1, 1)]     # ragged sizes: views start 16-byte aligned
+        bucket = GradBucket(shapes)
+        for i, v in enumerate(bucket.views):
+            assert v.shape == shapes[i] and v.data_ptr() % 16 == 0
+            v.copy_(torch.full(shapes[i], float(rank + 1) * (i + 1)))
+        bucket.allreduce()
+        total = sum(r + 1 for r in range(world))
+        for i, v in enumerate(bucket.views):
+            assert torch.equal(v, torch.full(shapes[i], float(total * (i + 1)))), i
+        # the pairwise helper: adjacent views (one collective) and separate tensors (packed copy)
+        pair = GradBucket([(8, 32), (16, 8)])
+        dA, dB = pair.views
+        dA.fill_(rank + 1.0)
+        dB.fill_(2.0 * (rank + 1))
+        allreduce_adapter_grads(dA, dB)
+        assert torch.all(dA == total) and torch.all(dB == 2.0 * total)
+        sA, sB = torch.full((8, 32), rank + 1.0), torch.full((16, 8), 3.0 * (rank + 1))
+        allreduce_adapter_grads(sA, sB)
+        assert torch.all(sA == total) and torch.all(sB == 3.0 * total)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gradient_bucket_single_allreduce_gloo():
+    mp.spawn(_bucket_worker, args=(2, _free_port()), nprocs=2, join=True)
