@@ -1,18 +1,22 @@
 #!/usr/bin/env python
 """Benchmark of the QLoRA NF4 hot path on B200.
 
-One step = one pass of the whole hot path over one batch of synthetic input:
-  nf4_quantize (fp32 W -> NF4 codes + fp32 absmax)
+The measured step is the largest single-GPU workload: the seven linears of a
+70B-shaped decoder layer (q, o 8192 x 8192; k, v 1024 x 8192 (GQA); gate, up
+28672 x 8192; down 8192 x 28672), NF4 + double quant, 2048 tokens, LoRA r = 16,
+alpha = 32.  One step is one pass of the whole hot path over one batch, for
+each linear in turn:
+  nf4_quantize (bf16 W -> NF4 codes + fp32 absmax)
   nf4_double_quant (absmax -> E4M3 codes + group scales + mean)
   qlora_linear_fwd (U = X A^T, Y = X dequant(W)^T + s U B^T; dequant fused)
-  qlora_linear_bwd (V, dB, dX = dY dequant(W) + s V A, dA)
-On the 4096 x 4096 projection with 4096 tokens, r = 16, alpha = 32 (the
-metric's workload).  Throughput counts the GEMM work 4 M N K + 6 M r (K + N)
-per step (dequantization and quantization are not counted as FLOPs).
+  qlora_linear_bwd (V, dX = dY dequant(W) + s V A, dA, dB)
+Throughput counts the GEMM work 4 M N K + 6 M r (K + N) per linear per step
+(dequantization and quantization are not counted as FLOPs).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-Under torchrun (N > 1) every rank runs its own batch (weak scaling) and the
-adapter gradients dA, dB are all-reduced over NCCL each step (the data-parallel
+Under torchrun (N > 1) every rank runs its own batch of 2048 tokens (weak
+scaling) and the adapter gradients of all seven linears, held in one flat
+buffer, are summed over NCCL by one all-reduce per step (the data-parallel
 exchange).  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
@@ -30,24 +34,26 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s & small-M weight GB/s vs B200 roofline"
+WORKLOAD = "layer_70b_linears"
 
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50)
-    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--no-secondary", action="store_true", help="skip the small-M and codec side measurements")
+    p.add_argument("--no-secondary", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    p.add_argument("--leg", choices=["projection", "smallm", "codec"], default="projection",
-                   help="with --profile: which workload to run (the bench line is the projection step)")
+    p.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    p.add_argument("--leg", choices=["layer", "projection", "smallm", "codec"], default="layer",
+                   help="with --profile: which workload to run")
     p.add_argument("--profile", action="store_true",
-                   help="fixed launch sequence for profilers: exactly --warmup then --steps steps, "
+                   help="fixed launch sequence for profilers: exactly --warmup then --steps steps of --leg, "
                         "no clock-sampling warm-up, no e2e, secondary or CPU legs")
     a = p.parse_args()
     if a.profile:
-        a.no_secondary = a.no_cpu = True
+        a.no_secondary = a.no_cpu = a.no_e2e = True
     return a
 
 
@@ -61,21 +67,22 @@ def peaks():
 
 
 def config(world: int) -> dict:
-    return {"workload": "projection 4096x4096 NF4+DQ, 4096 tokens/GPU, r=16, alpha=32: quantize + "
-                        "double quant + fwd + bwd (dX, dA, dB)",
-            "global_batch": 4096 * world, "N": 4096, "K": 4096, "r": 16,
-            "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, untimed)",
+    return {"workload": "70B-shaped decoder layer linears (q, o 8192x8192; k, v 1024x8192; gate, up 28672x8192; "
+                        "down 8192x28672), bf16 weights quantized to NF4 + double quant each step, 2048 tokens/GPU, "
+                        "LoRA r=16 alpha=32 on all seven: quantize + double quant + fwd + bwd (dX, dA, dB)",
+            "global_batch": 2048 * world, "tokens_per_gpu": 2048, "linears": 7, "r": 16,
+            "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, untimed); inputs > L2",
             "outputs": "Y, dX bf16; dA, dB fp32",
             "launch": "stream order" if os.environ.get("QL_PDL", "1") == "0" else "programmatic dependent launch"}
 
 
-def gemm_traffic():
-    """DRAM bytes per launch of the fused GEMM from the committed ncu summary,
-    or None when the kernel source has changed since it was captured."""
+def gemm_traffic(workload: str = WORKLOAD):
+    """Mean DRAM bytes per launch of the fused GEMM on `workload` from the
+    committed ncu capture, or None when the kernel source has changed since."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            d = json.load(f)["qlora_gemm_kernel"]
+            d = json.load(f)["qlora_gemm_kernel"][workload]
         with open(os.path.join(ROOT, "bit_nf4_quantized_10_b200", "csrc", "gemm.cu"), "rb") as f:
             sha = hashlib.sha256(f.read()).hexdigest()
         return float(d["dram_bytes_per_launch"]) if d["gemm_cu_sha256"] == sha else None
@@ -135,55 +142,91 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-# ------------------------------------------------------------ the workload
-class Projection:
-    """The 4096 x 4096 projection workload, resident on one device."""
+# ----------------------------------------------------------- the workloads
+def _lin_flops(M, N, K, r):
+    return 4.0 * M * N * K + 6.0 * M * r * (K + N)
 
-    def __init__(self, q, dev, rank=0):
+
+class LinearSet:
+    """A list of QLoRA linears resident on one device, each with its bf16 (or
+    fp32) master weight, the NF4 + double-quant buffers it is quantized into,
+    its batch (X, dY), adapters and outputs.  The adapter gradients of all the
+    linears live in one flat buffer (GradBucket), so the data-parallel exchange
+    is one all-reduce.  step() runs the whole hot path once."""
+
+    def __init__(self, q, dev, wl, rank=0, w_dtype=None, M=None):
         import torch
         from synthetic import inputs as S
-        self.q, self.dev = q, dev
-        w = S.WORKLOADS["c2"]
-        self.w = w
-        lin = w.linears[0]
-        self.N, self.K, self.M, self.r, self.s = lin.N, lin.K, w.M, w.r, w.s
-        d = S.linear_inputs(w, 0, device=dev)
-        self.W, self.X, self.A, self.B, self.dY = d["W"], d["X"], d["A"], d["B"], d["dY"]
-        if rank:   # a different batch per rank, same weights
-            self.X = S.normal((self.M, self.K), 1.0, 100000 + rank, device=dev, dtype=torch.bfloat16)
-            self.dY = S.normal((self.M, self.N), 1.0, 200000 + rank, device=dev, dtype=torch.bfloat16)
-        self.wq = q.NF4Weight.allocate(self.N, self.K, dev, dq=True)
-        n = self.N * self.K
-        self.absmax = torch.empty(-(-n // 64), dtype=torch.float32, device=dev)
-        self.ws_dq = torch.empty(q.qlora_workspace_size(q.QL_OP_DOUBLE_QUANT, self.absmax.numel()),
-                                 dtype=torch.uint8, device=dev)
-        self.Y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=dev)
-        self.U = torch.empty(self.M, self.r, dtype=torch.bfloat16, device=dev)
-        self.dX = torch.empty(self.M, self.K, dtype=torch.bfloat16, device=dev)
-        self.dA = torch.empty(self.r, self.K, dtype=torch.float32, device=dev)
-        self.dB = torch.empty(self.N, self.r, dtype=torch.float32, device=dev)
-        self.ws = torch.empty(max(q.qlora_workspace_size(q.QL_OP_FWD, self.M, self.N, self.K, self.r),
-                                  q.qlora_workspace_size(q.QL_OP_BWD, self.M, self.N, self.K, self.r)),
-                              dtype=torch.uint8, device=dev)
+        from bit_nf4_quantized_10_b200.dp import GradBucket
+        self.q, self.dev, self.wl = q, dev, wl
+        self.M = wl.M if M is None else M
+        self.r, self.s = wl.r, wl.s
+        M, r = self.M, self.r
+        self.items = []
+        ws = 16
+        for j, lin in enumerate(wl.linears):
+            d = S.linear_inputs(wl, j, M=M, device=dev)
+            W = d["W"] if w_dtype is None else d["W"].to(w_dtype)
+            if rank:     # a different batch per rank, same weights and adapters
+                d["X"] = S.normal((M, lin.K), 1.0, 100000 + 100 * rank + j, device=dev, dtype=torch.bfloat16)
+                d["dY"] = S.normal((M, lin.N), 1.0, 200000 + 100 * rank + j, device=dev, dtype=torch.bfloat16)
+            n = lin.N * lin.K
+            it = dict(N=lin.N, K=lin.K, W=W, X=d["X"], A=d["A"], B=d["B"], dY=d["dY"],
+                      wq=q.NF4Weight.allocate(lin.N, lin.K, dev, dq=True),
+                      absmax=torch.empty(-(-n // 64), dtype=torch.float32, device=dev),
+                      Y=torch.empty(M, lin.N, dtype=torch.bfloat16, device=dev),
+                      U=torch.empty(M, r, dtype=torch.bfloat16, device=dev),
+                      dX=torch.empty(M, lin.K, dtype=torch.bfloat16, device=dev))
+            it["ws_dq"] = torch.empty(q.qlora_workspace_size(q.QL_OP_DOUBLE_QUANT, it["absmax"].numel()),
+                                      dtype=torch.uint8, device=dev)
+            ws = max(ws, q.qlora_workspace_size(q.QL_OP_FWD, M, lin.N, lin.K, r),
+                     q.qlora_workspace_size(q.QL_OP_BWD, M, lin.N, lin.K, r))
+            self.items.append(it)
+            del d
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        shapes = []
+        for it in self.items:
+            shapes += [(r, it["K"]), (it["N"], r)]
+        self.bucket = GradBucket(shapes, device=dev)
+        for i, it in enumerate(self.items):
+            it["dA"], it["dB"] = self.bucket.views[2 * i], self.bucket.views[2 * i + 1]
 
     @property
     def flops(self) -> float:
-        M, N, K, r = self.M, self.N, self.K, self.r
-        return 4.0 * M * N * K + 6.0 * M * r * (K + N)
+        return sum(_lin_flops(self.M, it["N"], it["K"], self.r) for it in self.items)
 
     def gemm_flops(self) -> tuple[float, float]:
-        M, N, K, r = self.M, self.N, self.K, self.r
-        return 2.0 * M * N * K + 2.0 * M * r * N, 2.0 * M * N * K + 2.0 * M * r * K
+        """Algorithmic flop of the forward and backward GEMM launches of one
+        step: 2MNK + 2MrN (forward, main product + adapter K-steps) and
+        2MNK + 2MrK (backward)."""
+        M, r = self.M, self.r
+        f = sum(2.0 * M * it["N"] * it["K"] + 2.0 * M * r * it["N"] for it in self.items)
+        b = sum(2.0 * M * it["N"] * it["K"] + 2.0 * M * r * it["K"] for it in self.items)
+        return f, b
 
-    def step(self, allreduce=None):
-        q = self.q
-        q.nf4_quantize(self.W, self.wq.codes, self.absmax)
-        q.nf4_double_quant(self.absmax, self.wq.absmax_q, self.wq.scale2, self.wq.offset, self.ws_dq)
-        q.qlora_linear_fwd(self.wq, self.X, self.A, self.B, self.r, self.s, self.Y, U_out=self.U, ws=self.ws)
-        q.qlora_linear_bwd(self.wq, self.X, self.dY, self.A, self.B, self.r, self.s, self.U, self.dX, self.dA,
-                           self.dB, ws=self.ws)
+    def step(self, allreduce=False, quantize=True):
+        q, r, s = self.q, self.r, self.s
+        for it in self.items:
+            wq = it["wq"]
+            if quantize:
+                q.nf4_quantize(it["W"], wq.codes, it["absmax"])
+                q.nf4_double_quant(it["absmax"], wq.absmax_q, wq.scale2, wq.offset, it["ws_dq"])
+            q.qlora_linear_fwd(wq, it["X"], it["A"], it["B"], r, s, it["Y"], U_out=it["U"], ws=self.ws)
+            q.qlora_linear_bwd(wq, it["X"], it["dY"], it["A"], it["B"], r, s, it["U"], it["dX"], it["dA"],
+                               it["dB"], ws=self.ws)
         if allreduce:
-            allreduce(self.dA, self.dB)
+            self.bucket.allreduce()
+
+    def inputs(self):
+        """The step's inputs, in a fixed order (the e2e copies)."""
+        out = []
+        for it in self.items:
+            out += [it["W"], it["X"], it["A"], it["B"], it["dY"]]
+        return out
+
+    def outputs(self):
+        out = [it[k] for it in self.items for k in ("Y", "dX")]
+        return out + [self.bucket.buffer]
 
 
 def trace_read(q):
@@ -224,20 +267,44 @@ def trace_enable_kinds(q, names):
     L.qlora_trace_enable_kinds(mask)
 
 
+def gemm_roofline(q, ls, run_steps, n_steps, bf16_peak, peak_src, workload):
+    """Time `n_steps` steps with only the GEMM launches traced: algorithmic
+    flop of those launches / their summed device time, against the bf16 peak."""
+    trace_enable_kinds(q, ("qlora_gemm_fwd", "qlora_gemm_bwd"))
+    run_steps()
+    kern = trace_read(q)
+    trace_enable(q, False)
+    f_fwd, f_bwd = ls.gemm_flops()
+    ms_f, n_f = kern.get("qlora_gemm_fwd", (0.0, 0))
+    ms_b, n_b = kern.get("qlora_gemm_bwd", (0.0, 0))
+    gemm_ms = ms_f + ms_b
+    launches = n_f + n_b
+    per_step = len(ls.items)
+    achieved = (n_steps * (f_fwd + f_bwd)) / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 and n_f == n_b == n_steps * per_step else 0.0
+    return {"bound": "tensor", "kernel": "qlora_gemm (fused NF4 dequant + tcgen05 GEMM + LoRA K-steps)",
+            "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s", "frac": achieved / bf16_peak,
+            "peak_source": f"{peak_src} bf16 burst", "traffic": gemm_traffic(workload),
+            "algorithmic_flop_per_launch": (f_fwd + f_bwd) / (2 * per_step), "launches": launches,
+            "avg_launch_us": gemm_ms / max(launches, 1) * 1e3}
+
+
 # --------------------------------------------------------------- CPU oracle
 _ORACLE_INPUTS = {}
 
 
-def cpu_oracle_sample(rows: int = 256, tokens: int = 256):
-    """The oracle on a bounded sample of the projection step: quantize + double
-    quant + dequant of `rows` weight rows, fwd + bwd for `tokens` tokens."""
-    import numpy as np
+def cpu_oracle_sample(rows: int = 512, tokens: int = 256):
+    """The oracle on a bounded sample of the measured step: linear q of the
+    70B-shaped layer (8192 x 8192): quantize + double quant + dequant of `rows`
+    weight rows, forward + backward for `tokens` tokens."""
+    import torch
     from oracle import lora, nf4
     from synthetic import inputs as S
-    w = S.WORKLOADS["c2"]
-    if "c2" not in _ORACLE_INPUTS:
-        _ORACLE_INPUTS["c2"] = S.linear_inputs(w, 0)
-    d = _ORACLE_INPUTS["c2"]
+    w = S.WORKLOADS["c4"]
+    if "c4q" not in _ORACLE_INPUTS:
+        d = S.linear_inputs(w, 0)
+        d["W"] = d["W"].to(torch.bfloat16)
+        _ORACLE_INPUTS["c4q"] = d
+    d = _ORACLE_INPUTS["c4q"]
     W = d["W"][:rows]
     X, dY = d["X"][:tokens], d["dY"][:tokens, :rows]
     A, B = d["A"], d["B"][:rows]
@@ -249,21 +316,23 @@ def cpu_oracle_sample(rows: int = 256, tokens: int = 256):
     Y, U = lora.forward(X, What, A, B, w.s)
     lora.backward(X, What, A, B, w.s, dY, U=U)
     dt = time.perf_counter() - t0
-    flops = 4.0 * tokens * rows * K + 6.0 * tokens * w.r * (K + rows)
-    return flops, dt, f"weight rows {rows} of 4096 (quantize, double quant, dequant), fwd+bwd on {tokens} of 4096 tokens"
+    return _lin_flops(tokens, rows, K, w.r), dt, (f"linear q (8192x8192) of the 70B-shaped layer: weight rows {rows} "
+                                                 f"of 8192 (quantize, double quant, dequant), fwd+bwd on {tokens} "
+                                                 f"of 2048 tokens")
 
 
 def cpu_baseline_leg(min_s: float = 10.0, max_reps: int = 30) -> dict:
     """The oracle as it stands on the host cores: the same bounded sample of the
-    projection step repeated until at least `min_s` seconds of CPU work."""
+    measured step repeated until at least `min_s` seconds of CPU work."""
     tf, tt, reps, desc = 0.0, 0.0, 0, ""
     while tt < min_s and reps < max_reps:
-        f, t, desc = cpu_oracle_sample(1024, 512)
+        f, t, desc = cpu_oracle_sample()
         tf += f
         tt += t
         reps += 1
-    return {"value": tf / tt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{desc}; {reps} repetitions, {tt:.1f} s"}
+    return {"value": tf / tt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "host_cores": host_cores(),
+            "kind": "oracle", "sample": f"{desc}; {reps} repetitions, {tt:.1f} s (numpy float64: BLAS products on "
+                                        f"{blas_threads()} threads, elementwise steps on one)"}
 
 
 def blas_threads() -> int:
@@ -276,88 +345,104 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-# ---------------------------------------------------------- secondary lines
-def small_m_and_codec(q, dev, hbm_peak):
-    """Small-token forward on the 28672 x 8192 weight (HBM-bound on the packed
-    weight) and the standalone quantize + double quant over 4 Gi bf16 elements."""
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------ end to end
+def e2e_leg(q, dev, wl, flops_of, world, rank, n_steps, allreduce):
+    """The measured step through the public API with host buffers: every step
+    copies its inputs (bf16 weights, X, A, B, dY of the seven linears) in from
+    pinned host memory and its results (Y, dX, dA, dB) back out.  Two device
+    buffer sets and separate copy streams let step i's input copy and step
+    i-1's output copy overlap step i's compute (double buffering, ordered by
+    events).  Also measures the copy-only ceiling of the same bytes."""
     import torch
-    from synthetic import inputs as S
-    out = {}
-    w5 = S.WORKLOADS["c5"]
-    lin = w5.linears[0]
-    N, K, r, s = lin.N, lin.K, w5.r, w5.s
-    W = S.normal((N, K), w5.wstd, S.seed_of(5, 0, "W"), device=dev)
-    wq = q.quantize_weight(W, dq=True)
-    del W
-    A = S.uniform((r, K), 1.0 / K ** 0.5, S.seed_of(5, 0, "A"), device=dev)
-    B = S.normal((N, r), 0.01, S.seed_of(5, 0, "B"), device=dev, dtype=torch.bfloat16)
-    wbytes = q.nf4_storage_bytes(N * K, True)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    for M in w5.Ms:
-        X = S.normal((M, K), 1.0, S.seed_of(5, 0, "X") + M, device=dev, dtype=torch.bfloat16)
-        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(max(16, q.qlora_workspace_size(q.QL_OP_FWD, M, N, K, r)), dtype=torch.uint8, device=dev)
-        for _ in range(3):
-            q.qlora_linear_fwd(wq, X, A, B, r, s, Y, ws=ws)
-        times = []
-        for _ in range(20):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            q.qlora_linear_fwd(wq, X, A, B, r, s, Y, ws=ws)
-            e1.record()
-            torch.cuda.synchronize()
-            times.append(e0.elapsed_time(e1))
-        t = statistics.median(times) / 1e3
-        gbs = wbytes / t / 1e9
-        out[f"M{M}"] = {"us": round(t * 1e6, 2), "weight_GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 3)}
-    # adapter merge of the same weight, bf16 output and re-quantized codes + fp32 constants
-    n5 = N * K
-    W_out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
-    codes_out = torch.empty(n5 // 2, dtype=torch.uint8, device=dev)
-    absmax_out = torch.empty(n5 // 64, dtype=torch.float32, device=dev)
-    t = _time_calls(lambda: q.qlora_merge(wq, A, B, r, s, W_out=W_out, codes_out=codes_out, absmax_out=absmax_out),
-                    flush, n_warm=3, n=10)
-    # read codes + E4M3 constants + scales + A, B; write bf16 W' + codes + fp32 constants
-    moved = n5 // 2 + n5 // 64 + 4 * (n5 // 16384) + 2 * r * (N + K) + 2 * n5 + n5 // 2 + 4 * (n5 // 64)
-    out[f"merge_{N}x{K}_r{r}"] = {"us": round(t * 1e6, 2), "GBps": round(moved / t / 1e9, 1),
-                                 "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3), "bytes": moved,
-                                 "fma_per_element": r}
-    del W_out, codes_out, absmax_out, wq
+    import torch.distributed as dist
+    sets = [LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16) for _ in range(2)]
+    h_in = [torch.empty(t.shape, dtype=t.dtype).pin_memory().copy_(t) for t in sets[0].inputs()]
+    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in sets[0].outputs()]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_comp = torch.cuda.current_stream(dev)
+
+    def run(n):
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_comp = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        for i in range(n):
+            st = sets[i % 2]
+            if i >= 2:
+                s_in.wait_event(ev_comp[i - 2])          # set reused: its last compute read the inputs
+            with torch.cuda.stream(s_in):
+                for d, h in zip(st.inputs(), h_in):
+                    d.copy_(h, non_blocking=True)
+                ev_in[i].record(s_in)
+            s_comp.wait_event(ev_in[i])
+            if i >= 2:
+                s_comp.wait_event(ev_out[i - 2])         # its outputs have been read out
+            st.step(allreduce)
+            ev_comp[i].record(s_comp)
+            s_out.wait_event(ev_comp[i])
+            with torch.cuda.stream(s_out):
+                for h, d in zip(h_out, st.outputs()):
+                    h.copy_(d, non_blocking=True)
+                ev_out[i].record(s_out)
+        s_comp.wait_event(ev_out[n - 1])
+
+    run(3)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_comp)
+    run(n_steps)
+    e1.record(s_comp)
+    torch.cuda.synchronize(dev)
+    t = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        tt = torch.tensor([t], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+
+    # copy-only ceiling: the same bytes each way, no compute
+    def copies(n):
+        for _ in range(n):
+            with torch.cuda.stream(s_in):
+                for d, h in zip(sets[0].inputs(), h_in):
+                    d.copy_(h, non_blocking=True)
+            with torch.cuda.stream(s_out):
+                for h, d in zip(h_out, sets[1].outputs()):
+                    h.copy_(d, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(s_comp)
+    s_in.wait_event(c0)
+    s_out.wait_event(c0)
+    copies(3)
+    ea, eb = torch.cuda.Event(), torch.cuda.Event()
+    ea.record(s_in)
+    eb.record(s_out)
+    s_comp.wait_event(ea)
+    s_comp.wait_event(eb)
+    c1.record(s_comp)
+    torch.cuda.synchronize(dev)
+    t_copy = c0.elapsed_time(c1) / 1e3 / 3
+    fl = flops_of(sets[0])
+    out = {"value": world * n_steps * fl / t / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": n_steps, "ms_per_step": t / n_steps * 1e3,
+           "pipeline": "double-buffered: input copies, compute and output copies on three streams",
+           "copy_only_ms_per_step": t_copy * 1e3, "copy_bound_value": world * fl / t_copy / 1e12}
+    del sets
     torch.cuda.empty_cache()
-    # codec over 4 Gi bf16 elements
-    n = w5.codec_n
-    x = S.codec_tensor(n, 0.02, S.seed_of(5, 9, "W"), device=dev)
-    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
-    absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
-    aq = torch.empty(n // 64, dtype=torch.uint8, device=dev)
-    s2 = torch.empty(-(-n // 64 // 256), dtype=torch.float32, device=dev)
-    mu = torch.empty(1, dtype=torch.float32, device=dev)
-    ws = torch.empty(q.qlora_workspace_size(q.QL_OP_DOUBLE_QUANT, n // 64), dtype=torch.uint8, device=dev)
-    for _ in range(2):
-        q.nf4_quantize(x, codes, absmax)
-        q.nf4_double_quant(absmax, aq, s2, mu, ws)
-    times = []
-    for _ in range(5):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        q.nf4_quantize(x, codes, absmax)
-        q.nf4_double_quant(absmax, aq, s2, mu, ws)
-        e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
-    t = statistics.median(times) / 1e3
-    # bytes that must move: read x, write codes + absmax, read absmax twice (mean, encode), write E4M3 + scales
-    nb = n // 64
-    moved = 2 * n + n // 2 + 4 * nb + 2 * 4 * nb + nb + 4 * (nb // 256)
-    out["codec_4Gi_bf16"] = {"ms": round(t * 1e3, 3), "GBps": round(moved / t / 1e9, 1),
-                             "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3), "bytes": moved}
-    del x, codes, absmax, aq
-    torch.cuda.empty_cache()
-    out.update(large_token_legs(q, dev))
     return out
 
 
+# ---------------------------------------------------------- secondary lines
 def _time_calls(fn, flush, n_warm=2, n=5):
     import torch
     for _ in range(n_warm):
@@ -374,17 +459,42 @@ def _time_calls(fn, flush, n_warm=2, n=5):
     return statistics.median(times) / 1e3
 
 
-def large_token_legs(q, dev):
-    """The other two large-token workloads, forward + backward: the 7B MLP block
-    (gate/up 11008 x 4096, down 4096 x 11008, 8192 tokens, r = 64, SiLU-gated)
-    and the seven 70B-shaped layer linears (2048 tokens, r = 16), each step
-    timed whole with CUDA events; TFLOP/s counts 4MNK + 6Mr(K+N) per linear."""
+def secondary_legs(q, dev, hbm_peak, bf16_peak, peak_src, layer_set):
+    import torch
+    from synthetic import inputs as S
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # the measured layer without the per-step quantization (fwd + bwd only)
+    t = _time_calls(lambda: layer_set.step(quantize=False), flush, n_warm=2, n=10)
+    out["layer_70b_linears_fwd_bwd_only"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(layer_set.flops / t / 1e12, 1)}
+    # the 4096^2 projection: quantize + double quant + fwd + bwd, with its GEMM roofline
+    proj = LinearSet(q, dev, S.WORKLOADS["c2"])
+    t = _time_calls(proj.step, flush, n_warm=3, n=20)
+
+    def proj_steps():
+        for _ in range(10):
+            flush.zero_()
+            proj.step()
+        torch.cuda.synchronize()
+    proj_steps()
+    rf = gemm_roofline(q, proj, proj_steps, 10, bf16_peak, peak_src, "projection_4096")
+    out["projection_4096"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(proj.flops / t / 1e12, 1),
+                              "gemm_avg_launch_us": round(rf["avg_launch_us"], 2), "gemm_frac": round(rf["frac"], 3),
+                              "gemm_traffic": rf["traffic"]}
+    del proj
+    torch.cuda.empty_cache()
+    out.update(mlp_leg(q, dev, flush))
+    out.update(small_m_and_codec(q, dev, hbm_peak, flush))
+    out.update(adamw_leg(q, dev, hbm_peak, layer_set, flush))
+    return out
+
+
+def mlp_leg(q, dev, flush):
+    """The 7B MLP block (gate/up 11008 x 4096, down 4096 x 11008, 8192 tokens,
+    r = 64, SiLU-gated), forward + backward."""
     import torch
     from synthetic import inputs as S
     from bit_nf4_quantized_10_b200.mlp import QLoRAMLP
-    out = {}
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    # 7B MLP
     w3 = S.WORKLOADS["c3"]
     D, H, M, r, s = 4096, 11008, w3.M, w3.r, w3.s
     ws = [q.quantize_weight(S.custom_weight(n, k, w3.wstd, 3000 + i, device=dev), dq=True)
@@ -405,42 +515,106 @@ def large_token_legs(q, dev):
         mlp.backward(X, dy)
 
     t = _time_calls(mlp_step, flush)
-    out["mlp_7b"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(mlp.flops() / t / 1e12, 1),
-                     "tokens": M, "r": r}
+    res = {"mlp_7b": {"ms": round(t * 1e3, 3), "TFLOPs": round(mlp.flops() / t / 1e12, 1), "tokens": M, "r": r}}
     del mlp, ws, X, dy, y
     torch.cuda.empty_cache()
-    # 70B-shaped layer linears
-    w4 = S.WORKLOADS["c4"]
-    M, r, s = w4.M, w4.r, w4.s
-    legs, flops = [], 0.0
-    for j, lin in enumerate(w4.linears):
-        d = S.linear_inputs(w4, j, device=dev)
-        wq = q.quantize_weight(d["W"], dq=True)
-        del d["W"]
-        N, K = lin.N, lin.K
+    return res
+
+
+def small_m_and_codec(q, dev, hbm_peak, flush):
+    """Small-token forward on the 28672 x 8192 weight (HBM-bound on the packed
+    weight), the adapter merge of that weight, and the standalone codecs over
+    4 Gi bf16 elements (NF4 + double quant; NVFP4; MXFP4)."""
+    import torch
+    from synthetic import inputs as S
+    out = {}
+    w5 = S.WORKLOADS["c5"]
+    lin = w5.linears[0]
+    N, K, r, s = lin.N, lin.K, w5.r, w5.s
+    W = S.normal((N, K), w5.wstd, S.seed_of(5, 0, "W"), device=dev)
+    wq = q.quantize_weight(W, dq=True)
+    del W
+    A = S.uniform((r, K), 1.0 / K ** 0.5, S.seed_of(5, 0, "A"), device=dev)
+    B = S.normal((N, r), 0.01, S.seed_of(5, 0, "B"), device=dev, dtype=torch.bfloat16)
+    wbytes = q.nf4_storage_bytes(N * K, True)
+    for M in w5.Ms:
+        X = S.normal((M, K), 1.0, S.seed_of(5, 0, "X") + M, device=dev, dtype=torch.bfloat16)
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        U = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
-        dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-        dA = torch.empty(r, K, dtype=torch.float32, device=dev)
-        dB = torch.empty(N, r, dtype=torch.float32, device=dev)
-        wsb = torch.empty(max(q.qlora_workspace_size(q.QL_OP_FWD, M, N, K, r),
-                              q.qlora_workspace_size(q.QL_OP_BWD, M, N, K, r), 16), dtype=torch.uint8, device=dev)
-        legs.append((wq, d, Y, U, dX, dA, dB, wsb))
-        flops += 4.0 * M * N * K + 6.0 * M * r * (K + N)
+        ws = torch.empty(max(16, q.qlora_workspace_size(q.QL_OP_FWD, M, N, K, r)), dtype=torch.uint8, device=dev)
+        t = _time_calls(lambda: q.qlora_linear_fwd(wq, X, A, B, r, s, Y, ws=ws), flush, n_warm=3, n=20)
+        gbs = wbytes / t / 1e9
+        out[f"M{M}"] = {"us": round(t * 1e6, 2), "weight_GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 3)}
+    # adapter merge, bf16 output and re-quantized codes + fp32 constants
+    n5 = N * K
+    W_out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    codes_out = torch.empty(n5 // 2, dtype=torch.uint8, device=dev)
+    absmax_out = torch.empty(n5 // 64, dtype=torch.float32, device=dev)
+    t = _time_calls(lambda: q.qlora_merge(wq, A, B, r, s, W_out=W_out, codes_out=codes_out, absmax_out=absmax_out),
+                    flush, n_warm=3, n=10)
+    moved = n5 // 2 + n5 // 64 + 4 * (n5 // 16384) + 2 * r * (N + K) + 2 * n5 + n5 // 2 + 4 * (n5 // 64)
+    out[f"merge_{N}x{K}_r{r}"] = {"us": round(t * 1e6, 2), "GBps": round(moved / t / 1e9, 1),
+                                 "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3), "bytes": moved,
+                                 "fma_per_element": r}
+    del W_out, codes_out, absmax_out, wq
+    torch.cuda.empty_cache()
+    # codecs over 4 Gi bf16 elements
+    n = w5.codec_n
+    x = S.codec_tensor(n, 0.02, S.seed_of(5, 9, "W"), device=dev)
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+    aq = torch.empty(n // 64, dtype=torch.uint8, device=dev)
+    s2 = torch.empty(-(-n // 64 // 256), dtype=torch.float32, device=dev)
+    mu = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(q.qlora_workspace_size(q.QL_OP_DOUBLE_QUANT, n // 64), dtype=torch.uint8, device=dev)
 
-    def layer_step():
-        for wq, d, Y, U, dX, dA, dB, wsb in legs:
-            q.qlora_linear_fwd(wq, d["X"], d["A"], d["B"], r, s, Y, U_out=U, ws=wsb)
-            q.qlora_linear_bwd(wq, d["X"], d["dY"], d["A"], d["B"], r, s, U, dX, dA, dB, ws=wsb)
-
-    t = _time_calls(layer_step, flush)
-    out["layer_70b_linears"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(flops / t / 1e12, 1), "tokens": M, "r": r}
+    def nf4_codec():
+        q.nf4_quantize(x, codes, absmax)
+        q.nf4_double_quant(absmax, aq, s2, mu, ws)
+    t = _time_calls(nf4_codec, flush, n_warm=2, n=5)
+    nb = n // 64
+    # read x, write codes + absmax, read absmax twice (mean, encode), write E4M3 + scales
+    moved = 2 * n + n // 2 + 4 * nb + 2 * 4 * nb + nb + 4 * (nb // 256)
+    out["codec_4Gi_bf16"] = {"ms": round(t * 1e3, 3), "GBps": round(moved / t / 1e9, 1),
+                             "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3), "bytes": moved}
+    del absmax, aq
+    sc = torch.empty(n // 16, dtype=torch.uint8, device=dev)
+    ts = torch.empty(4, dtype=torch.float32, device=dev)
+    wsn = torch.empty(256, dtype=torch.uint8, device=dev)
+    t = _time_calls(lambda: q.nvfp4_quantize(x, codes, sc, ts, wsn), flush, n_warm=2, n=5)
+    moved = 2 * 2 * n + n // 2 + n // 16         # x read twice (tensor maximum, then codes)
+    out["nvfp4_4Gi_bf16"] = {"ms": round(t * 1e3, 3), "GBps": round(moved / t / 1e9, 1),
+                             "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3), "bytes": moved}
+    t = _time_calls(lambda: q.mxfp4_quantize(x, codes, sc[: n // 32]), flush, n_warm=2, n=5)
+    moved = 2 * n + n // 2 + n // 32
+    out["mxfp4_4Gi_bf16"] = {"ms": round(t * 1e3, 3), "GBps": round(moved / t / 1e9, 1),
+                             "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3), "bytes": moved}
     st = q.qlora_get_status()
     if st != q.QL_OK:
-        raise RuntimeError(f"device status after the large-token legs: {q.status_string(st)}")
-    del legs
+        raise RuntimeError(f"device status after the codec legs: {q.status_string(st)}")
+    del x, codes, sc
     torch.cuda.empty_cache()
     return out
+
+
+def adamw_leg(q, dev, hbm_peak, layer_set, flush):
+    """One fused AdamW step over every adapter parameter of the measured layer
+    (fp32 parameters and states in device memory; gradients from the bucket)."""
+    import torch
+    g = layer_set.bucket.buffer
+    n = g.numel()
+    p = torch.randn(n, device=dev) * 0.01
+    m = torch.zeros(n, device=dev)
+    v = torch.zeros(n, device=dev)
+    pb = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    step = [0]
+
+    def upd():
+        step[0] += 1
+        q.qlora_adamw_step(p, g, m, v, n, step[0], 2e-4, weight_decay=0.01, p_bf16=pb)
+    t = _time_calls(upd, flush, n_warm=3, n=20)
+    moved = n * (4 * 4 + 3 * 4 + 2)
+    return {"adamw_adapters_70b_layer": {"us": round(t * 1e6, 2), "params": n, "GBps": round(moved / t / 1e9, 1),
+                                         "frac_hbm": round(moved / t / 1e9 / hbm_peak, 3)}}
 
 
 # ------------------------------------------------------------------- arms
@@ -453,7 +627,7 @@ def run_reference(args, rank):
     total_f, total_t = 0.0, 0.0
     desc = ""
     for _ in range(args.steps):
-        f, t, desc = cpu_oracle_sample(1024, 512)
+        f, t, desc = cpu_oracle_sample()
         total_f += f
         total_t += t
     v = total_f / total_t / 1e12
@@ -462,19 +636,25 @@ def run_reference(args, rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": config(max(1, args.gpus)),
-            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "host_cores": host_cores(),
+                             "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 def profile_leg(args, q, dev):
-    """A fixed launch sequence of one secondary workload for profilers:
-    smallm = the 16-token forward on the 28672 x 8192 weight; codec = quantize
-    + double quant of 256 Mi bf16 elements.  Prints per-call device times."""
+    """A fixed launch sequence of one workload for profilers: layer = the
+    measured step; projection = the 4096^2 step; smallm = the 16-token forward
+    on the 28672 x 8192 weight; codec = quantize + double quant of 256 Mi bf16
+    elements.  Prints per-call device times."""
     import torch
     from synthetic import inputs as S
     w5 = S.WORKLOADS["c5"]
-    if args.leg == "smallm":
+    if args.leg in ("layer", "projection"):
+        ls = LinearSet(q, dev, S.WORKLOADS["c4" if args.leg == "layer" else "c2"],
+                       w_dtype=torch.bfloat16 if args.leg == "layer" else None)
+        call = ls.step
+    elif args.leg == "smallm":
         lin = w5.linears[0]
         N, K, r, s, M = lin.N, lin.K, w5.r, w5.s, 16
         W = S.normal((N, K), w5.wstd, S.seed_of(5, 0, "W"), device=dev)
@@ -521,31 +701,30 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     import bit_nf4_quantized_10_b200 as q
+    from synthetic import inputs as S
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    if args.profile and args.leg != "projection":
+    if args.profile:
         profile_leg(args, q, dev)
         return
     hbm_peak, bf16_peak, bf16_sus, peak_src = peaks()
-    wl = Projection(q, dev, rank)
-    allreduce = None
-    if world > 1:
-        from bit_nf4_quantized_10_b200.dp import allreduce_adapter_grads
-        allreduce = allreduce_adapter_grads
+    wl = S.WORKLOADS["c4"]
+    ls = LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16)
+    allreduce = world > 1
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2 (126 MB)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
     t_warm = time.time()
     for _ in range(args.warmup):
-        wl.step(allreduce)
+        ls.step(allreduce)
     torch.cuda.synchronize()
     # clock samples under load: a wall-clock bound, so the step count differs
     # between ranks; these steps therefore skip the collective (every rank must
     # issue the same all-reduces in the same order)
-    while not args.profile and time.time() - t_warm < 0.5:
-        wl.step(None)
+    while time.time() - t_warm < 0.5:
+        ls.step(False)
         torch.cuda.synchronize()
     st = q.qlora_get_status()
     if st != q.QL_OK:
@@ -554,18 +733,15 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    trace_enable_kinds(q, ("qlora_gemm_fwd", "qlora_gemm_bwd"))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record()
-        wl.step(allreduce)
+        ls.step(allreduce)
         ev[i][1].record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    kern = trace_read(q)
-    trace_enable(q, False)
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_s = sum(step_ms) / 1e3
@@ -576,80 +752,40 @@ def run_ours(args, rank, world, local_rank):
     st = q.qlora_get_status()
     if st != q.QL_OK:
         raise RuntimeError(f"device status after timing: {q.status_string(st)}")
-    value = world * args.steps * wl.flops / total_s / 1e12
+    value = world * args.steps * ls.flops / total_s / 1e12
 
-    # dominant kernel: the fused dequant GEMM (forward and backward launches)
-    f_fwd, f_bwd = wl.gemm_flops()
-    ms_f, n_f = kern.get("qlora_gemm_fwd", (0.0, 0))
-    ms_b, n_b = kern.get("qlora_gemm_bwd", (0.0, 0))
-    gemm_ms = ms_f + ms_b
-    gemm_launches = n_f + n_b
-    achieved = (n_f * f_fwd + n_b * f_bwd) / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
+    # dominant kernel: the fused dequant GEMM, its launches timed by events on
+    # the launching stream over the same number of steps (only its kind traced)
+    n_rf = args.steps
 
-    # per-kernel breakdown: the same steps again (untimed) with every kind traced
+    def rf_steps():
+        for _ in range(n_rf):
+            flush.zero_()
+            ls.step(allreduce)
+        torch.cuda.synchronize()
+    roofline = gemm_roofline(q, ls, rf_steps, n_rf, bf16_peak, peak_src, WORKLOAD)
+
+    # per-kernel breakdown: more steps (untimed) with every kind traced
     trace_enable(q, True)
-    n_br = min(args.steps, 10)
+    n_br = min(args.steps, 5)
     for _ in range(n_br):
         flush.zero_()
-        wl.step(allreduce)
+        ls.step(allreduce)
     torch.cuda.synchronize()
     breakdown = trace_read(q)
     trace_enable(q, False)
     launches_per_step = sum(c for _, c in breakdown.values()) / n_br
     gpu_launches = int(round(launches_per_step * args.steps))
 
-    # end to end through the public API with pinned host buffers
     e2e = None
-    if not args.profile:
-        hW = torch.empty_like(wl.W, device="cpu").pin_memory().copy_(wl.W)
-        hX = torch.empty_like(wl.X, device="cpu").pin_memory().copy_(wl.X)
-        hA = torch.empty_like(wl.A, device="cpu").pin_memory().copy_(wl.A)
-        hB = torch.empty_like(wl.B, device="cpu").pin_memory().copy_(wl.B)
-        hdY = torch.empty_like(wl.dY, device="cpu").pin_memory().copy_(wl.dY)
-        oY = torch.empty_like(wl.Y, device="cpu").pin_memory()
-        odX = torch.empty_like(wl.dX, device="cpu").pin_memory()
-        odA = torch.empty_like(wl.dA, device="cpu").pin_memory()
-        odB = torch.empty_like(wl.dB, device="cpu").pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (hW, hX, hA, hB, hdY))
-        d2h = sum(t.numel() * t.element_size() for t in (oY, odX, odA, odB))
-
-        def e2e_step():
-            wl.W.copy_(hW, non_blocking=True)
-            wl.X.copy_(hX, non_blocking=True)
-            wl.A.copy_(hA, non_blocking=True)
-            wl.B.copy_(hB, non_blocking=True)
-            wl.dY.copy_(hdY, non_blocking=True)
-            wl.step(allreduce)
-            oY.copy_(wl.Y, non_blocking=True)
-            odX.copy_(wl.dX, non_blocking=True)
-            odA.copy_(wl.dA, non_blocking=True)
-            odB.copy_(wl.dB, non_blocking=True)
-
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_e2e = max(5, args.steps // 2)
-        e0.record()
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record()
-        torch.cuda.synchronize()
-        t_e2e = e0.elapsed_time(e1) / 1e3
-        if world > 1:
-            tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            t_e2e = float(tt.item())
-        e2e = {"value": world * n_e2e * wl.flops / t_e2e / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+    if not args.no_e2e:
+        e2e = e2e_leg(q, dev, wl, lambda s: s.flops, world, rank, max(5, args.steps // 3), allreduce)
 
     secondary = None
     if rank == 0 and not args.no_secondary:
         del flush
         torch.cuda.empty_cache()
-        secondary = small_m_and_codec(q, dev, hbm_peak)
+        secondary = secondary_legs(q, dev, hbm_peak, bf16_peak, peak_src, ls)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -661,12 +797,9 @@ def run_ours(args, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config(world),
-            "roofline": {"bound": "tensor", "kernel": "qlora_gemm (fused NF4 dequant + tcgen05 GEMM + LoRA)",
-                         "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
-                         "frac": achieved / bf16_peak, "peak_source": f"{peak_src} bf16 burst",
-                         "traffic": gemm_traffic(), "launches": gemm_launches,
-                         "avg_launch_us": gemm_ms / max(gemm_launches, 1) * 1e3},
-            "kernels": {k: {"us_per_launch": round(v[0] / v[1] * 1e3, 2), "launches_per_step": v[1] / n_br}
+            "roofline": roofline,
+            "kernels": {k: {"us_per_launch": round(v[0] / v[1] * 1e3, 2), "launches_per_step": v[1] / n_br,
+                            "ms_per_step": round(v[0] / n_br, 4)}
                         for k, v in breakdown.items()},
             "gpu_launches": gpu_launches,
             "cpu_baseline": cpu,

@@ -22,9 +22,18 @@ def test_peaks_measured_and_fallback(tmp_path, monkeypatch):
 def test_config_is_weak_scaling():
     for world in (1, 2, 8):
         c = bench.config(world)
-        assert c["global_batch"] == 4096 * world
+        assert c["global_batch"] == 2048 * world
         assert c["parallelism"] == f"dp{world}"
-        assert (c["N"], c["K"], c["r"]) == (4096, 4096, 16)
+        assert (c["tokens_per_gpu"], c["linears"], c["r"]) == (2048, 7, 16)
+
+
+def test_measured_step_flops_match_the_workload():
+    """The layer's FLOP count per step: sum over the seven linears of
+    4 M N K + 6 M r (K + N) (7,041.2 GFLOP at 2048 tokens, r = 16)."""
+    from synthetic import inputs as S
+    w = S.WORKLOADS["c4"]
+    tot = sum(bench._lin_flops(w.M, l.N, l.K, w.r) for l in w.linears)
+    assert abs(tot / 1e9 - 7041.2) < 0.1
 
 
 def _fake_tree(tmp_path, src: bytes, recorded_sha: str):
@@ -34,7 +43,7 @@ def _fake_tree(tmp_path, src: bytes, recorded_sha: str):
     prof = tmp_path / "profiles"
     prof.mkdir()
     (prof / "traffic.json").write_text(json.dumps(
-        {"qlora_gemm_kernel": {"dram_bytes_per_launch": 45117440, "gemm_cu_sha256": recorded_sha}}))
+        {"qlora_gemm_kernel": {bench.WORKLOAD: {"dram_bytes_per_launch": 45117440, "gemm_cu_sha256": recorded_sha}}}))
 
 
 def test_gemm_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
@@ -53,5 +62,5 @@ def test_gemm_traffic_missing_file(tmp_path, monkeypatch):
 
 @pytest.mark.skipif(not os.path.exists(os.path.join(bench.ROOT, "profiles", "traffic.json")), reason="no capture")
 def test_committed_traffic_record_is_well_formed():
-    d = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))["qlora_gemm_kernel"]
-    assert d["dram_bytes_per_launch"] > 0 and len(d["gemm_cu_sha256"]) == 64
+    for d in json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))["qlora_gemm_kernel"].values():
+        assert d["dram_bytes_per_launch"] > 0 and len(d["gemm_cu_sha256"]) == 64
