@@ -72,14 +72,24 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// {c, c} in one 64-bit register, the multiplier of a packed product.
+__device__ __forceinline__ uint64_t pack_cc(float c) {
+  uint64_t cc;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c));
+  return cc;
+}
+
 // Two codes (the low and high nibble of byte b of `w`) -> bf16x2 of
 // bf16(fl32(q * c)), the low code in the low half.  e4 / o4 hold 4 * low / high
 // nibble of each byte; the level table's low address byte is replaced by it.
-__device__ __forceinline__ uint32_t expand_pair(uint32_t e4, uint32_t o4, uint32_t qbase, uint32_t sel, float c) {
+// cc = {c, c}: one packed instruction takes both fp32 products.
+__device__ __forceinline__ uint32_t expand_pair(uint32_t e4, uint32_t o4, uint32_t qbase, uint32_t sel, uint64_t cc) {
   const float lo = lds_f32_const(__byte_perm(e4, qbase, sel));
   const float hi = lds_f32_const(__byte_perm(o4, qbase, sel));
   float pl, ph;
-  mul2_rn(lo, hi, c, pl, ph);
+  asm("{\n .reg .b64 x, z;\n mov.b64 x, {%2, %3};\n mul.rn.f32x2 z, x, %4;\n mov.b64 {%0, %1}, z;\n}"
+      : "=f"(pl), "=f"(ph)
+      : "f"(lo), "f"(hi), "l"(cc));
   return pack_bf16x2(pl, ph);
 }
 
@@ -95,45 +105,41 @@ __device__ __forceinline__ void load_codes(const Params& p, int row, int kb0, in
   }
 }
 
-// Raw block constants of one row's blocks: the E4M3 byte (or the fp32 bits of
-// a plain constant) per block, and the group scales s_2 of the first and the
-// last block (blocks of a row chunk span at most two groups of 256).  Only
-// loads here: the decode waits until the row block is expanded, so the loads
-// of the next row block stay in flight while this one computes.
+// Raw block constant of one row's block kb0 + tq (thread tq of each quad takes
+// one block of the warp's chunk, so each constant is loaded and decoded once per
+// quad and handed to the other three by shuffles): the E4M3 byte, or the fp32
+// bits of a plain constant, and its group scale s_2.  Only loads here: the
+// decode waits until the row block is expanded, so the loads of the next row
+// block stay in flight while this one computes.
 template <int KV>
-__device__ __forceinline__ void load_consts(const Params& p, int row, int kb0, int nbw, uint32_t (&q)[KV / 64],
-                                            float (&s2)[2]) {
-  s2[0] = s2[1] = 0.0f;
-#pragma unroll
-  for (int j = 0; j < KV / 64; ++j) {
-    q[j] = 0u;
-    if (row < p.N && j < nbw) {
-      const int64_t b = (int64_t)row * p.kb + kb0 + j;
-      q[j] = p.wc.absmax ? __float_as_uint(__ldg(p.wc.absmax + b)) : (uint32_t)__ldg(p.wc.absmax_q + b);
+__device__ __forceinline__ void load_const(const Params& p, int row, int kb0, int nbw, int tq, uint32_t& q,
+                                           float& s2) {
+  q = 0u;
+  s2 = 0.0f;
+  if (row < p.N && tq < nbw && tq < KV / 64) {
+    const int64_t b = (int64_t)row * p.kb + kb0 + tq;
+    if (p.wc.absmax) {
+      q = __float_as_uint(__ldg(p.wc.absmax + b));
+    } else {
+      q = (uint32_t)__ldg(p.wc.absmax_q + b);
+      s2 = __ldg(p.wc.scale2 + (b >> 8));
     }
   }
-  if (!p.wc.absmax && row < p.N && nbw > 0) {
-    const int64_t b0 = (int64_t)row * p.kb + kb0;
-    s2[0] = __ldg(p.wc.scale2 + (b0 >> 8));
-    s2[1] = __ldg(p.wc.scale2 + ((b0 + nbw - 1) >> 8));
-  }
 }
 
-// The reconstructed constant of block j of a row chunk starting at block b0:
 // c_hat = fl32(fl32(E4M3(q) s_2) + mu) (double quant) or the plain fp32 value.
-__device__ __forceinline__ float decode_const(const WeightConsts& wc, uint32_t q, const float (&s2)[2], int64_t b0,
-                                              int j, float mu) {
+__device__ __forceinline__ float decode_const(const WeightConsts& wc, uint32_t q, float s2, float mu) {
   if (wc.absmax) return __uint_as_float(q);
-  const float s = ((b0 + j) >> 8) == (b0 >> 8) ? s2[0] : s2[1];
-  return __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)q), s), mu);
+  return __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)q), s2), mu);
 }
 
-// Per row block of 16 T rows: the codes and raw constants a thread expands.
+// Per row block of 16 T rows: the codes a thread expands and the raw constant
+// of its quad index's block for each of its rows.
 template <int NT, int KV, int T>
 struct Frag {
   uint2 w[T][2][KV / 64];     // [tile][row g / g+8][block]
-  uint32_t q[T][2][KV / 64];
-  float s2[T][2][2];
+  uint32_t q[T][2];
+  float s2[T][2];
 };
 
 template <int NT, int KV, int T>
@@ -145,29 +151,35 @@ __device__ __forceinline__ void load_frag(const Params& p, int rb, int kb0, int 
     for (int h = 0; h < 2; ++h) {
       const int row = rb * 16 * T + 16 * t + g + 8 * h;
       load_codes<KV>(p, row, kb0, nbw, tq, f.w[t][h]);
-      load_consts<KV>(p, row, kb0, nbw, f.q[t][h], f.s2[t][h]);
+      load_const<KV>(p, row, kb0, nbw, tq, f.q[t][h], f.s2[t][h]);
     }
   }
 }
 
 template <int NT, int KV, int T>
-__device__ __forceinline__ void compute_frag(const Params& p, const Frag<NT, KV, T>& f, int rb, int kb0, float mu,
-                                             const uint32_t (&xb)[KV / 16][NT][2], uint32_t qbase, int nbw,
-                                             int g, float (&acc)[T][NT][4]) {
+__device__ __forceinline__ void compute_frag(const Params& p, const Frag<NT, KV, T>& f, float mu,
+                                             const uint32_t (&xb)[KV / 16][NT][2], uint32_t qbase, int nbw, int g,
+                                             float (&acc)[T][NT][4]) {
 #pragma unroll
   for (int t = 0; t < T; ++t)
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[t][n][i] = 0.0f;
+  // this thread's decoded constants (its quad index's block, rows g and g+8)
+  float cmine[T][2];
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) cmine[t][h] = decode_const(p.wc, f.q[t][h], f.s2[t][h], mu);
 #pragma unroll
   for (int j = 0; j < KV / 64; ++j) {
     if (j < nbw) {
 #pragma unroll
       for (int t = 0; t < T; ++t) {
-        const int row = rb * 16 * T + 16 * t + g;
-        const float cg = decode_const(p.wc, f.q[t][0][j], f.s2[t][0], (int64_t)row * p.kb + kb0, j, mu);
-        const float c8 = decode_const(p.wc, f.q[t][1][j], f.s2[t][1], (int64_t)(row + 8) * p.kb + kb0, j, mu);
+        // block j's constants come from quad lane j (all lanes take part)
+        const uint64_t cg = pack_cc(__shfl_sync(0xffffffffu, cmine[t][0], 4 * g + j));
+        const uint64_t c8 = pack_cc(__shfl_sync(0xffffffffu, cmine[t][1], 4 * g + j));
 #pragma unroll
         for (int half = 0; half < 2; ++half) {        // word .x: k-steps 0, 1; word .y: k-steps 2, 3
           const uint32_t wg = half ? f.w[t][0][j].y : f.w[t][0][j].x;
@@ -254,10 +266,10 @@ __global__ void __launch_bounds__(THREADS, 1) smallm_kernel(Params p) {
     float acc[T][NT][4];
     if ((it & 1) == 0) {
       if (nxt < p.row_blocks) load_frag<NT, KV, T>(p, nxt, kb0, nbw, g, tq, f[1]);
-      compute_frag<NT, KV, T>(p, f[0], rb, kb0, mu, xb, qbase, nbw, g, acc);
+      compute_frag<NT, KV, T>(p, f[0], mu, xb, qbase, nbw, g, acc);
     } else {
       if (nxt < p.row_blocks) load_frag<NT, KV, T>(p, nxt, kb0, nbw, g, tq, f[0]);
-      compute_frag<NT, KV, T>(p, f[1], rb, kb0, mu, xb, qbase, nbw, g, acc);
+      compute_frag<NT, KV, T>(p, f[1], mu, xb, qbase, nbw, g, acc);
     }
     float* rbuf = red_dyn + (it & 1) * red_floats<NT, T>();
     stash<NT, T>(rbuf, acc, warp, g, tq);

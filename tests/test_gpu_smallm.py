@@ -1,8 +1,9 @@
-"""GPU parity of the small-token forward (M <= 16 tokens: the split-K cluster
-kernel) against the oracle, on shapes that exercise its tiling: ragged N,
-K slices that are not whole code stages, a short last slice, several weight
-tiles per cluster (double-buffered accumulators), no adapter and rank 64,
-both constant forms and both output types."""
+"""GPU parity of the small-token forward (M <= 16 tokens) against the oracle,
+on shapes that exercise its tiling: ragged N (a partial last 16-row block),
+K ranges that end inside a warp's chunk, several K parts (one part is 4096
+reduction elements for up to 8 tokens, 2048 above), token counts on both sides
+of the 8-token tile, no adapter and rank 64, both constant forms and both
+output types."""
 import numpy as np
 import pytest
 import torch
@@ -15,10 +16,12 @@ pytestmark = pytest.mark.gpu
 
 CASES = [
     # N, K, M, r, s
-    (5120, 1408, 16, 16, 2.0),     # 22 K-blocks: 8 slices of 3 (last 1); 40 tiles, several per cluster
-    (1000, 1344, 1, 64, 0.25),     # 21 K-blocks: 7 slices of 3; ragged N; one token; rank 64
-    (2056, 4096, 7, 0, 1.0),       # no adapter; odd token count; N = 8 mod 16
-    (384, 192, 4, 8, 0.5),         # 3 K-blocks: a 3-CTA cluster, one sub-step per slice
+    (5120, 1408, 16, 16, 2.0),     # two token tiles; 11 warp chunks of 128 in one part, 5 warps idle
+    (1000, 1344, 1, 64, 0.25),     # one token; a last chunk of one block; N = 8 mod 16; rank 64
+    (2056, 4096, 7, 0, 1.0),       # no adapter; odd token count; exactly one part
+    (384, 192, 4, 8, 0.5),         # one warp chunk of 3 blocks; rank 8 (half an adapter tile)
+    (1024, 9216, 9, 16, 2.0),      # 9 tokens (two tiles, one nearly empty); 5 parts, the last one half
+    (264, 8256, 8, 32, 1.0),       # 8 tokens (one tile); 3 parts, the last one a single block
 ]
 
 
