@@ -38,6 +38,8 @@ ql_status launch_grad_b(const void* dY, int64_t M, int N, const void* Ut, int64_
 ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t ld_vt, int r, float s, void* dA,
                         ql_dtype dt, cudaStream_t st);
 ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st);
+ql_status launch_transpose2(const void* src0, int64_t rows0, int cols0, void* dst0, int64_t ld0, const void* src1,
+                            int64_t rows1, int cols1, void* dst1, int64_t ld1, cudaStream_t st);
 // smallm.cu
 bool smallm_supported(int64_t N, int64_t K);
 size_t smallm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
@@ -252,12 +254,12 @@ ql_status qlora_linear_bwd(const ql_nf4_weight* w, const void* X, const void* dY
   void* Ut = wp + L.ut;
   void* V = wp + L.v;
   void* Vt = wp + L.vt;
-  st = ql::launch_transpose(B, N, r, Bt, N, cs);                              // B^T [r, N]
-  if (st != QL_OK) return st;
   if (!U) {
+    st = ql::launch_transpose(B, N, r, Bt, N, cs);                            // B^T [r, N]
+    if (st != QL_OK) return st;
     st = ql::launch_proj(X, M, K, A, K, r, nullptr, Ut, Mp, cs);     // U^T = bf16(X A^T)^T
   } else {
-    st = ql::launch_transpose(U, M, r, Ut, Mp, cs);                          // U^T [r, Mp]
+    st = ql::launch_transpose2(B, N, r, Bt, N, U, M, r, Ut, Mp, cs);          // B^T [r, N] and U^T [r, Mp]
   }
   if (st != QL_OK) return st;
   st = ql::launch_proj(dY, M, N, Bt, N, r, V, Vt, Mp, cs);          // V = bf16(dY B), and V^T

@@ -11,6 +11,8 @@
 // All kernels are HBM-bound streaming passes.  Loads and stores are 16 bytes
 // wide, grids are sized to a multiple of the SM count and loop grid-stride,
 // and every index is 64-bit so tensors above 2^32 elements work.
+#include <algorithm>
+
 #include "common.cuh"
 #include "trace.cuh"
 
@@ -137,6 +139,21 @@ __device__ __forceinline__ void unpack8(const Raw8<__nv_bfloat16>& r, float (&v)
   }
 }
 
+// The largest |x| bit pattern of eight elements, as fp32 bits: for bf16 input
+// the maximum is taken on the packed halves (the sign bits cleared, two 16-bit
+// maxima per instruction) before unpacking.
+__device__ __forceinline__ uint32_t raw_absmax_bits(const Raw8<float>& r) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = max(m, r.w[i] & 0x7FFFFFFFu);
+  return m;
+}
+__device__ __forceinline__ uint32_t raw_absmax_bits(const Raw8<__nv_bfloat16>& r) {
+  uint32_t m = __vmaxu2(r.w[0] & 0x7FFF7FFFu, r.w[1] & 0x7FFF7FFFu);
+  m = __vmaxu2(m, __vmaxu2(r.w[2] & 0x7FFF7FFFu, r.w[3] & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16) << 16;
+}
+
 // 8 threads per 64-block, 8 consecutive elements per thread.  The loop runs
 // over blocks, so the 8 threads of a block always iterate together and can
 // reduce the absmax with shuffles.  The absmax is the integer maximum of the
@@ -166,11 +183,10 @@ __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, 
     const int64_t b = wb + bq;
     const int64_t e0 = b * 64 + lane8 * 8;   // >= n for a block past the end
     float v[8];
+    const uint32_t abits0 = raw_absmax_bits(nxt);
     unpack8(nxt, v);
     if (wb + warps_per_grid * 4 < nb) load8<T>(x, (wb + warps_per_grid * 4 + bq) * 64 + lane8 * 8, n, nxt);
-    uint32_t abits = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) abits = max(abits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+    uint32_t abits = abits0;
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
     if (abits >= 0x7F800000u && lane8 == 0 && b < nb) raise_status(ST_NONFINITE);
@@ -334,10 +350,26 @@ __global__ void __launch_bounds__(256) dequant_f32_kernel(const uint8_t* __restr
 // bf16 values is exact in fp32, so each fma is the rounded fp32 sum.
 // Optionally the merged values are quantized again (same code selection as
 // quantize_kernel), without a round trip of the bf16 weight through HBM.
-// Layout as in quantize_kernel: 8 threads per 64-block, 8 consecutive elements
-// each, a warp's four blocks iterate together.  K % 64 == 0, so a block lies in
-// one row and its A columns are 16-byte aligned.
-__global__ void __launch_bounds__(256) merge_kernel(const uint8_t* __restrict__ codes, WeightConsts wc, int64_t N,
+// The rank-r product d = B A is a small matrix product, so each thread owns a
+// register tile of 8 rows x 8 consecutive columns of a 64-row x 256-column CTA
+// tile and accumulates its 64 sums with packed fp32 FMAs (two independent
+// IEEE fmas per instruction, j in order), reading A (as fp32) and B (as
+// broadcast pairs) from shared memory staged once per tile: every A and B
+// value is reused by 8 rows or 8 columns.  The 8 threads holding a row's
+// 64-block are 8 consecutive lanes, so the re-quantization's absmax is the same
+// 8-lane shuffle as in quantize_kernel.  K % 64 == 0, so a block lies in one
+// row and a tile edge never splits one.
+constexpr int MG_ROWS = 64;     // rows per CTA tile: 8 warps x 8 rows
+constexpr int MG_COLS = 256;    // columns per CTA tile: 32 lanes x 8 columns
+
+__device__ __forceinline__ void fma2_rn(float2& d, float2 a, float2 b) {
+  asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n mov.b64 z, {%0, %1};\n"
+      " fma.rn.f32x2 z, x, y, z;\n mov.b64 {%0, %1}, z;\n}"
+      : "+f"(d.x), "+f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+}
+
+__global__ void __launch_bounds__(256, 2) merge_kernel(const uint8_t* __restrict__ codes, WeightConsts wc, int64_t N,
                                                     int64_t K, const __nv_bfloat16* __restrict__ A,
                                                     const __nv_bfloat16* __restrict__ B, int r, float s,
                                                     __nv_bfloat16* __restrict__ out, uint8_t* __restrict__ codes_out,
@@ -346,63 +378,111 @@ __global__ void __launch_bounds__(256) merge_kernel(const uint8_t* __restrict__ 
   pdl_trigger();
   __shared__ uint2 bins[64];
   __shared__ float q[16];
+  extern __shared__ __align__(16) float mg_smem[];
+  float* a_s = mg_smem;                                               // [r][256] fp32
+  float2* b_s = reinterpret_cast<float2*>(mg_smem + (size_t)r * MG_COLS);   // [r][64] (b, b)
   if (threadIdx.x < 64) bins[threadIdx.x] = make_uint2(__float_as_uint(bins_in.m[threadIdx.x]), bins_in.base[threadIdx.x]);
   if (threadIdx.x < 16) q[threadIdx.x] = tab.q[threadIdx.x];
-  __syncthreads();
-  const int64_t nb = N * K / 64;
   const float mu = wc.absmax ? 0.0f : *wc.offset;
-  const int lane8 = threadIdx.x & 7;
-  const int wib = threadIdx.x >> 5;
-  const int bq = (threadIdx.x >> 3) & 3;
-  const int64_t warps_per_grid = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t wb = ((int64_t)blockIdx.x * (blockDim.x >> 5) + wib) * 4; wb < nb; wb += warps_per_grid * 4) {
-    const int64_t b = wb + bq;
-    const bool live = b < nb;
-    const int64_t e0 = b * 64 + lane8 * 8;
-    float v[8];
-    if (live) {
-      const int64_t row = e0 / K, k0 = e0 - row * K;
-      const float c = block_const(wc, b, mu);
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + (e0 >> 1));
-      float d[8];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int lane8 = tx & 7;
+  const int64_t kb = K / 64;
+  const int64_t tiles_c = (K + MG_COLS - 1) / MG_COLS;
+  const int64_t tiles = (N + MG_ROWS - 1) / MG_ROWS * tiles_c;
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const int64_t r0 = tile / tiles_c * MG_ROWS, c0 = tile % tiles_c * MG_COLS;
+    const int64_t col = c0 + 8 * tx;                 // this thread's 8 columns
+    const bool col_live = col < K;
+    __syncthreads();                                 // the previous tile is done with a_s, b_s
+    // stage A[0..r)[c0 .. c0+256) as fp32 and B[r0 .. r0+64)[0..r) as pairs
+    for (int i = threadIdx.x; i < r * (MG_COLS / 8); i += blockDim.x) {
+      const int j = i / (MG_COLS / 8), ch = i % (MG_COLS / 8);
+      const int64_t k = c0 + 8 * ch;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (k < K) v = *reinterpret_cast<const uint4*>(A + (size_t)j * K + k);
+      float4* dst = reinterpret_cast<float4*>(a_s + (size_t)j * MG_COLS + 8 * ch);
+      dst[0] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+      dst[1] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+    }
+    for (int i = threadIdx.x; i < r * MG_ROWS; i += blockDim.x) {
+      const int row = i / r, j = i % r;
+      const float b = (r0 + row < N) ? __bfloat162float(B[(size_t)(r0 + row) * r + j]) : 0.0f;
+      b_s[(size_t)j * MG_ROWS + row] = make_float2(b, b);
+    }
+    // codes and block constants of the thread's 8 rows (in flight during the sums)
+    uint32_t w[8];
+    float c[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) d[i] = 0.0f;
-      const __nv_bfloat16* brow = B + row * r;
-      for (int j = 0; j < r; ++j) {
-        const float bj = __bfloat162float(brow[j]);
-        const uint4 a = *reinterpret_cast<const uint4*>(A + (int64_t)j * K + k0);
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+    for (int i = 0; i < 8; ++i) {
+      const int64_t row = r0 + 8 * ty + i;
+      w[i] = 0u;
+      c[i] = 0.0f;
+      if (row < N && col_live) {
+        const int64_t e0 = row * K + col;
+        w[i] = __ldcs(reinterpret_cast<const uint32_t*>(codes + (e0 >> 1)));
+        c[i] = block_const(wc, row * kb + col / 64, mu);
+      }
+    }
+    __syncthreads();
+    // d[i][c] = sum over j in order of B[row i, j] A[j, col c]
+    float2 d[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int h = 0; h < 4; ++h) d[i][h] = make_float2(0.0f, 0.0f);
+    for (int j = 0; j < r; ++j) {
+      const float4 a0 = *reinterpret_cast<const float4*>(a_s + (size_t)j * MG_COLS + 8 * tx);
+      const float4 a1 = *reinterpret_cast<const float4*>(a_s + (size_t)j * MG_COLS + 8 * tx + 4);
+      const float2 ap[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w), make_float2(a1.x, a1.y),
+                            make_float2(a1.z, a1.w)};
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const float4 bb = *reinterpret_cast<const float4*>(b_s + (size_t)j * MG_ROWS + 8 * ty + i);
+        const float2 b0 = make_float2(bb.x, bb.y), b1 = make_float2(bb.z, bb.w);
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          d[2 * h] = __fmaf_rn(bj, bf16_lo(aw[h]), d[2 * h]);
-          d[2 * h + 1] = __fmaf_rn(bj, bf16_hi(aw[h]), d[2 * h + 1]);
+          fma2_rn(d[i][h], b0, ap[h]);
+          fma2_rn(d[i + 1][h], b1, ap[h]);
         }
       }
-      uint32_t pk[4];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float wh = __bfloat162float(__float2bfloat16_rn(__fmul_rn(q[(w >> (4 * i)) & 0xFu], c)));
-        v[i] = __bfloat162float(__float2bfloat16_rn(__fadd_rn(wh, __fmul_rn(s, d[i]))));
-      }
-#pragma unroll
-      for (int h = 0; h < 4; ++h) pk[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
-      if (out) *reinterpret_cast<uint4*>(out + e0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
     }
-    if (codes_out) {   // uniform over the grid: every lane takes part in the shuffles
-      uint32_t abits = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) abits = max(abits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+    for (int i = 0; i < 8; ++i) {
+      const int64_t row = r0 + 8 * ty + i;
+      const bool live = row < N && col_live;
+      const int64_t e0 = row * K + col;
+      float v[8];
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
-      if (abits >= 0x7F800000u && lane8 == 0 && live) raise_status(ST_NONFINITE);
-      const float c2 = __uint_as_float(abits);
-      const uint32_t word = encode8(v, c2, bins, tab);
-      if (live) {
-        *reinterpret_cast<uint32_t*>(codes_out + (e0 >> 1)) = word;
-        if (lane8 == 0) absmax_out[b] = c2;
+      for (int h = 0; h < 4; ++h) {
+        const float dd[2] = {d[i][h].x, d[i][h].y};
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int e = 2 * h + u;
+          const float wh = __bfloat162float(__float2bfloat16_rn(__fmul_rn(q[(w[i] >> (4 * e)) & 0xFu], c[i])));
+          v[e] = live ? __bfloat162float(__float2bfloat16_rn(__fadd_rn(wh, __fmul_rn(s, dd[u])))) : 0.0f;
+        }
+      }
+      if (out && live) {
+        uint4 pk;
+        pk.x = pack_bf16x2(v[0], v[1]);
+        pk.y = pack_bf16x2(v[2], v[3]);
+        pk.z = pack_bf16x2(v[4], v[5]);
+        pk.w = pack_bf16x2(v[6], v[7]);
+        *reinterpret_cast<uint4*>(out + e0) = pk;
+      }
+      if (codes_out) {   // uniform over the grid: every lane takes part in the shuffles
+        uint32_t abits = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) abits = max(abits, __float_as_uint(v[e]) & 0x7FFFFFFFu);
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
+        if (abits >= 0x7F800000u && lane8 == 0 && live) raise_status(ST_NONFINITE);
+        const float c2 = __uint_as_float(abits);
+        const uint32_t word = encode8(v, c2, bins, tab);
+        if (live) {
+          *reinterpret_cast<uint32_t*>(codes_out + (e0 >> 1)) = word;
+          if (lane8 == 0) absmax_out[e0 >> 6] = c2;
+        }
       }
     }
   }
@@ -546,14 +626,26 @@ ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStr
 
 ql_status launch_merge(const ql_nf4_weight* w, const void* A, const void* B, int r, float s, void* out,
                        uint8_t* codes_out, float* absmax_out, cudaStream_t st) {
-  const int64_t nb = w->rows * w->cols / 64;
   WeightConsts wc{w->absmax, w->absmax_q, w->scale2, w->offset};
-  const int bps = ctas_per_sm(merge_kernel);
+  const size_t smem = (size_t)r * (MG_COLS * sizeof(float) + MG_ROWS * sizeof(float2));
+  // the shared-memory size depends on r: set the limit for the largest rank once per device
+  const bool attr = per_device(reinterpret_cast<const void*>(merge_kernel), 0, [] {
+                      const int most = QL_MAX_RANK * (MG_COLS * (int)sizeof(float) + MG_ROWS * (int)sizeof(float2));
+                      if (cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, most) !=
+                          cudaSuccess) {
+                        cudaGetLastError();
+                        return -1;
+                      }
+                      return 1;
+                    }) > 0;
+  if (!attr) return QL_ERR_CUDA;
+  const int64_t tiles = (w->rows + MG_ROWS - 1) / MG_ROWS * ((w->cols + MG_COLS - 1) / MG_COLS);
+  const int64_t cap = (int64_t)sm_count() * 2;
   static const QuantBins bins = build_bins(nf4_table());
   TraceScope ts(TK_MERGE, st);
-  QL_CUDA_TRY(launch(merge_kernel, dim3(grid_for(nb, 32, bps)), dim3(256), 0, st, 1, 1, w->codes, wc, w->rows, w->cols,
-                     (const __nv_bfloat16*)A, (const __nv_bfloat16*)B, r, s, (__nv_bfloat16*)out, codes_out, absmax_out,
-                     nf4_table(), bins));
+  QL_CUDA_TRY(launch(merge_kernel, dim3((unsigned)std::max<int64_t>(1, std::min(tiles, cap))), dim3(256), smem, st, 1,
+                     1, w->codes, wc, w->rows, w->cols, (const __nv_bfloat16*)A, (const __nv_bfloat16*)B, r, s,
+                     (__nv_bfloat16*)out, codes_out, absmax_out, nf4_table(), bins));
   QL_LAUNCH_CHECK();
   return QL_OK;
 }

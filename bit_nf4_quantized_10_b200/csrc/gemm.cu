@@ -94,6 +94,7 @@ struct Params {
   int out_bf16;
   int accumulate;
   int tma_store;     // bf16 output written through shared memory by bulk tensor stores
+  int token_fast;    // tile order: token tiles of a column tile consecutive
   NF4Table tab;
   uint32_t wait_limit;
 };
@@ -180,9 +181,20 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();          // 0 = even CTA (issues the MMAs)
-  const int j0 = (blockIdx.x >> 1) * BN;         // the pair's output-column tile
+  // The pair's tile.  Pairs are dispatched roughly in order of their linear
+  // index; with token_fast the token tiles of one column tile are consecutive,
+  // so that column tile's codes come from DRAM once and from L2 for the other
+  // token tiles (for outputs much wider than the token count, whose codes do
+  // not stay in L2 across a whole pass over the columns).
+  int col_tile = blockIdx.x >> 1, tok_tile = blockIdx.y;
+  if (p.token_fast) {
+    const int pidx = blockIdx.y * (gridDim.x >> 1) + (blockIdx.x >> 1);
+    tok_tile = pidx % gridDim.y;
+    col_tile = pidx / gridDim.y;
+  }
+  const int j0 = col_tile * BN;                  // the pair's output-column tile
   const int jb = j0 + (int)rank * BNH;           // this CTA's weight half
-  const int m0 = blockIdx.y * (2 * BM) + (int)rank * BM;   // this CTA's 256 tokens
+  const int m0 = tok_tile * (2 * BM) + (int)rank * BM;   // this CTA's 256 tokens
   const bool lora = p.r > 0;
   volatile int* abort_flag = sm.abort;
 
@@ -617,6 +629,9 @@ static ql_status launch_gemm_impl(const ql_nf4_weight* w, const void* act, int64
   if (!p.tma_store) memset(&map_out, 0, sizeof(map_out));
   p.tab = nf4_table();
   p.wait_limit = 1u << 22;
+  // token tiles first when the weight side is the larger operand and the
+  // activations (all token tiles) fit in half of L2
+  p.token_fast = (int64_t)M * red * 2 <= (int64_t)64 << 20 && (int64_t)p.n_out > 4 * M;
   const dim3 grid(2u * (unsigned)((p.n_out + BN - 1) / BN), (unsigned)((M + 2 * BM - 1) / (2 * BM)));
   TraceScope ts(BWD ? TK_GEMM_BWD : TK_GEMM_FWD, st);
   QL_CUDA_TRY(launch(qlora_gemm_kernel<BWD>, grid, dim3(THREADS), SMEM_BYTES, st, 2, 1, map_act, map_codes, map_out, p));

@@ -233,11 +233,26 @@ __global__ void __launch_bounds__(THREADS, 1)
 // dst [cols, ld_dst] = src [rows, cols]^T (bf16, cols = r <= 64, a multiple of
 // 8): one thread per source row reads it with 16-byte loads; for each output
 // row the warp's 32 consecutive source rows give 64 contiguous bytes.
-__global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ src, int rows, int cols,
-                                                        uint16_t* __restrict__ dst, int ld_dst) {
+// Row-per-thread transpose of a bf16 [rows, cols] matrix into [cols, ld_dst]
+// (consecutive threads write consecutive columns of dst).  One launch can do
+// two independent transposes: CTAs below `split` take the first matrix, the
+// rest the second (the backward transposes B and U together).
+struct TransposeJob {
+  const uint16_t* src;
+  int rows, cols;
+  uint16_t* dst;
+  int ld_dst;
+};
+
+__global__ void __launch_bounds__(256) transpose_kernel(TransposeJob j0, TransposeJob j1, int split) {
   pdl_wait();
   pdl_trigger();
-  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  const bool first = (int)blockIdx.x < split;
+  const TransposeJob& jb = first ? j0 : j1;
+  const uint16_t* src = jb.src;
+  const int rows = jb.rows, cols = jb.cols, ld_dst = jb.ld_dst;
+  uint16_t* dst = jb.dst;
+  const int row = (int)(first ? blockIdx.x : blockIdx.x - split) * blockDim.x + threadIdx.x;
   if (row >= rows) return;
   const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)row * cols);
   for (int c8 = 0; c8 < cols / 8; ++c8) {
@@ -394,14 +409,22 @@ ql_status launch_grad_a(const void* X, int64_t M, int K, const void* Vt, int64_t
   return skinny_launch(true, X, K, M, Vt, r, ld_vt, s, nullptr, dt, dA, K, dt, TK_COLACC, st);
 }
 
-// dst [cols, ld_dst] = src [rows, cols]^T, bf16
-ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st) {
-  if (cols % 8 != 0 || rows <= 0) return QL_ERR_UNSUPPORTED;
-  const unsigned g = (unsigned)((rows + 255) / 256);
+// dst [cols, ld_dst] = src [rows, cols]^T, bf16; two transposes in one launch
+// (the second may be empty: src1 == NULL).
+ql_status launch_transpose2(const void* src0, int64_t rows0, int cols0, void* dst0, int64_t ld0, const void* src1,
+                            int64_t rows1, int cols1, void* dst1, int64_t ld1, cudaStream_t st) {
+  if (cols0 % 8 != 0 || rows0 <= 0) return QL_ERR_UNSUPPORTED;
+  if (src1 && (cols1 % 8 != 0 || rows1 <= 0)) return QL_ERR_UNSUPPORTED;
+  const int g0 = (int)((rows0 + 255) / 256), g1 = src1 ? (int)((rows1 + 255) / 256) : 0;
+  const skinny::TransposeJob j0{(const uint16_t*)src0, (int)rows0, cols0, (uint16_t*)dst0, (int)ld0};
+  const skinny::TransposeJob j1{(const uint16_t*)src1, (int)rows1, cols1, (uint16_t*)dst1, (int)ld1};
   TraceScope ts(TK_TRANSPOSE, st);
-  QL_CUDA_TRY(launch(skinny::transpose_kernel, dim3(g), dim3(256), 0, st, 1, 1, (const uint16_t*)src, (int)rows, cols,
-                     (uint16_t*)dst, (int)ld_dst));
+  QL_CUDA_TRY(launch(skinny::transpose_kernel, dim3((unsigned)(g0 + g1)), dim3(256), 0, st, 1, 1, j0, j1, g0));
   return QL_OK;
+}
+
+ql_status launch_transpose(const void* src, int64_t rows, int cols, void* dst, int64_t ld_dst, cudaStream_t st) {
+  return launch_transpose2(src, rows, cols, dst, ld_dst, nullptr, 0, 0, nullptr, 0, st);
 }
 
 }  // namespace ql
