@@ -86,17 +86,19 @@ def quantize_sharded(W_slab: torch.Tensor, group=None):
     nodes = torch.empty(-(-nb // 2048), dtype=torch.float64, device=dev)
     L.nf4_double_quant_level1(absmax, nodes)
     world = dist.get_world_size(group)
-    counts = [torch.zeros(1, dtype=torch.int64, device=dev) for _ in range(world)]
-    dist.all_gather(counts, torch.tensor([nb], dtype=torch.int64, device=dev), group=group)
+    # the exchange runs on the device under NCCL and through host memory under gloo
+    xdev = dev if dist.get_backend(group) == "nccl" else torch.device("cpu")
+    counts = [torch.zeros(1, dtype=torch.int64, device=xdev) for _ in range(world)]
+    dist.all_gather(counts, torch.tensor([nb], dtype=torch.int64, device=xdev), group=group)
     nbs = [int(c.item()) for c in counts]
     if any(x % 2048 for x in nbs[:-1]):
         raise ValueError("every slab but the last must hold a multiple of 2048 block constants")
     most = max(-(-x // 2048) for x in nbs)
-    mine = torch.zeros(most, dtype=torch.float64, device=dev)
-    mine[:nodes.numel()] = nodes
-    gathered = [torch.empty(most, dtype=torch.float64, device=dev) for _ in range(world)]
+    mine = torch.zeros(most, dtype=torch.float64, device=xdev)
+    mine[:nodes.numel()] = nodes.to(xdev)
+    gathered = [torch.empty(most, dtype=torch.float64, device=xdev) for _ in range(world)]
     dist.all_gather(gathered, mine, group=group)
-    all_nodes = torch.cat([g[:-(-x // 2048)] for g, x in zip(gathered, nbs)]).contiguous()
+    all_nodes = torch.cat([g[:-(-x // 2048)] for g, x in zip(gathered, nbs)]).to(dev).contiguous()
     nb_total = sum(nbs)
     absmax_q = torch.empty(nb, dtype=torch.uint8, device=dev)
     scale2 = torch.empty(-(-nb // 256), dtype=torch.float32, device=dev)

@@ -46,3 +46,41 @@ def test_slabs_equal_the_whole(rows, split):
     assert torch.equal(torch.cat(s2), whole.scale2)
     for o in mu:
         assert torch.equal(o.view(torch.int32), whole.offset.view(torch.int32))
+
+
+def _sharded_worker(rank, world, port, rows_split):
+    import os
+    import torch.distributed as dist
+    import bit_nf4_quantized_10_b200 as q
+    from bit_nf4_quantized_10_b200.dp import quantize_sharded
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        torch.cuda.set_device(0)
+        W = S.custom_weight(rows_split[-1], 4096, 0.02, 9).to("cuda")
+        r0, r1 = rows_split[rank], rows_split[rank + 1]
+        part = quantize_sharded(W[r0:r1].contiguous())
+        whole = q.quantize_weight(W, dq=True)
+        torch.cuda.synchronize()
+        assert q.qlora_get_status() == q.QL_OK
+        b0, b1 = r0 * 4096 // 64, r1 * 4096 // 64
+        assert torch.equal(part.codes, whole.codes[b0 * 32:b1 * 32])
+        assert torch.equal(part.absmax_q, whole.absmax_q[b0:b1])
+        assert torch.equal(part.scale2, whole.scale2[b0 // 256:-(-b1 // 256)])
+        assert torch.equal(part.offset.view(torch.int32), whole.offset.view(torch.int32))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("rows_split", [[0, 64, 128], [0, 32, 100]])
+def test_quantize_sharded_two_ranks_gloo(rows_split):
+    """dp.quantize_sharded with two ranks (gloo, both on this GPU, each running
+    only its own slab's kernels): every rank's codes, scales and mean are its
+    slice of the single-process quantization."""
+    import socket
+    import torch.multiprocessing as mp
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    mp.spawn(_sharded_worker, args=(2, port, rows_split), nprocs=2, join=True)
