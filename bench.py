@@ -46,7 +46,7 @@ def parse():
     p.add_argument("--no-secondary", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
-    p.add_argument("--leg", choices=["layer", "projection", "smallm", "codec"], default="layer",
+    p.add_argument("--leg", choices=["layer", "projection", "smallm", "codec", "merge"], default="layer",
                    help="with --profile: which workload to run")
     p.add_argument("--profile", action="store_true",
                    help="fixed launch sequence for profilers: exactly --warmup then --steps steps of --leg, "
@@ -154,7 +154,7 @@ class LinearSet:
     linears live in one flat buffer (GradBucket), so the data-parallel exchange
     is one all-reduce.  step() runs the whole hot path once."""
 
-    def __init__(self, q, dev, wl, rank=0, w_dtype=None, M=None):
+    def __init__(self, q, dev, wl, rank=0, w_dtype=None, M=None, streams=1):
         import torch
         from synthetic import inputs as S
         from bit_nf4_quantized_10_b200.dp import GradBucket
@@ -183,7 +183,14 @@ class LinearSet:
                      q.qlora_workspace_size(q.QL_OP_BWD, M, lin.N, lin.K, r))
             self.items.append(it)
             del d
-        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        # the linears are independent: with several streams, linear j runs on
+        # stream j % streams (each with its own workspace), so that one GEMM's
+        # last, partly filled wave of tiles overlaps the next linear's work
+        self.streams = [torch.cuda.Stream(dev) for _ in range(streams)] if streams > 1 else []
+        self.ws_list = [torch.empty(ws, dtype=torch.uint8, device=dev) for _ in range(max(1, streams))]
+        self.ws = self.ws_list[0]
+        self.fork = torch.cuda.Event()
+        self.joins = [torch.cuda.Event() for _ in self.streams]
         shapes = []
         for it in self.items:
             shapes += [(r, it["K"]), (it["N"], r)]
@@ -204,16 +211,33 @@ class LinearSet:
         b = sum(2.0 * M * it["N"] * it["K"] + 2.0 * M * r * it["K"] for it in self.items)
         return f, b
 
-    def step(self, allreduce=False, quantize=True):
+    def _linear(self, it, ws, quantize):
         q, r, s = self.q, self.r, self.s
-        for it in self.items:
-            wq = it["wq"]
-            if quantize:
-                q.nf4_quantize(it["W"], wq.codes, it["absmax"])
-                q.nf4_double_quant(it["absmax"], wq.absmax_q, wq.scale2, wq.offset, it["ws_dq"])
-            q.qlora_linear_fwd(wq, it["X"], it["A"], it["B"], r, s, it["Y"], U_out=it["U"], ws=self.ws)
-            q.qlora_linear_bwd(wq, it["X"], it["dY"], it["A"], it["B"], r, s, it["U"], it["dX"], it["dA"],
-                               it["dB"], ws=self.ws)
+        wq = it["wq"]
+        if quantize:
+            q.nf4_quantize(it["W"], wq.codes, it["absmax"])
+            q.nf4_double_quant(it["absmax"], wq.absmax_q, wq.scale2, wq.offset, it["ws_dq"])
+        q.qlora_linear_fwd(wq, it["X"], it["A"], it["B"], r, s, it["Y"], U_out=it["U"], ws=ws)
+        q.qlora_linear_bwd(wq, it["X"], it["dY"], it["A"], it["B"], r, s, it["U"], it["dX"], it["dA"],
+                           it["dB"], ws=ws)
+
+    def step(self, allreduce=False, quantize=True, concurrent=True):
+        import torch
+        if not self.streams or not concurrent:
+            for it in self.items:
+                self._linear(it, self.ws, quantize)
+        else:
+            cur = torch.cuda.current_stream(self.dev)
+            self.fork.record(cur)
+            for st in self.streams:
+                st.wait_event(self.fork)
+            for j, it in enumerate(self.items):
+                k = j % len(self.streams)
+                with torch.cuda.stream(self.streams[k]):
+                    self._linear(it, self.ws_list[k], quantize)
+            for st, ev in zip(self.streams, self.joins):
+                ev.record(st)
+                cur.wait_event(ev)
         if allreduce:
             self.bucket.allreduce()
 
@@ -362,7 +386,7 @@ def e2e_leg(q, dev, wl, flops_of, world, rank, n_steps, allreduce):
     events).  Also measures the copy-only ceiling of the same bytes."""
     import torch
     import torch.distributed as dist
-    sets = [LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16) for _ in range(2)]
+    sets = [LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16, streams=2) for _ in range(2)]
     h_in = [torch.empty(t.shape, dtype=t.dtype).pin_memory().copy_(t) for t in sets[0].inputs()]
     h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in sets[0].outputs()]
     h2d = sum(t.numel() * t.element_size() for t in h_in)
@@ -467,6 +491,8 @@ def secondary_legs(q, dev, hbm_peak, bf16_peak, peak_src, layer_set):
     # the measured layer without the per-step quantization (fwd + bwd only)
     t = _time_calls(lambda: layer_set.step(quantize=False), flush, n_warm=2, n=10)
     out["layer_70b_linears_fwd_bwd_only"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(layer_set.flops / t / 1e12, 1)}
+    t = _time_calls(lambda: layer_set.step(concurrent=False), flush, n_warm=2, n=10)
+    out["layer_70b_linears_one_stream"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(layer_set.flops / t / 1e12, 1)}
     # the 4096^2 projection: quantize + double quant + fwd + bwd, with its GEMM roofline
     proj = LinearSet(q, dev, S.WORKLOADS["c2"])
     t = _time_calls(proj.step, flush, n_warm=3, n=20)
@@ -644,16 +670,29 @@ def run_reference(args, rank):
 
 def profile_leg(args, q, dev):
     """A fixed launch sequence of one workload for profilers: layer = the
-    measured step; projection = the 4096^2 step; smallm = the 16-token forward
-    on the 28672 x 8192 weight; codec = quantize + double quant of 256 Mi bf16
-    elements.  Prints per-call device times."""
+    measured step (one stream); projection = the 4096^2 step; smallm = the
+    16-token forward on the 28672 x 8192 weight; merge = the adapter merge of
+    that weight (bf16 output and re-quantized codes); codec = quantize + double
+    quant of 256 Mi bf16 elements.  Prints per-call device times."""
     import torch
     from synthetic import inputs as S
     w5 = S.WORKLOADS["c5"]
     if args.leg in ("layer", "projection"):
         ls = LinearSet(q, dev, S.WORKLOADS["c4" if args.leg == "layer" else "c2"],
                        w_dtype=torch.bfloat16 if args.leg == "layer" else None)
-        call = ls.step
+        call = lambda: ls.step(concurrent=False)
+    elif args.leg == "merge":
+        lin = w5.linears[0]
+        N, K, r = lin.N, lin.K, w5.r
+        W = S.normal((N, K), w5.wstd, S.seed_of(5, 0, "W"), device=dev)
+        wq = q.quantize_weight(W, dq=True)
+        del W
+        A = S.uniform((r, K), 1.0 / K ** 0.5, S.seed_of(5, 0, "A"), device=dev)
+        B = S.normal((N, r), 0.01, S.seed_of(5, 0, "B"), device=dev, dtype=torch.bfloat16)
+        W_out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+        codes_out = torch.empty(N * K // 2, dtype=torch.uint8, device=dev)
+        absmax_out = torch.empty(N * K // 64, dtype=torch.float32, device=dev)
+        call = lambda: q.qlora_merge(wq, A, B, r, w5.s, W_out=W_out, codes_out=codes_out, absmax_out=absmax_out)
     elif args.leg == "smallm":
         lin = w5.linears[0]
         N, K, r, s, M = lin.N, lin.K, w5.r, w5.s, 16
@@ -710,7 +749,7 @@ def run_ours(args, rank, world, local_rank):
         return
     hbm_peak, bf16_peak, bf16_sus, peak_src = peaks()
     wl = S.WORKLOADS["c4"]
-    ls = LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16)
+    ls = LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16, streams=2)
     allreduce = world > 1
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2 (126 MB)
 
@@ -758,19 +797,20 @@ def run_ours(args, rank, world, local_rank):
     # the launching stream over the same number of steps (only its kind traced)
     n_rf = args.steps
 
+    # (one stream here: the event pairs time each launch alone)
     def rf_steps():
         for _ in range(n_rf):
             flush.zero_()
-            ls.step(allreduce)
+            ls.step(allreduce, concurrent=False)
         torch.cuda.synchronize()
     roofline = gemm_roofline(q, ls, rf_steps, n_rf, bf16_peak, peak_src, WORKLOAD)
 
-    # per-kernel breakdown: more steps (untimed) with every kind traced
+    # per-kernel breakdown: more steps (untimed, one stream) with every kind traced
     trace_enable(q, True)
     n_br = min(args.steps, 5)
     for _ in range(n_br):
         flush.zero_()
-        ls.step(allreduce)
+        ls.step(allreduce, concurrent=False)
     torch.cuda.synchronize()
     breakdown = trace_read(q)
     trace_enable(q, False)
