@@ -73,6 +73,7 @@ def config(world: int) -> dict:
             "global_batch": 2048 * world, "tokens_per_gpu": 2048, "linears": 7, "r": 16,
             "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, untimed); inputs > L2",
             "outputs": "Y, dX bf16; dA, dB fp32",
+            "schedule": "the seven linears on 3 streams, longest first to the least-loaded stream",
             "launch": "stream order" if os.environ.get("QL_PDL", "1") == "0" else "programmatic dependent launch"}
 
 
@@ -183,10 +184,19 @@ class LinearSet:
                      q.qlora_workspace_size(q.QL_OP_BWD, M, lin.N, lin.K, r))
             self.items.append(it)
             del d
-        # the linears are independent: with several streams, linear j runs on
-        # stream j % streams (each with its own workspace), so that one GEMM's
-        # last, partly filled wave of tiles overlaps the next linear's work
+        # the linears are independent: with several streams each runs on one of
+        # them (each stream with its own workspace), so that one GEMM's last,
+        # partly filled wave of tiles overlaps the next linear's work
         self.streams = [torch.cuda.Stream(dev) for _ in range(streams)] if streams > 1 else []
+        # longest first, each to the least-loaded stream, so the streams end
+        # together and the small linears fill the last waves
+        order = sorted(range(len(wl.linears)), key=lambda j: -wl.linears[j].N * wl.linears[j].K)
+        load = [0] * max(1, streams)
+        self.plan = []
+        for j in order:
+            k = load.index(min(load))
+            load[k] += wl.linears[j].N * wl.linears[j].K
+            self.plan.append((j, k))
         self.ws_list = [torch.empty(ws, dtype=torch.uint8, device=dev) for _ in range(max(1, streams))]
         self.ws = self.ws_list[0]
         self.fork = torch.cuda.Event()
@@ -231,10 +241,9 @@ class LinearSet:
             self.fork.record(cur)
             for st in self.streams:
                 st.wait_event(self.fork)
-            for j, it in enumerate(self.items):
-                k = j % len(self.streams)
+            for j, k in self.plan:
                 with torch.cuda.stream(self.streams[k]):
-                    self._linear(it, self.ws_list[k], quantize)
+                    self._linear(self.items[j], self.ws_list[k], quantize)
             for st, ev in zip(self.streams, self.joins):
                 ev.record(st)
                 cur.wait_event(ev)
@@ -386,7 +395,7 @@ def e2e_leg(q, dev, wl, flops_of, world, rank, n_steps, allreduce):
     events).  Also measures the copy-only ceiling of the same bytes."""
     import torch
     import torch.distributed as dist
-    sets = [LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16, streams=2) for _ in range(2)]
+    sets = [LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16, streams=3) for _ in range(2)]
     h_in = [torch.empty(t.shape, dtype=t.dtype).pin_memory().copy_(t) for t in sets[0].inputs()]
     h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in sets[0].outputs()]
     h2d = sum(t.numel() * t.element_size() for t in h_in)
@@ -749,7 +758,7 @@ def run_ours(args, rank, world, local_rank):
         return
     hbm_peak, bf16_peak, bf16_sus, peak_src = peaks()
     wl = S.WORKLOADS["c4"]
-    ls = LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16, streams=2)
+    ls = LinearSet(q, dev, wl, rank, w_dtype=torch.bfloat16, streams=3)
     allreduce = world > 1
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2 (126 MB)
 

@@ -21,9 +21,12 @@
 //   * K is split over the 16 warps of a CTA (KV codes per row each) and over
 //     parts of K handled by different CTAs; each warp keeps the activation
 //     fragments of its K range in registers for the whole kernel and walks the
-//     CTA's row blocks, loading the next row block's codes into registers while
-//     it expands the current one.  The 16 warps' partial sums meet in shared
-//     memory in warp order; each part's sums go to the workspace.
+//     CTA's row blocks.  A row block's codes and block constants reach the
+//     warp through its own ring of STAGES shared-memory buffers filled by
+//     cp.async, STAGES - 1 row blocks ahead (about 48-96 KB per SM in flight,
+//     what HBM latency times bandwidth asks for).  The 16 warps' partial sums
+//     meet in shared memory in warp order; each part's sums go to the
+//     workspace.
 //   * The CTA that owns the last row block of each part also computes that
 //     part's share of U = X A^T with the same fragments (A rows as M).
 //   * A second kernel sums the parts in order, rounds U to bf16, adds
@@ -93,36 +96,67 @@ __device__ __forceinline__ uint32_t expand_pair(uint32_t e4, uint32_t o4, uint32
   return pack_bf16x2(pl, ph);
 }
 
-// One row's 16 codes of each of this warp's blocks (8 bytes each) for this
-// thread.  Rows past N read nothing and expand to zero (constant 0).
-template <int KV>
-__device__ __forceinline__ void load_codes(const Params& p, int row, int kb0, int nbw, int tq, uint2 (&w)[KV / 64]) {
-#pragma unroll
-  for (int j = 0; j < KV / 64; ++j) {
-    w[j] = make_uint2(0u, 0u);
-    if (row < p.N && j < nbw)
-      w[j] = __ldcs(reinterpret_cast<const uint2*>(p.codes + (size_t)row * (p.K / 2) + (size_t)(kb0 + j) * 32 + tq * 8));
-  }
-}
+// Ring stages per warp, and the bytes of one stage: 16 T rows of KV / 2 code
+// bytes, then per (row, block) the 4-byte word holding the block constant (the
+// aligned word around an E4M3 byte, or a plain fp32 constant) and the group
+// scale s_2, as [block][row] words.
+constexpr int STAGES = 4;
+template <int KV, int T>
+__host__ __device__ constexpr int code_bytes() { return 16 * T * (KV / 2); }
+template <int KV, int T>
+__host__ __device__ constexpr int stage_bytes() { return code_bytes<KV, T>() + 2 * 4 * 16 * T * (KV / 64); }
 
-// Raw block constant of one row's block kb0 + tq (thread tq of each quad takes
-// one block of the warp's chunk, so each constant is loaded and decoded once per
-// quad and handed to the other three by shuffles): the E4M3 byte, or the fp32
-// bits of a plain constant, and its group scale s_2.  Only loads here: the
-// decode waits until the row block is expanded, so the loads of the next row
-// block stay in flight while this one computes.
+// In a stage, row `row`'s 32-byte segment of block j sits at segment
+// j ^ seg_swizzle(row): the 8 rows g a warp's 64-bit fragment read touches
+// then cover every bank twice (two wavefronts, the least for 256 bytes).
 template <int KV>
-__device__ __forceinline__ void load_const(const Params& p, int row, int kb0, int nbw, int tq, uint32_t& q,
-                                           float& s2) {
-  q = 0u;
-  s2 = 0.0f;
-  if (row < p.N && tq < nbw && tq < KV / 64) {
-    const int64_t b = (int64_t)row * p.kb + kb0 + tq;
-    if (p.wc.absmax) {
-      q = __float_as_uint(__ldg(p.wc.absmax + b));
-    } else {
-      q = (uint32_t)__ldg(p.wc.absmax_q + b);
-      s2 = __ldg(p.wc.scale2 + (b >> 8));
+__device__ __forceinline__ int seg_swizzle(int row) { return KV == 128 ? ((row >> 1) & 1) : (row & 3); }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// The warp's codes of row block rb (16 T rows x KV codes from block kb0) into
+// the stage at shared address `stage`, 16 bytes per copy.  Rows past N and
+// blocks past K are zero-filled (source size 0), and expand to zero.
+template <int KV, int T>
+__device__ __forceinline__ void issue_codes(const Params& p, uint32_t stage, int rb, int kb0, int nbw, int lane) {
+  constexpr int CPR = KV / 32;                 // 16-byte chunks per row
+#pragma unroll
+  for (int i = 0; i < 16 * T * CPR / 32; ++i) {
+    const int c = lane + 32 * i;
+    const int row = c / CPR, cc = c % CPR, j = cc >> 1;
+    const int grow = rb * 16 * T + row;
+    const bool live = grow < p.N && j < nbw;
+    const uint8_t* src = live ? p.codes + (size_t)grow * (p.K / 2) + (size_t)kb0 * 32 + cc * 16 : p.codes;
+    cp_async16(stage + row * (KV / 2) + ((((j ^ seg_swizzle<KV>(row)) << 1) | (cc & 1)) << 4), src, live ? 16u : 0u);
+  }
+  // constants: one (row, block) pair per lane and round.  An E4M3 byte comes
+  // in the aligned 4-byte word that holds it (a word never straddles a page,
+  // so the bytes around it are safe to read); its byte is picked at decode.
+  constexpr int PAIRS = 16 * T * (KV / 64);
+  const uint32_t cw = stage + code_bytes<KV, T>(), sw = cw + 4 * PAIRS;
+#pragma unroll
+  for (int i = 0; i < (PAIRS + 31) / 32; ++i) {
+    const int idx = lane + 32 * i;
+    if (idx < PAIRS) {
+      const int row = idx % (16 * T), j = idx / (16 * T);
+      const int grow = rb * 16 * T + row;
+      const bool live = grow < p.N && j < nbw;
+      const int64_t b = live ? (int64_t)grow * p.kb + kb0 + j : 0;
+      if (p.wc.absmax) {
+        cp_async4(cw + 4 * idx, p.wc.absmax + b, live ? 4u : 0u);
+        cp_async4(sw + 4 * idx, p.wc.absmax + b, 0u);
+      } else {
+        cp_async4(cw + 4 * idx, p.wc.absmax_q + (b & ~(int64_t)3), live ? 4u : 0u);
+        cp_async4(sw + 4 * idx, p.wc.scale2 + (b >> 8), live ? 4u : 0u);
+      }
     }
   }
 }
@@ -133,45 +167,47 @@ __device__ __forceinline__ float decode_const(const WeightConsts& wc, uint32_t q
   return __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)q), s2), mu);
 }
 
-// Per row block of 16 T rows: the codes a thread expands and the raw constant
-// of its quad index's block for each of its rows.
 template <int NT, int KV, int T>
-struct Frag {
-  uint2 w[T][2][KV / 64];     // [tile][row g / g+8][block]
-  uint32_t q[T][2];
-  float s2[T][2];
-};
-
-template <int NT, int KV, int T>
-__device__ __forceinline__ void load_frag(const Params& p, int rb, int kb0, int nbw, int g, int tq,
-                                          Frag<NT, KV, T>& f) {
+__device__ __forceinline__ void compute_frag(const Params& p, const uint8_t* stage, int rb, int kb0, float mu,
+                                             const uint32_t (&xb)[KV / 16][NT][2], uint32_t qbase, int nbw,
+                                             int g, int tq, float (&acc)[T][NT][4]) {
+  // this thread's 16 codes of each (row, block): rows 16 t + g (+ 8)
+  uint2 w[T][2][KV / 64];
 #pragma unroll
-  for (int t = 0; t < T; ++t) {
+  for (int t = 0; t < T; ++t)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int row = rb * 16 * T + 16 * t + g + 8 * h;
-      load_codes<KV>(p, row, kb0, nbw, tq, f.w[t][h]);
-      load_const<KV>(p, row, kb0, nbw, tq, f.q[t][h], f.s2[t][h]);
+      const int row = 16 * t + g + 8 * h;
+#pragma unroll
+      for (int j = 0; j < KV / 64; ++j)
+        w[t][h][j] = *reinterpret_cast<const uint2*>(stage + row * (KV / 2) + ((j ^ seg_swizzle<KV>(row)) << 5) + tq * 8);
     }
-  }
-}
-
-template <int NT, int KV, int T>
-__device__ __forceinline__ void compute_frag(const Params& p, const Frag<NT, KV, T>& f, float mu,
-                                             const uint32_t (&xb)[KV / 16][NT][2], uint32_t qbase, int nbw, int g,
-                                             float (&acc)[T][NT][4]) {
 #pragma unroll
   for (int t = 0; t < T; ++t)
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[t][n][i] = 0.0f;
-  // this thread's decoded constants (its quad index's block, rows g and g+8)
+  // this thread's decoded constants (its quad index's block, rows g and g+8):
+  // each is decoded once per quad and handed to the other three by shuffles
+  constexpr int NB = KV / 64;
+  const uint32_t* cw = reinterpret_cast<const uint32_t*>(stage + code_bytes<KV, T>());
+  const float* sw = reinterpret_cast<const float*>(cw + 16 * T * NB);
   float cmine[T][2];
 #pragma unroll
   for (int t = 0; t < T; ++t)
 #pragma unroll
-    for (int h = 0; h < 2; ++h) cmine[t][h] = decode_const(p.wc, f.q[t][h], f.s2[t][h], mu);
+    for (int h = 0; h < 2; ++h) {
+      const int row = 16 * t + g + 8 * h;
+      const int jq = tq < NB ? tq : 0;
+      const uint32_t word = cw[jq * 16 * T + row];
+      uint32_t q = word;
+      if (!p.wc.absmax) {
+        const int64_t b = (int64_t)(rb * 16 * T + row) * p.kb + kb0 + jq;
+        q = (word >> (8 * (int)(b & 3))) & 0xFFu;
+      }
+      cmine[t][h] = decode_const(p.wc, q, sw[jq * 16 * T + row], mu);
+    }
 #pragma unroll
   for (int j = 0; j < KV / 64; ++j) {
     if (j < nbw) {
@@ -182,8 +218,8 @@ __device__ __forceinline__ void compute_frag(const Params& p, const Frag<NT, KV,
         const uint64_t c8 = pack_cc(__shfl_sync(0xffffffffu, cmine[t][1], 4 * g + j));
 #pragma unroll
         for (int half = 0; half < 2; ++half) {        // word .x: k-steps 0, 1; word .y: k-steps 2, 3
-          const uint32_t wg = half ? f.w[t][0][j].y : f.w[t][0][j].x;
-          const uint32_t w8 = half ? f.w[t][1][j].y : f.w[t][1][j].x;
+          const uint32_t wg = half ? w[t][0][j].y : w[t][0][j].x;
+          const uint32_t w8 = half ? w[t][1][j].y : w[t][1][j].x;
           const uint32_t eg = (wg << 2) & 0x3C3C3C3Cu, og = (wg >> 2) & 0x3C3C3C3Cu;
           const uint32_t e8 = (w8 << 2) & 0x3C3C3C3Cu, o8 = (w8 >> 2) & 0x3C3C3C3Cu;
 #pragma unroll
@@ -219,16 +255,21 @@ __device__ __forceinline__ void stash(float* red, const float (&acc)[T][NT][4], 
     }
 }
 
-// Dynamic shared memory of the main kernel: two reduction buffers.
+// Dynamic shared memory of the main kernel: two reduction buffers, then the
+// warps' code rings.
 template <int NT, int T>
 __host__ __device__ constexpr size_t red_floats() { return (size_t)WARPS * 16 * T * 8 * NT; }
+template <int NT, int KV, int T>
+__host__ __device__ constexpr size_t smallm_smem_bytes() {
+  return sizeof(float) * 2 * red_floats<NT, T>() + (size_t)WARPS * STAGES * stage_bytes<KV, T>();
+}
 
 template <int NT, int KV, int T>
 __global__ void __launch_bounds__(THREADS, 1) smallm_kernel(Params p) {
   constexpr int ROWS = 16 * T;
   constexpr int TOK = 8 * NT;
   __shared__ __align__(256) float qlev[64];
-  extern __shared__ __align__(16) float red_dyn[];   // two reduction buffers of red_floats<NT, T>()
+  extern __shared__ __align__(16) float red_dyn[];   // two reduction buffers of red_floats<NT, T>(), the rings
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   if (threadIdx.x < 16) qlev[threadIdx.x] = p.tab.q[threadIdx.x];
@@ -258,19 +299,27 @@ __global__ void __launch_bounds__(THREADS, 1) smallm_kernel(Params p) {
   __syncthreads();
   const uint32_t qbase = opaque_after_barrier(smem_u32(qlev));   // table reads stay below the barrier
   const int rb_first = blockIdx.y, rb_step = gridDim.y;
-  Frag<NT, KV, T> f[2];
+  constexpr int SB = stage_bytes<KV, T>();
+  uint8_t* ring = reinterpret_cast<uint8_t*>(red_dyn + 2 * red_floats<NT, T>()) + (size_t)warp * STAGES * SB;
+  const uint32_t ring_s = smem_u32(ring);
+#pragma unroll
+  for (int st = 0; st < STAGES - 1; ++st) {
+    const int rb = rb_first + st * rb_step;
+    if (rb < p.row_blocks) issue_codes<KV, T>(p, ring_s + st * SB, rb, kb0, nbw, lane);
+    cp_async_commit();
+  }
   int it = 0;
-  if (rb_first < p.row_blocks) load_frag<NT, KV, T>(p, rb_first, kb0, nbw, g, tq, f[0]);
   for (int rb = rb_first; rb < p.row_blocks; rb += rb_step, ++it) {
-    const int nxt = rb + rb_step;
+    // refill the stage the previous row block used, STAGES - 1 row blocks ahead
+    const int ahead = rb + (STAGES - 1) * rb_step;
+    if (ahead < p.row_blocks) issue_codes<KV, T>(p, ring_s + ((it + STAGES - 1) % STAGES) * SB, ahead, kb0, nbw, lane);
+    cp_async_commit();
+    cp_async_wait<STAGES - 1>();                 // this row block's copies (this lane's) have landed
+    __syncwarp();                                // ... and every lane's
+    const uint8_t* stage = ring + (it % STAGES) * SB;
     float acc[T][NT][4];
-    if ((it & 1) == 0) {
-      if (nxt < p.row_blocks) load_frag<NT, KV, T>(p, nxt, kb0, nbw, g, tq, f[1]);
-      compute_frag<NT, KV, T>(p, f[0], mu, xb, qbase, nbw, g, acc);
-    } else {
-      if (nxt < p.row_blocks) load_frag<NT, KV, T>(p, nxt, kb0, nbw, g, tq, f[0]);
-      compute_frag<NT, KV, T>(p, f[1], mu, xb, qbase, nbw, g, acc);
-    }
+    compute_frag<NT, KV, T>(p, stage, rb, kb0, mu, xb, qbase, nbw, g, tq, acc);
+    __syncwarp();                                // the stage is free for the next refill
     float* rbuf = red_dyn + (it & 1) * red_floats<NT, T>();
     stash<NT, T>(rbuf, acc, warp, g, tq);
     __syncthreads();
@@ -284,6 +333,7 @@ __global__ void __launch_bounds__(THREADS, 1) smallm_kernel(Params p) {
       p.part_y[((size_t)part * p.N + row) * p.M + tok] = sum;
     }
   }
+  cp_async_wait<0>();
   // this part's share of U = X A^T: the CTA with the last row block of the part
   if (blockIdx.y == (p.row_blocks - 1) % gridDim.y && p.r > 0) {
     __syncthreads();
@@ -423,7 +473,7 @@ ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, co
   const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
   const int gy = std::max(1, std::min(p.row_blocks, std::max(1, sms / parts)));
   const dim3 grid((unsigned)parts, (unsigned)gy);
-  const size_t smem = sizeof(float) * 2 * (sh.nt == 1 ? red_floats<1, 1>() : red_floats<2, 1>());
+  const size_t smem = sh.nt == 1 ? smallm_smem_bytes<1, 256, 1>() : smallm_smem_bytes<2, 128, 1>();
   auto set_smem = [smem](const void* k) {
     return per_device(k, 0, [k, smem] {
              if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
