@@ -22,50 +22,73 @@ QL_DEFINE_STATUS_ACCESSOR(status_word_codec)
 
 // ---------------------------------------------------------------- quantize
 // Code of x: #{j : x > t_j} over the 15 sorted thresholds t_j = fl32(m_j c)
-// (ties go to the lower level).  The search goes through y = x/c, but only to
-// pick a candidate: the 33 bins round(16 y + 16) are 1/16 wide, narrower than
-// the closest two midpoints (0.093 apart), so each bin (widened by 1e-5 on both
-// sides, far more than the rounding of y) holds at most one threshold j.  The
-// bin table gives j and the count of thresholds below the bin; one exact
-// comparison x > fl32(m_j c) then settles the code.  Bins with no threshold
-// carry m = 4, which no |x| <= c exceeds.
-struct QuantBins {
-  float m[64];
-  uint32_t base[64];
+// (ties go to the lower level).  A first guess goes through y = x/c: one fma
+// with the addend 1.5 * 2^21 + 16 (ulp 1/4) rounds 16 y + 16 to a quarter, so
+// the sum's bit pattern masked with 0x1FC is 4k, k = floor(round(64 y + 64) / 4)
+// the bin y lies in, [(4k - 0.5)/64 - 1, (4k + 3.5)/64 - 1).  Bins are 1/16
+// wide, narrower than the closest two midpoints (0.093 apart), so each bin
+// (widened by 1e-5 on both sides, far more than the error of the approximate
+// 16/c) holds at most one threshold.  Per bin the tables give j, the count of
+// thresholds below the bin, and m_j (4 past the last): the code is then
+// j + [x > fl32(m_j c)], one exact comparison.  Bins 33..127 are reached only
+// from a NaN or from a y one rounding below -1; they hold j = 0, m = 4.  m and
+// j sit in tables of 4-byte words, so 32 lanes reading 33 live entries meet no
+// bank conflict, and 4k is their byte offset as it is.
+struct QuantTab {
+  float m[128];
+  uint32_t j[128];
 };
 
-QuantBins build_bins(const NF4Table& t) {
-  QuantBins b{};
-  for (int k = 0; k < 64; ++k) {
+QuantTab build_quant_tab(const NF4Table& t) {
+  QuantTab b{};
+  for (int k = 0; k < 128; ++k) {
     b.m[k] = 4.0f;
-    b.base[k] = 0;
-    if (k > 32) continue;   // reachable only from a NaN y
-    const double lo = (k - 16.5) / 16.0 - 1e-5, hi = (k - 15.5) / 16.0 + 1e-5;
+    b.j[k] = 0;
+  }
+  for (int k = 0; k <= 32; ++k) {
+    const double lo = (4.0 * k - 0.5) / 64.0 - 1.0 - 1e-5;
     uint32_t below = 0;
-    for (int j = 0; j < 15; ++j) {
+    for (int j = 0; j < 15; ++j)
       if ((double)t.m[j] < lo) ++below;
-      else if ((double)t.m[j] <= hi) b.m[k] = t.m[j];
-    }
-    b.base[k] = below;
+    b.j[k] = below;
+    b.m[k] = below < 15 ? t.m[below] : 4.0f;
   }
   return b;
 }
 
+constexpr float kBinMagic = 3145744.0f;   // 1.5 * 2^21 + 16
+
+template <typename W>
+__device__ __forceinline__ W lds_at(const W* table, uint32_t byte_off) {
+  return *reinterpret_cast<const W*>(reinterpret_cast<const char*>(table) + byte_off);
+}
+
+// Shared-memory copy of the QuantTab, j once per nibble slot i of a code word
+// pre-shifted to j << 4i.
+struct QuantTabSmem {
+  float m[128];
+  uint32_t j[8][128];
+};
+
 // The eight codes of v (elements 0..7 in nibbles 0..7) given the block's
-// absmax c.  `bins` is the QuantBins table in shared memory as (m bits, count
-// below) pairs.
-__device__ __forceinline__ uint32_t encode8(const float (&v)[8], float c, const uint2* bins, const NF4Table& tab) {
+// absmax c.  Scalar fma / mul / compare: the comparison x > fl32(m c) is a
+// compare, never the sign of fl32(m c) - x, which the compiler may contract
+// with the product into one fma (one rounding of m c - x) and so misjudge a
+// tie x = fl32(m c).
+__device__ __forceinline__ uint32_t encode8(const float (&v)[8], float c, const QuantTabSmem& T,
+                                            const NF4Table& tab) {
   uint32_t word = 0;
   if (c >= 1e-30f) {
-    // 16/c: c >= 1e-30 keeps it finite; its rounding moves y by < 1e-6
-    const float s16 = __fmul_rn(16.0f, __frcp_rn(c));
+    // 16/c as the reciprocal of c/16 (exact scaling; 1/(c/16) is normal for
+    // every finite c >= 1e-30)
+    float s16;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(s16) : "f"(c * 0.0625f));
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      // 1.5 * 2^23 + 16: the sum's low bits are round(16 y + 16), in 0..32
-      const float t = __fmaf_rn(v[i], s16, 12582928.0f);
-      const uint2 e = bins[__float_as_uint(t) & 63u];
-      const float th = __fmul_rn(__uint_as_float(e.x), c);
-      word |= (e.y + (v[i] > th ? 1u : 0u)) << (4 * i);
+      const float t = __fmaf_rn(v[i], s16, kBinMagic);
+      const uint32_t o = __float_as_uint(t) & 0x1FCu;
+      const float th = __fmul_rn(lds_at(T.m, o), c);
+      word += lds_at(T.j[i], o) + (v[i] > th ? (1u << (4 * i)) : 0u);
     }
   } else {
     // tiny (or NaN) absmax: count the thresholds directly
@@ -79,6 +102,16 @@ __device__ __forceinline__ uint32_t encode8(const float (&v)[8], float c, const 
   }
   if (c == 0.0f) word = 0x88888888u;
   return word;
+}
+
+// The QuantTab staged into shared memory by threads 0..127.
+__device__ __forceinline__ void stage_quant_tab(const QuantTab& in, QuantTabSmem& T) {
+  if (threadIdx.x < 128) {
+    T.m[threadIdx.x] = in.m[threadIdx.x];
+    const uint32_t j = in.j[threadIdx.x];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) T.j[i][threadIdx.x] = j << (4 * i);
+  }
 }
 
 // Eight consecutive elements as loaded (raw words), and as fp32 values.
@@ -139,71 +172,95 @@ __device__ __forceinline__ void unpack8(const Raw8<__nv_bfloat16>& r, float (&v)
   }
 }
 
-// The largest |x| bit pattern of eight elements, as fp32 bits: for bf16 input
-// the maximum is taken on the packed halves (the sign bits cleared, two 16-bit
-// maxima per instruction) before unpacking.
-__device__ __forceinline__ uint32_t raw_absmax_bits(const Raw8<float>& r) {
-  uint32_t m = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m = max(m, r.w[i] & 0x7FFFFFFFu);
-  return m;
-}
-__device__ __forceinline__ uint32_t raw_absmax_bits(const Raw8<__nv_bfloat16>& r) {
-  uint32_t m = __vmaxu2(r.w[0] & 0x7FFF7FFFu, r.w[1] & 0x7FFF7FFFu);
-  m = __vmaxu2(m, __vmaxu2(r.w[2] & 0x7FFF7FFFu, r.w[3] & 0x7FFF7FFFu));
-  return max(m & 0xFFFFu, m >> 16) << 16;
+// max(a, b), NaN if either is NaN.
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
 }
 
-// 8 threads per 64-block, 8 consecutive elements per thread.  The loop runs
-// over blocks, so the 8 threads of a block always iterate together and can
-// reduce the absmax with shuffles.  The absmax is the integer maximum of the
-// |x| bit patterns (the same order as the values), which also flags NaN and
-// Inf: their patterns are the largest.
+// Block absmax of the eight lanes 8b..8b+7 holding one 64-block: max |x| over
+// the lane's values, then xor shuffles.  NaN propagates and Inf is the
+// largest, so a non-finite block gives a non-finite constant.
+__device__ __forceinline__ float block_absmax(const float (&v)[8]) {
+  float m = fabsf(v[0]);
+#pragma unroll
+  for (int i = 1; i < 8; ++i) m = fmax_nan(m, fabsf(v[i]));
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, o));
+  return m;
+}
+
+// A warp takes 4 QU consecutive 64-blocks per iteration, as QU chunks of 256
+// elements: lane l holds elements 8l..8l+7 of each chunk (one 16-byte load per
+// chunk for bf16, two for fp32; a warp's load is 512 or 1024 contiguous bytes),
+// so lanes 8b..8b+7 hold block b of the chunk and reduce its absmax with
+// shuffles.  The next iteration's chunks are loaded while this one is coded.
+// Addresses are one 64-bit base per iteration plus 32-bit lane offsets; only an
+// iteration that reaches past n checks element bounds.
+constexpr int QU = 2;   // chunks per warp iteration
 template <typename T>
 __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, int64_t n,
                                                        uint8_t* __restrict__ codes,
-                                                       float* __restrict__ absmax, NF4Table tab, QuantBins bins_in) {
+                                                       float* __restrict__ absmax, NF4Table tab, QuantTab tab_in) {
   pdl_wait();
   pdl_trigger();
-  __shared__ uint2 bins[64];   // (m bits, count below)
-  if (threadIdx.x < 64) bins[threadIdx.x] = make_uint2(__float_as_uint(bins_in.m[threadIdx.x]), bins_in.base[threadIdx.x]);
+  __shared__ QuantTabSmem qt;
+  stage_quant_tab(tab_in, qt);
   __syncthreads();
-  const int64_t nb = (n + 63) / 64;
-  const int lane8 = threadIdx.x & 7;
-  const int wib = threadIdx.x >> 5;              // warp in CTA
-  const int bq = (threadIdx.x >> 3) & 3;         // block within the warp's four
-  // the whole warp (4 blocks) iterates together so the shuffles see all lanes
+  constexpr int GE = 256 * QU;                   // elements per warp iteration
+  const int64_t ng = (n + GE - 1) / GE;
+  const int lane = threadIdx.x & 31, lane8 = lane & 7;
   const int64_t warps_per_grid = (int64_t)gridDim.x * (blockDim.x >> 5);
-  // the next iteration's eight elements are loaded (as raw words) while this
-  // one is coded
-  int64_t wb = ((int64_t)blockIdx.x * (blockDim.x >> 5) + wib) * 4;
-  Raw8<T> nxt;
-  if (wb < nb) load8<T>(x, (wb + bq) * 64 + lane8 * 8, n, nxt);
-  for (; wb < nb; wb += warps_per_grid * 4) {
-    const int64_t b = wb + bq;
-    const int64_t e0 = b * 64 + lane8 * 8;   // >= n for a block past the end
-    float v[8];
-    const uint32_t abits0 = raw_absmax_bits(nxt);
-    unpack8(nxt, v);
-    if (wb + warps_per_grid * 4 < nb) load8<T>(x, (wb + warps_per_grid * 4 + bq) * 64 + lane8 * 8, n, nxt);
-    uint32_t abits = abits0;
+  int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  Raw8<T> nxt[QU];
+  if (g < ng) {
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
-    if (abits >= 0x7F800000u && lane8 == 0 && b < nb) raise_status(ST_NONFINITE);
-    const float c = __uint_as_float(abits);
-    const uint32_t word = encode8(v, c, bins, tab);
-    if (e0 + 8 <= n) {
-      __stcs(reinterpret_cast<uint32_t*>(codes + (e0 >> 1)), word);
-    } else if (e0 < n) {
-      const int valid = (int)(n - e0);          // 1..7
-      for (int i = 0; i < valid; i += 2) {
-        uint32_t lo = (word >> (4 * i)) & 0xFu;
-        uint32_t hi = (i + 1 < valid) ? ((word >> (4 * (i + 1))) & 0xFu) : 8u;
-        codes[(e0 + i) >> 1] = (uint8_t)(lo | (hi << 4));
+    for (int u = 0; u < QU; ++u) load8<T>(x, g * GE + 256 * u + 8 * lane, n, nxt[u]);
+  }
+  bool nonfinite = false;
+  for (; g < ng; g += warps_per_grid) {
+    Raw8<T> cur[QU];
+#pragma unroll
+    for (int u = 0; u < QU; ++u) cur[u] = nxt[u];
+    const int64_t gn = g + warps_per_grid;
+    if (gn < ng) {
+#pragma unroll
+      for (int u = 0; u < QU; ++u) load8<T>(x, gn * GE + 256 * u + 8 * lane, n, nxt[u]);
+    }
+    const int64_t base = g * GE;
+    const bool full = base + GE <= n;            // no element of the iteration past the end
+    uint8_t* cbase = codes + (base >> 1);
+    float* abase = absmax + (base >> 6);
+#pragma unroll
+    for (int u = 0; u < QU; ++u) {
+      float v[8];
+      unpack8(cur[u], v);
+      const float c = block_absmax(v);
+      nonfinite |= !(c <= 3.402823466e38f);
+      const uint32_t word = encode8(v, c, qt, tab);
+      const int off = 256 * u + 8 * lane;        // element offset in the iteration
+      if (full) {
+        __stcs(reinterpret_cast<uint32_t*>(cbase + (off >> 1)), word);
+        if (lane8 == 0) abase[off >> 6] = c;
+      } else {
+        const int64_t e0 = base + off;           // >= n for a block past the end
+        if (e0 + 8 <= n) {
+          __stcs(reinterpret_cast<uint32_t*>(cbase + (off >> 1)), word);
+        } else if (e0 < n) {
+          const int valid = (int)(n - e0);       // 1..7
+          for (int i = 0; i < valid; i += 2) {
+            uint32_t lo = (word >> (4 * i)) & 0xFu;
+            uint32_t hi = (i + 1 < valid) ? ((word >> (4 * (i + 1))) & 0xFu) : 8u;
+            cbase[(off + i) >> 1] = (uint8_t)(lo | (hi << 4));
+          }
+        }
+        if (lane8 == 0 && e0 < n) abase[off >> 6] = c;
       }
     }
-    if (lane8 == 0 && b < nb) absmax[b] = c;
   }
+  // padding past n is zero, so only real elements can be non-finite
+  if (nonfinite) raise_status(ST_NONFINITE);
 }
 
 // --------------------------------------------------------- double quant: mean
@@ -352,115 +409,152 @@ __global__ void __launch_bounds__(256) dequant_f32_kernel(const uint8_t* __restr
 // quantize_kernel), without a round trip of the bf16 weight through HBM.
 // The rank-r product d = B A is a small matrix product, so each thread owns a
 // register tile of 8 rows x 8 consecutive columns of a 64-row x 256-column CTA
-// tile and accumulates its 64 sums with packed fp32 FMAs (two independent
-// IEEE fmas per instruction, j in order), reading A (as fp32) and B (as
-// broadcast pairs) from shared memory staged once per tile: every A and B
-// value is reused by 8 rows or 8 columns.  The 8 threads holding a row's
-// 64-block are 8 consecutive lanes, so the re-quantization's absmax is the same
-// 8-lane shuffle as in quantize_kernel.  K % 64 == 0, so a block lies in one
-// row and a tile edge never splits one.
+// tile and accumulates its 64 sums with scalar fp32 fmas (j in order), reading
+// A and B as fp32 from shared memory (a warp's B values are one broadcast):
+// every A and B value is reused by 8 rows or 8 columns.  The FMA pipe takes
+// scalar and packed fmas at the same element rate, and the scalar form needs no
+// register-pair assembly around each instruction.  A CTA keeps one 256-column tile for its whole life and walks
+// row tiles, so A's slice is staged once; B's 64 x r slice of the next row tile
+// is loaded into registers while the current one computes.  The 8 threads
+// holding a row's 64-block are 8 consecutive lanes, so the re-quantization's
+// absmax is the same 8-lane shuffle as in quantize_kernel.  K % 64 == 0, so a
+// block lies in one row and a tile edge never splits one.
 constexpr int MG_ROWS = 64;     // rows per CTA tile: 8 warps x 8 rows
 constexpr int MG_COLS = 256;    // columns per CTA tile: 32 lanes x 8 columns
 
-__device__ __forceinline__ void fma2_rn(float2& d, float2 a, float2 b) {
-  asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n mov.b64 z, {%0, %1};\n"
-      " fma.rn.f32x2 z, x, y, z;\n mov.b64 {%0, %1}, z;\n}"
-      : "+f"(d.x), "+f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+// Element i of B's 64 x r slice of row tile rt (row i / r, column i % r), 0
+// past the slice, the row tiles or N.
+__device__ __forceinline__ float merge_b(const __nv_bfloat16* B, int64_t N, int r, int tiles_r, int rt, int i) {
+  const int64_t row = (int64_t)rt * MG_ROWS + i / r;
+  return (i < MG_ROWS * r && rt < tiles_r && row < N) ? __bfloat162float(B[(size_t)row * r + i % r]) : 0.0f;
 }
 
+// RMAX >= r: B's 64 x r slice of a row tile is spread over the 256 threads,
+// MG_ROWS * RMAX / 256 values each.
+template <int RMAX>
 __global__ void __launch_bounds__(256, 2) merge_kernel(const uint8_t* __restrict__ codes, WeightConsts wc, int64_t N,
                                                     int64_t K, const __nv_bfloat16* __restrict__ A,
                                                     const __nv_bfloat16* __restrict__ B, int r, float s,
                                                     __nv_bfloat16* __restrict__ out, uint8_t* __restrict__ codes_out,
-                                                    float* __restrict__ absmax_out, NF4Table tab, QuantBins bins_in) {
+                                                    float* __restrict__ absmax_out, NF4Table tab, QuantTab tab_in) {
   pdl_wait();
   pdl_trigger();
-  __shared__ uint2 bins[64];
+  __shared__ QuantTabSmem qt;
   __shared__ float q[16];
   extern __shared__ __align__(16) float mg_smem[];
   float* a_s = mg_smem;                                               // [r][256] fp32
-  float2* b_s = reinterpret_cast<float2*>(mg_smem + (size_t)r * MG_COLS);   // [r][64] (b, b)
-  if (threadIdx.x < 64) bins[threadIdx.x] = make_uint2(__float_as_uint(bins_in.m[threadIdx.x]), bins_in.base[threadIdx.x]);
-  if (threadIdx.x < 16) q[threadIdx.x] = tab.q[threadIdx.x];
+  float* b_s = mg_smem + (size_t)r * MG_COLS;                          // [r][64] fp32
+  uint32_t* w_s = reinterpret_cast<uint32_t*>(b_s + (size_t)r * MG_ROWS);    // [64][32] code words of the tile
+  stage_quant_tab(tab_in, qt);
+#pragma unroll
+  for (int k = 0; k < 16; ++k)                       // constant indices: the table stays in parameter space
+    if (threadIdx.x == k) q[k] = tab.q[k];
   const float mu = wc.absmax ? 0.0f : *wc.offset;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int lane8 = tx & 7;
   const int64_t kb = K / 64;
-  const int64_t tiles_c = (K + MG_COLS - 1) / MG_COLS;
-  const int64_t tiles = (N + MG_ROWS - 1) / MG_ROWS * tiles_c;
-  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-    const int64_t r0 = tile / tiles_c * MG_ROWS, c0 = tile % tiles_c * MG_COLS;
-    const int64_t col = c0 + 8 * tx;                 // this thread's 8 columns
-    const bool col_live = col < K;
-    __syncthreads();                                 // the previous tile is done with a_s, b_s
-    // stage A[0..r)[c0 .. c0+256) as fp32 and B[r0 .. r0+64)[0..r) as pairs
-    for (int i = threadIdx.x; i < r * (MG_COLS / 8); i += blockDim.x) {
-      const int j = i / (MG_COLS / 8), ch = i % (MG_COLS / 8);
-      const int64_t k = c0 + 8 * ch;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (k < K) v = *reinterpret_cast<const uint4*>(A + (size_t)j * K + k);
-      float4* dst = reinterpret_cast<float4*>(a_s + (size_t)j * MG_COLS + 8 * ch);
-      dst[0] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
-      dst[1] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+  const int tiles_c = (int)((K + MG_COLS - 1) / MG_COLS);
+  const int tiles_r = (int)((N + MG_ROWS - 1) / MG_ROWS);
+  // this CTA's column tile, and its share of the row tiles
+  const int ct = blockIdx.x % tiles_c;
+  const int rt0 = blockIdx.x / tiles_c, rt_step = gridDim.x / tiles_c;
+  const int64_t c0 = (int64_t)ct * MG_COLS;
+  const int64_t col = c0 + 8 * tx;                   // this thread's 8 columns
+  const bool col_live = col < K;
+  // stage A[0..r)[c0 .. c0+256) as fp32, once
+  for (int i = threadIdx.x; i < r * (MG_COLS / 8); i += blockDim.x) {
+    const int j = i / (MG_COLS / 8), ch = i % (MG_COLS / 8);
+    const int64_t k = c0 + 8 * ch;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (k < K) v = *reinterpret_cast<const uint4*>(A + (size_t)j * K + k);
+    float4* dst = reinterpret_cast<float4*>(a_s + (size_t)j * MG_COLS + 8 * ch);
+    dst[0] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+    dst[1] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+  }
+  constexpr int MG_BPT = MG_ROWS * RMAX / 256;
+  // B[r0 .. r0+64)[0..r) of a row tile, MG_BPT values per thread (element
+  // i = threadIdx.x + 256 u of the slice, row i / r, column i % r)
+  float bnext[MG_BPT];
+#pragma unroll
+  for (int u = 0; u < MG_BPT; ++u) bnext[u] = merge_b(B, N, r, tiles_r, rt0, threadIdx.x + 256 * u);
+  for (int rt = rt0; rt < tiles_r; rt += rt_step) {
+    const int64_t r0 = (int64_t)rt * MG_ROWS;
+    __syncthreads();                                 // the previous tile is done with b_s (and A is staged)
+#pragma unroll
+    for (int u = 0; u < MG_BPT; ++u) {
+      const int i = threadIdx.x + 256 * u;
+      if (i < MG_ROWS * r) b_s[(size_t)(i % r) * MG_ROWS + i / r] = bnext[u];
     }
-    for (int i = threadIdx.x; i < r * MG_ROWS; i += blockDim.x) {
-      const int row = i / r, j = i % r;
-      const float b = (r0 + row < N) ? __bfloat162float(B[(size_t)(r0 + row) * r + j]) : 0.0f;
-      b_s[(size_t)j * MG_ROWS + row] = make_float2(b, b);
+    // the tile's codes into shared memory (in flight during the sums): 64 rows
+    // of 128 bytes, two 16-byte copies per thread, zero past N or K
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int id = threadIdx.x + 256 * u, row = id >> 3, ch = id & 7;
+      const bool live = r0 + row < N && c0 + 32 * ch < K;
+      const uint8_t* src = live ? codes + (((r0 + row) * K + c0) >> 1) + 16 * ch : codes;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(w_s) + 16 * id), "l"(src),
+                   "r"(live ? 16u : 0u)
+                   : "memory");
     }
-    // codes and block constants of the thread's 8 rows (in flight during the sums)
-    uint32_t w[8];
-    float c[8];
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    // raw block constants of the thread's 8 rows (in flight during the sums;
+    // decoded after them): the fp32 constant's bits, or the E4M3 byte and s_2
+    uint32_t craw[8];
+    float cs2[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int64_t row = r0 + 8 * ty + i;
-      w[i] = 0u;
-      c[i] = 0.0f;
+      craw[i] = 0u;
+      cs2[i] = 0.0f;
       if (row < N && col_live) {
-        const int64_t e0 = row * K + col;
-        w[i] = __ldcs(reinterpret_cast<const uint32_t*>(codes + (e0 >> 1)));
-        c[i] = block_const(wc, row * kb + col / 64, mu);
-      }
-    }
-    __syncthreads();
-    // d[i][c] = sum over j in order of B[row i, j] A[j, col c]
-    float2 d[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int h = 0; h < 4; ++h) d[i][h] = make_float2(0.0f, 0.0f);
-    for (int j = 0; j < r; ++j) {
-      const float4 a0 = *reinterpret_cast<const float4*>(a_s + (size_t)j * MG_COLS + 8 * tx);
-      const float4 a1 = *reinterpret_cast<const float4*>(a_s + (size_t)j * MG_COLS + 8 * tx + 4);
-      const float2 ap[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w), make_float2(a1.x, a1.y),
-                            make_float2(a1.z, a1.w)};
-#pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        const float4 bb = *reinterpret_cast<const float4*>(b_s + (size_t)j * MG_ROWS + 8 * ty + i);
-        const float2 b0 = make_float2(bb.x, bb.y), b1 = make_float2(bb.z, bb.w);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          fma2_rn(d[i][h], b0, ap[h]);
-          fma2_rn(d[i + 1][h], b1, ap[h]);
+        const int64_t b = row * kb + col / 64;
+        if (wc.absmax) {
+          craw[i] = __float_as_uint(__ldg(wc.absmax + b));
+        } else {
+          craw[i] = __ldg(wc.absmax_q + b);
+          cs2[i] = __ldg(wc.scale2 + (b >> 8));
         }
       }
     }
+#pragma unroll
+    for (int u = 0; u < MG_BPT; ++u)                 // the next row tile's B, in flight
+      bnext[u] = merge_b(B, N, r, tiles_r, rt + rt_step, threadIdx.x + 256 * u);
+    __syncthreads();
+    // d[i][c] = sum over j in order of B[row i, j] A[j, col c]
+    float d[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) d[i][cc] = 0.0f;
+    for (int j = 0; j < r; ++j) {
+      const float4 a0 = *reinterpret_cast<const float4*>(a_s + (size_t)j * MG_COLS + 8 * tx);
+      const float4 a1 = *reinterpret_cast<const float4*>(a_s + (size_t)j * MG_COLS + 8 * tx + 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(b_s + (size_t)j * MG_ROWS + 8 * ty);
+      const float4 b1 = *reinterpret_cast<const float4*>(b_s + (size_t)j * MG_ROWS + 8 * ty + 4);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) d[i][cc] = __fmaf_rn(bv[i], av[cc], d[i][cc]);
+    }
+    float c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      c[i] = wc.absmax ? __uint_as_float(craw[i]) : __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)craw[i]), cs2[i]), mu);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();                                 // every thread's code copies have landed
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int64_t row = r0 + 8 * ty + i;
       const bool live = row < N && col_live;
+      const uint32_t wi = w_s[(8 * ty + i) * 32 + tx];
       const int64_t e0 = row * K + col;
       float v[8];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float dd[2] = {d[i][h].x, d[i][h].y};
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int e = 2 * h + u;
-          const float wh = __bfloat162float(__float2bfloat16_rn(__fmul_rn(q[(w[i] >> (4 * e)) & 0xFu], c[i])));
-          v[e] = live ? __bfloat162float(__float2bfloat16_rn(__fadd_rn(wh, __fmul_rn(s, dd[u])))) : 0.0f;
-        }
+      for (int e = 0; e < 8; ++e) {
+        const float wh = __bfloat162float(__float2bfloat16_rn(__fmul_rn(q[(wi >> (4 * e)) & 0xFu], c[i])));
+        v[e] = live ? __bfloat162float(__float2bfloat16_rn(__fadd_rn(wh, __fmul_rn(s, d[i][e])))) : 0.0f;
       }
       if (out && live) {
         uint4 pk;
@@ -478,7 +572,7 @@ __global__ void __launch_bounds__(256, 2) merge_kernel(const uint8_t* __restrict
         for (int o = 1; o < 8; o <<= 1) abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
         if (abits >= 0x7F800000u && lane8 == 0 && live) raise_status(ST_NONFINITE);
         const float c2 = __uint_as_float(abits);
-        const uint32_t word = encode8(v, c2, bins, tab);
+        const uint32_t word = encode8(v, c2, qt, tab);
         if (live) {
           *reinterpret_cast<uint32_t*>(codes_out + (e0 >> 1)) = word;
           if (lane8 == 0) absmax_out[e0 >> 6] = c2;
@@ -519,16 +613,16 @@ static unsigned grid_for(int64_t work_items, int per_cta, int ctas_per_sm) {
 ql_status launch_quantize(const void* x, ql_dtype dt, int64_t n, uint8_t* codes, float* absmax,
                           cudaStream_t st) {
   const int64_t nb = (n + 63) / 64;
-  // one resident wave of CTAs (grid-stride loop), 32 blocks (8 warps x 4) per CTA iteration
+  // one resident wave of CTAs (grid-stride loop), 8 warps x 4 QU blocks per CTA iteration
   const int bps = dt == QL_F32 ? ctas_per_sm(quantize_kernel<float>) : ctas_per_sm(quantize_kernel<__nv_bfloat16>);
-  const unsigned grid = grid_for(nb, 32, bps);
-  static const QuantBins bins = build_bins(nf4_table());
+  const unsigned grid = grid_for(nb, 8 * 4 * QU, bps);
+  static const QuantTab qtab = build_quant_tab(nf4_table());
   TraceScope ts(TK_QUANTIZE, st);
   if (dt == QL_F32)
-    QL_CUDA_TRY(launch(quantize_kernel<float>, dim3(grid), dim3(256), 0, st, 1, 1, (const float*)x, n, codes, absmax, nf4_table(), bins));
+    QL_CUDA_TRY(launch(quantize_kernel<float>, dim3(grid), dim3(256), 0, st, 1, 1, (const float*)x, n, codes, absmax, nf4_table(), qtab));
   else
     QL_CUDA_TRY(launch(quantize_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, 1, 1, (const __nv_bfloat16*)x, n, codes, absmax,
-                                                         nf4_table(), bins));
+                                                         nf4_table(), qtab));
   QL_LAUNCH_CHECK();
   return QL_OK;
 }
@@ -624,30 +718,42 @@ ql_status launch_dequant(const ql_nf4_weight* w, void* out, ql_dtype dt, cudaStr
 }
 
 
-ql_status launch_merge(const ql_nf4_weight* w, const void* A, const void* B, int r, float s, void* out,
-                       uint8_t* codes_out, float* absmax_out, cudaStream_t st) {
+template <int RMAX>
+static ql_status launch_merge_r(const ql_nf4_weight* w, const void* A, const void* B, int r, float s, void* out,
+                                uint8_t* codes_out, float* absmax_out, cudaStream_t st) {
   WeightConsts wc{w->absmax, w->absmax_q, w->scale2, w->offset};
-  const size_t smem = (size_t)r * (MG_COLS * sizeof(float) + MG_ROWS * sizeof(float2));
+  const size_t smem = (size_t)r * (MG_COLS + MG_ROWS) * sizeof(float) + MG_ROWS * MG_COLS / 2;
   // the shared-memory size depends on r: set the limit for the largest rank once per device
-  const bool attr = per_device(reinterpret_cast<const void*>(merge_kernel), 0, [] {
-                      const int most = QL_MAX_RANK * (MG_COLS * (int)sizeof(float) + MG_ROWS * (int)sizeof(float2));
-                      if (cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, most) !=
-                          cudaSuccess) {
+  const bool attr = per_device(reinterpret_cast<const void*>(merge_kernel<RMAX>), 0, [] {
+                      const int most = RMAX * (MG_COLS + MG_ROWS) * (int)sizeof(float) + MG_ROWS * MG_COLS / 2;
+                      if (cudaFuncSetAttribute(merge_kernel<RMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               most) != cudaSuccess) {
                         cudaGetLastError();
                         return -1;
                       }
                       return 1;
                     }) > 0;
   if (!attr) return QL_ERR_CUDA;
-  const int64_t tiles = (w->rows + MG_ROWS - 1) / MG_ROWS * ((w->cols + MG_COLS - 1) / MG_COLS);
-  const int64_t cap = (int64_t)sm_count() * 2;
-  static const QuantBins bins = build_bins(nf4_table());
+  // each CTA keeps one column tile: the grid is the column tiles times the
+  // number of CTAs that share each one's row tiles (about two CTAs per SM)
+  const int64_t tiles_c = (w->cols + MG_COLS - 1) / MG_COLS;
+  const int64_t tiles_r = (w->rows + MG_ROWS - 1) / MG_ROWS;
+  const int64_t rsplit = std::max<int64_t>(1, std::min<int64_t>(tiles_r, (int64_t)sm_count() * 2 / tiles_c));
+  static const QuantTab qtab = build_quant_tab(nf4_table());
   TraceScope ts(TK_MERGE, st);
-  QL_CUDA_TRY(launch(merge_kernel, dim3((unsigned)std::max<int64_t>(1, std::min(tiles, cap))), dim3(256), smem, st, 1,
-                     1, w->codes, wc, w->rows, w->cols, (const __nv_bfloat16*)A, (const __nv_bfloat16*)B, r, s,
-                     (__nv_bfloat16*)out, codes_out, absmax_out, nf4_table(), bins));
+  QL_CUDA_TRY(launch(merge_kernel<RMAX>, dim3((unsigned)(tiles_c * rsplit)), dim3(256), smem, st, 1, 1, w->codes, wc,
+                     w->rows, w->cols, (const __nv_bfloat16*)A, (const __nv_bfloat16*)B, r, s, (__nv_bfloat16*)out,
+                     codes_out, absmax_out, nf4_table(), qtab));
   QL_LAUNCH_CHECK();
   return QL_OK;
+}
+
+ql_status launch_merge(const ql_nf4_weight* w, const void* A, const void* B, int r, float s, void* out,
+                       uint8_t* codes_out, float* absmax_out, cudaStream_t st) {
+  static_assert(QL_MAX_RANK <= 64, "merge stages at most 64 adapter columns");
+  if (r <= 16) return launch_merge_r<16>(w, A, B, r, s, out, codes_out, absmax_out, st);
+  if (r <= 32) return launch_merge_r<32>(w, A, B, r, s, out, codes_out, absmax_out, st);
+  return launch_merge_r<64>(w, A, B, r, s, out, codes_out, absmax_out, st);
 }
 
 }  // namespace ql
