@@ -500,8 +500,10 @@ def secondary_legs(q, dev, hbm_peak, bf16_peak, peak_src, layer_set):
     # the measured layer without the per-step quantization (fwd + bwd only)
     t = _time_calls(lambda: layer_set.step(quantize=False), flush, n_warm=2, n=10)
     out["layer_70b_linears_fwd_bwd_only"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(layer_set.flops / t / 1e12, 1)}
+    t_own = t
     t = _time_calls(lambda: layer_set.step(concurrent=False), flush, n_warm=2, n=10)
     out["layer_70b_linears_one_stream"] = {"ms": round(t * 1e3, 3), "TFLOPs": round(layer_set.flops / t / 1e12, 1)}
+    out.update(dense_context_leg(layer_set, flush, t_own))
     # the 4096^2 projection: quantize + double quant + fwd + bwd, with its GEMM roofline
     proj = LinearSet(q, dev, S.WORKLOADS["c2"])
     t = _time_calls(proj.step, flush, n_warm=3, n=20)
@@ -522,6 +524,29 @@ def secondary_legs(q, dev, hbm_peak, bf16_peak, peak_src, layer_set):
     out.update(small_m_and_codec(q, dev, hbm_peak, flush))
     out.update(adamw_leg(q, dev, hbm_peak, layer_set, flush))
     return out
+
+
+def dense_context_leg(layer_set, flush, t_nf4):
+    """Same-box context, not the product: the layer's forward and dX GEMMs with
+    the unquantized bf16 weights through torch.matmul (cuBLAS), next to the
+    NF4 path's fwd + bwd on the same shapes.  The pages put the cost of
+    dequantizing on the fly at under 15% of unquantized throughput
+    ("QLoRA: Quantize Base Weights to 4-Bit", Section 3)."""
+    import torch
+    outs = [(torch.empty_like(it["Y"]), torch.empty_like(it["dX"])) for it in layer_set.items]
+
+    def dense():
+        for it, (y, dx) in zip(layer_set.items, outs):
+            torch.matmul(it["X"], it["W"].t(), out=y)
+            torch.matmul(it["dY"], it["W"], out=dx)
+
+    t = _time_calls(dense, flush, n_warm=2, n=10)
+    flop = sum(4.0 * layer_set.M * it["N"] * it["K"] for it in layer_set.items)
+    del outs
+    return {"torch_bf16_dense_layer_70b": {
+        "ms": round(t * 1e3, 3), "TFLOPs": round(flop / t / 1e12, 1),
+        "what": "Y = X W^T and dX = dY W per linear, bf16 dense weights, torch.matmul (context only)",
+        "nf4_fwd_bwd_over_dense": round(t_nf4 / t, 3)}}
 
 
 def mlp_leg(q, dev, flush):
