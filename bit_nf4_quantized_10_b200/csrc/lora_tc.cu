@@ -37,13 +37,20 @@ namespace skinny {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int B_BYTES = 64 * BK * 2;   // 8 KB (r <= 64)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 6 * 32;        // TMA, MMA, 4 drain warps
 constexpr int TMEM_COLS = 64;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+// Ring depth.  The K-major form (U, V) has only M/128 row tiles (16 at 2048
+// tokens), so a cluster of split CTAs per tile leaves one CTA per SM, whose
+// ring alone must cover HBM latency: 8 stages (128 KB of activations in
+// flight).  The MN-major form (dA, dB) has a row tile per 128 columns and two
+// CTAs per SM, with 4 stages each.
+template <bool A_MN>
+__host__ __device__ constexpr int stages() { return A_MN ? 4 : 8; }
+template <bool A_MN>
+__host__ __device__ constexpr size_t smem_bytes() { return 1024 + (size_t)stages<A_MN>() * STAGE_BYTES + 256; }
 
 constexpr int MAX_SPLITS = 8;           // portable cluster size
 
@@ -91,6 +98,7 @@ template <bool A_MN>
 __global__ void __launch_bounds__(THREADS, 1)
     skinny_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                   const Params p) {
+  constexpr int STAGES = stages<A_MN>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * STAGE_BYTES);
@@ -287,7 +295,7 @@ static void split_plan_compute(bool a_mn, int rows, int64_t red, int& splits, in
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)tiles, (unsigned)sp);
     cfg.blockDim = dim3(skinny::THREADS);
-    cfg.dynamicSmemBytes = skinny::SMEM_BYTES;
+    cfg.dynamicSmemBytes = a_mn ? skinny::smem_bytes<true>() : skinny::smem_bytes<false>();
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = 1;
@@ -342,8 +350,9 @@ static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, 
   using namespace skinny;
   // two CTAs per SM need the largest shared-memory carveout (per-device attributes)
   auto k = a_mn ? skinny_kernel<true> : skinny_kernel<false>;
-  if (per_device(reinterpret_cast<const void*>(k), 0, [k] {
-        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) != cudaSuccess ||
+  const size_t smem = a_mn ? smem_bytes<true>() : smem_bytes<false>();
+  if (per_device(reinterpret_cast<const void*>(k), 0, [k, smem] {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
             cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) {
           cudaGetLastError();
           return -1;
@@ -384,8 +393,8 @@ static ql_status skinny_launch(bool a_mn, const void* z, int rows, int64_t red, 
   const dim3 grid((unsigned)tiles, (unsigned)splits);
   {
     TraceScope ts(kind, st);
-    if (a_mn) QL_CUDA_TRY(launch(skinny_kernel<true>, grid, dim3(THREADS), SMEM_BYTES, st, 1, (unsigned)splits, ma, mb, p));
-    else QL_CUDA_TRY(launch(skinny_kernel<false>, grid, dim3(THREADS), SMEM_BYTES, st, 1, (unsigned)splits, ma, mb, p));
+    if (a_mn) QL_CUDA_TRY(launch(skinny_kernel<true>, grid, dim3(THREADS), smem, st, 1, (unsigned)splits, ma, mb, p));
+    else QL_CUDA_TRY(launch(skinny_kernel<false>, grid, dim3(THREADS), smem, st, 1, (unsigned)splits, ma, mb, p));
   }
   return QL_OK;
 }

@@ -59,6 +59,10 @@ SHAPES = [
     (136, 192, 64, 0.5),      # the largest rank
     (96, 128, 3, 1.0),        # a rank that is no multiple of 8
     (64, 128, 0, 2.0),        # no adapter: the merge is the dequantized weight
+    # K = 16384 leaves 4 CTAs per 256-column tile, so each walks several 64-row
+    # tiles (the next tile's B and codes load during the current one's sums)
+    (520, 16384, 32, 0.75),   # ranks 17..32, a ragged last row tile of 8 rows
+    (640, 16384, 64, 0.5),    # ranks 33..64
 ]
 
 
