@@ -25,7 +25,8 @@ EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_double_quant_noalloc", "nf4_
            "qlora_silu_gate_fwd", "qlora_silu_gate_bwd", "qlora_workspace_size", "nf4_storage_bytes",
            "nf4_codebook", "qlora_get_status", "qlora_status_string", "qlora_selftest_wait_timeout",
            "qlora_merge", "nf4_double_quant_level1", "nf4_double_quant_finish", "nvfp4_quantize", "mxfp4_quantize",
-           "nvfp4_dequant", "mxfp4_dequant", "qlora_adamw_step", "qlora_paged_prefetch")
+           "nvfp4_dequant", "mxfp4_dequant", "qlora_adamw_step", "qlora_paged_prefetch", "nvfp4_scale_atoms_bytes",
+           "nvfp4_scale_atoms", "nvfp4_gemm")
 
 
 class QLoraError(RuntimeError):
@@ -70,6 +71,9 @@ def _load() -> ctypes.CDLL:
         "mxfp4_dequant": (i32, [vp, vp, i64, vp, vp]),
         "qlora_adamw_step": (i32, [vp, vp, vp, vp, vp, i64, i64, f32, f32, f32, f32, f32, vp]),
         "qlora_paged_prefetch": (i32, [vp, sz, i32, vp]),
+        "nvfp4_scale_atoms_bytes": (sz, [i64, i64]),
+        "nvfp4_scale_atoms": (i32, [vp, i64, i64, vp, vp]),
+        "nvfp4_gemm": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -176,6 +180,21 @@ def nvfp4_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, t
     _check(LIB.nvfp4_quantize(_ptr(x), _dt(x.dtype), x.numel(), 1 if use_tensor_scale else 0, _ptr(codes),
                               _ptr(scales), _ptr(tensor_scale), _ptr(ws), ws.numel() * ws.element_size(),
                               _stream(stream)), "nvfp4_quantize")
+
+
+def nvfp4_scale_atoms_bytes(rows: int, K: int) -> int:
+    return int(LIB.nvfp4_scale_atoms_bytes(int(rows), int(K)))
+
+
+def nvfp4_scale_atoms(scales: torch.Tensor, rows: int, K: int, atoms: torch.Tensor, stream=None) -> None:
+    _check(LIB.nvfp4_scale_atoms(_ptr(scales), int(rows), int(K), _ptr(atoms), _stream(stream)), "nvfp4_scale_atoms")
+
+
+def nvfp4_gemm(a_codes: torch.Tensor, a_atoms: torch.Tensor, a_tensor_scale: torch.Tensor, b_codes: torch.Tensor,
+               b_atoms: torch.Tensor, b_tensor_scale: torch.Tensor, M: int, N: int, K: int, Y: torch.Tensor,
+               stream=None) -> None:
+    _check(LIB.nvfp4_gemm(_ptr(a_codes), _ptr(a_atoms), _ptr(a_tensor_scale), _ptr(b_codes), _ptr(b_atoms),
+                          _ptr(b_tensor_scale), int(M), int(N), int(K), _ptr(Y), _stream(stream)), "nvfp4_gemm")
 
 
 def mxfp4_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None) -> None:

@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libqlora_nf4.so")
-SOURCES = ["codebook.cu", "codec.cu", "gemm.cu", "lora_tc.cu", "smallm.cu", "mlp.cu", "fp4.cu", "adamw.cu", "trace.cu", "noalloc.cu", "diag.cu", "api.cu"]
+SOURCES = ["codebook.cu", "codec.cu", "gemm.cu", "lora_tc.cu", "smallm.cu", "mlp.cu", "fp4.cu", "fp4_gemm.cu", "adamw.cu", "trace.cu", "noalloc.cu", "diag.cu", "api.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "trace.cuh"]
 
 

@@ -53,6 +53,12 @@ ql_status launch_mxfp4_quantize(const void* x, ql_dtype dt, int64_t n, uint8_t* 
 ql_status launch_fp4_dequant(const uint8_t* codes, const uint8_t* scales, const float* ts, int64_t n, int fmt,
                              float* out, cudaStream_t st);
 unsigned status_word_fp4(cudaStream_t st);
+unsigned status_word_fp4g(cudaStream_t st);
+size_t nvfp4_atoms_bytes(int64_t rows, int64_t K);
+ql_status launch_nvfp4_atoms(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, cudaStream_t st);
+ql_status launch_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts, const uint8_t* b_codes,
+                            const uint8_t* b_atoms, const float* b_ts, int64_t M, int64_t N, int64_t K, float* Y,
+                            cudaStream_t st);
 // adamw.cu
 ql_status launch_adamw(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int64_t t, float lr,
                        float b1, float b2, float eps, float wd, cudaStream_t st);
@@ -303,6 +309,32 @@ ql_status mxfp4_dequant(const uint8_t* codes, const uint8_t* scales, int64_t n, 
   return ql::launch_fp4_dequant(codes, scales, nullptr, n, 1, out, as_stream(stream));
 }
 
+size_t nvfp4_scale_atoms_bytes(int64_t rows, int64_t K) {
+  if (rows < 1 || K < 64) return 0;
+  return ql::nvfp4_atoms_bytes(rows, K);
+}
+
+ql_status nvfp4_scale_atoms(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/nvfp4_scale_atoms");
+  if (rows < 1 || K < 1 || !aligned16(scales) || !aligned16(atoms)) return QL_ERR_INVALID_ARG;
+  if (K % 256 != 0 || rows >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31)) return QL_ERR_UNSUPPORTED;
+  return ql::launch_nvfp4_atoms(scales, rows, K, atoms, as_stream(stream));
+}
+
+ql_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_tensor_scale,
+                     const uint8_t* b_codes, const uint8_t* b_atoms, const float* b_tensor_scale, int64_t M,
+                     int64_t N, int64_t K, float* Y, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/nvfp4_gemm");
+  if (M < 1 || N < 1 || K < 1) return QL_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_atoms) || !aligned16(b_codes) || !aligned16(b_atoms) ||
+      !aligned16(Y) || !a_tensor_scale || !b_tensor_scale)
+    return QL_ERR_INVALID_ARG;
+  if (K % 256 != 0 || M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31))
+    return QL_ERR_UNSUPPORTED;
+  return ql::launch_nvfp4_gemm(a_codes, a_atoms, a_tensor_scale, b_codes, b_atoms, b_tensor_scale, M, N, K, Y,
+                               as_stream(stream));
+}
+
 ql_status qlora_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int64_t t, float lr,
                            float beta1, float beta2, float eps, float weight_decay, void* stream) {
   NvtxRange nvtx_range("qlora_nf4/qlora_adamw_step");
@@ -365,7 +397,8 @@ ql_status qlora_get_status(void* stream) {
   // one status word per translation unit that raises status bits
   unsigned v = 0;
   for (unsigned (*word)(cudaStream_t) : {ql::status_word_codec, ql::status_word_gemm, ql::status_word_lora,
-                                         ql::status_word_smallm, ql::status_word_diag, ql::status_word_fp4}) {
+                                         ql::status_word_smallm, ql::status_word_diag, ql::status_word_fp4,
+                                         ql::status_word_fp4g}) {
     const unsigned w = word(cs);
     if (w == ~0u) return QL_ERR_CUDA;
     v |= w;

@@ -1,0 +1,303 @@
+// NVFP4 x NVFP4 GEMM on the block-scaled tensor cores ("Lesson 4 of the
+// Finetuning Sessions", "From Turing to Blackwell": the 5th-generation tensor
+// cores execute the 4-bit block formats natively; "From FP32 to the 4-Bit
+// Horizon": NVFP4 is E2M1 elements with one E4M3 scale per 16 and an fp32
+// tensor scale):
+//   Y[m, n] = s_a s_b sum_k (E_a[m, k] S_a[m, k/16]) (E_b[n, k] S_b[n, k/16])
+// with E the E2M1 values, S the E4M3 block scales and s the tensor scales, for
+// operands quantized by nvfp4_quantize as row-major [rows, K] tensors (so a
+// block of 16 runs along K).
+//
+// One CTA per 128 x 128 output tile, cta_group::1:
+//   * warp 0, one thread: TMA of the A and B code tiles (128 rows x 256
+//     elements = 128 bytes per row, 128-byte swizzle) and a 1-D bulk copy of
+//     each operand's scale atoms for the stage, into a 4-stage ring;
+//   * warp 1, one thread: per 64-element K block, tcgen05.cp of the A and B
+//     scale atoms into TMEM (32 lanes x 128 bits, broadcast to the four lane
+//     quarters), then tcgen05.mma kind::mxf4nvf4 with 16-element scale blocks,
+//     accumulating in TMEM; a thread's tcgen05.cp and tcgen05.mma execute in
+//     issue order, so the same TMEM scale columns serve every stage;
+//   * warps 2-5: the 128 x 128 fp32 accumulator out of TMEM, times s_a s_b,
+//     into Y.
+// Scale atoms: the tensor cores take a 128-row block's scales for one
+// 64-element K block as 512 bytes, row m = m0 + 32 m1 (m0 < 32, m1 < 4) and
+// scale index kb < 4 at byte 16 m0 + 4 m1 + kb; nvfp4_scale_atoms writes the
+// row-major scales of nvfp4_quantize in that order, [row tile][K block][512].
+// Every wait is bounded: a lost arrival ends the kernel with QL_ERR_TIMEOUT.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "sm100.cuh"
+#include "trace.cuh"
+
+namespace ql {
+using namespace sm100;
+
+QL_DEFINE_STATUS_ACCESSOR(status_word_fp4g)
+
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
+                 uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+
+namespace fp4g {
+
+constexpr int BM = 128, BN = 128;
+constexpr int KS = 256;                                   // K elements per stage: 128 code bytes per row
+constexpr int KBLK = 64;                                  // K elements per MMA
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * KS / 2;                      // 16 KB
+constexpr int B_BYTES = BN * KS / 2;                      // 16 KB
+constexpr int SF_BYTES = (KS / KBLK) * 512;               // 2 KB of scale atoms per operand
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;
+constexpr int THREADS = 6 * 32;
+constexpr int TMEM_COLS = 256;                            // accumulator 0..127, scales 128..159
+constexpr int SFA_COL = 128, SFB_COL = 128 + 4 * (KS / KBLK);
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+
+// Instruction descriptor, kind::mxf4nvf4: E2M1 A and B (format 1), K-major,
+// N >> 3 at bit 17, M >> 4 at bit 24, E4M3 scales (bit 23 clear), K = 64,
+// scale-factor ids 0.
+constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+struct Params {
+  int M, N, K;
+  int ksteps;                 // K / KS
+  const uint8_t* sfa;         // scale atoms of A, [ceil(M/128)][K/64][512]
+  const uint8_t* sfb;         // scale atoms of B, [ceil(N/128)][K/64][512]
+  int64_t sf_tile_bytes;      // (K / 64) * 512
+  const float* sa;            // tensor scales (device)
+  const float* sb;
+  float* Y;                   // [M, N] fp32
+  uint32_t wait_limit;
+};
+
+// Global -> shared bulk copy completing on an mbarrier (no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Shared-memory matrix descriptor without swizzle, K-major core matrices of
+// 8 rows x 16 bytes: SBO = byte distance between 8-row groups.
+__device__ __forceinline__ uint64_t sdesc_plain(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  return d;
+}
+
+// One 512-byte scale atom (32 rows x 16 bytes in shared memory) into 4 TMEM
+// columns of all 128 lanes (each lane quarter receives the same 32 rows).
+__device__ __forceinline__ void tmem_cp_atom(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// D[tmem] (+)= (A * SFA)[smem] * (B * SFB)[smem]^T, kind::mxf4nvf4 with
+// 16-element scale blocks.
+__device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %6, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint32_t* tmem_addr = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<int*>(tmem_addr + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_addr, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_addr;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmap_a);
+      prefetch_tmap(&tmap_b);
+      const uint8_t* sfa = p.sfa + (int64_t)blockIdx.y * p.sf_tile_bytes;
+      const uint8_t* sfb = p.sfb + (int64_t)blockIdx.x * p.sf_tile_bytes;
+      int issued = 0;
+      for (int i = 0; i < p.ksteps; ++i) {
+        const int s = i % STAGES, use = i / STAGES;
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, abort_flag, p.wait_limit)) break;
+        uint8_t* st = base + s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+        tma_load_2d(st, &tmap_a, &full[s], i * (KS / 2), m0);
+        tma_load_2d(st + A_BYTES, &tmap_b, &full[s], i * (KS / 2), n0);
+        bulk_load(st + A_BYTES + B_BYTES, sfa + (int64_t)i * SF_BYTES, SF_BYTES, &full[s]);
+        bulk_load(st + A_BYTES + B_BYTES + SF_BYTES, sfb + (int64_t)i * SF_BYTES, SF_BYTES, &full[s]);
+        issued = i + 1;
+      }
+      // no copy may still be landing when the CTA exits
+      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+        mbar_wait(&full[i % STAGES], (i / STAGES) & 1, abort_flag, p.wait_limit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int i = 0; i < p.ksteps; ++i) {
+        const int s = i % STAGES, use = i / STAGES;
+        if (!mbar_wait(&full[s], use & 1, abort_flag, p.wait_limit)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(base + s * STAGE_BYTES);
+        const uint32_t b_addr = a_addr + A_BYTES;
+        const uint32_t sfa_addr = b_addr + B_BYTES, sfb_addr = sfa_addr + SF_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < KS / KBLK; ++kk) {
+          tmem_cp_atom(tmem + SFA_COL + 4 * kk, sdesc_plain(sfa_addr + 512 * kk, 16, 128));
+          tmem_cp_atom(tmem + SFB_COL + 4 * kk, sdesc_plain(sfb_addr + 512 * kk, 16, 128));
+        }
+#pragma unroll
+        for (int kk = 0; kk < KS / KBLK; ++kk) {
+          const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
+          mma_nvfp4(tmem, ad, bd, IDESC, tmem + SFA_COL + 4 * kk, tmem + SFB_COL + 4 * kk,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(acc_full);
+    }
+  } else {
+    // drain (warps 2-5): warp w reads TMEM lanes 32 (w % 4) .. +31, one output
+    // row per thread, 16 columns per load
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.wait_limit) && !*abort_flag);
+    const int quad = warp & 3;
+    const int row = m0 + quad * 32 + lane;
+    const float scale = __fmul_rn(*p.sa, *p.sb);
+    if (ok) {
+      tc_fence_after();
+      for (int c16 = 0; c16 < BN / 16; ++c16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(c16 * 16), v);
+        tmem_ld_wait();
+        if (row < p.M) {
+          float* y = p.Y + (size_t)row * p.N + n0 + c16 * 16;
+          const int left = p.N - (n0 + c16 * 16);
+          if (left >= 16 && (p.N & 3) == 0) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              reinterpret_cast<float4*>(y)[q] =
+                  make_float4(__fmul_rn(__uint_as_float(v[4 * q]), scale), __fmul_rn(__uint_as_float(v[4 * q + 1]), scale),
+                              __fmul_rn(__uint_as_float(v[4 * q + 2]), scale),
+                              __fmul_rn(__uint_as_float(v[4 * q + 3]), scale));
+          } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              if (q < left) y[q] = __fmul_rn(__uint_as_float(v[q]), scale);
+          }
+        }
+      }
+    }
+  }
+  if (warp == 1 && lane == 0 && *abort_flag) mbar_wait(acc_full, 0, abort_flag, p.wait_limit);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Row-major block scales [rows][K/16] -> scale atoms [ceil(rows/128)][K/64][512]
+// (zero for the rows past `rows` that pad the last tile).
+__global__ void __launch_bounds__(256) nvfp4_atoms_kernel(const uint8_t* __restrict__ sf, int64_t rows, int64_t K,
+                                                          uint8_t* __restrict__ out, int64_t total) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t kblocks = K / KBLK, per_row = K / 16;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t atom = idx >> 9;
+    const int within = (int)(idx & 511);
+    const int64_t t = atom / kblocks, q = atom % kblocks;
+    const int mm0 = within >> 4, m1 = (within >> 2) & 3, kb = within & 3;
+    const int64_t r = t * 128 + m1 * 32 + mm0;
+    out[idx] = r < rows ? sf[r * per_row + q * 4 + kb] : (uint8_t)0;
+  }
+}
+
+}  // namespace fp4g
+
+size_t nvfp4_atoms_bytes(int64_t rows, int64_t K) { return (size_t)((rows + 127) / 128) * (size_t)(K / 64) * 512; }
+
+ql_status launch_nvfp4_atoms(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, cudaStream_t st) {
+  const int64_t total = (int64_t)nvfp4_atoms_bytes(rows, K);
+  const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, (int64_t)sms * 8));
+  TraceScope ts(TK_FP4, st);
+  QL_CUDA_TRY(launch(fp4g::nvfp4_atoms_kernel, dim3(grid), dim3(256), 0, st, 1, 1, scales, rows, K, atoms, total));
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
+ql_status launch_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts, const uint8_t* b_codes,
+                            const uint8_t* b_atoms, const float* b_ts, int64_t M, int64_t N, int64_t K, float* Y,
+                            cudaStream_t st) {
+  using namespace fp4g;
+  if (per_device(reinterpret_cast<const void*>(nvfp4_gemm_kernel), 0, [] {
+        if (cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+            cudaSuccess) {
+          cudaGetLastError();
+          return -1;
+        }
+        return 1;
+      }) < 0)
+    return QL_ERR_CUDA;
+  CUtensorMap map_a, map_b;
+  if (!make_map_2d(&map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
+                   KS / 2, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                   KS / 2, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QL_ERR_CUDA;
+  Params p;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.ksteps = (int)(K / KS);
+  p.sfa = a_atoms;
+  p.sfb = b_atoms;
+  p.sf_tile_bytes = (K / KBLK) * 512;
+  p.sa = a_ts;
+  p.sb = b_ts;
+  p.Y = Y;
+  p.wait_limit = 1u << 22;
+  const dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  TraceScope ts(TK_FP4GEMM, st);
+  QL_CUDA_TRY(launch(nvfp4_gemm_kernel, grid, dim3(THREADS), SMEM_BYTES, st, 1, 1, map_a, map_b, p));
+  QL_LAUNCH_CHECK();
+  return QL_OK;
+}
+
+}  // namespace ql

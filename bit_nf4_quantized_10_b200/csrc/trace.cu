@@ -21,7 +21,7 @@ std::vector<cudaEvent_t> g_free;
 const char* const kNames[TK_COUNT] = {"nf4_quantize",   "dq_tree_sum",    "dq_encode",       "nf4_dequant",
                                       "qlora_gemm_fwd", "qlora_gemm_bwd", "lora_side_proj", "lora_grad",
                                       "lora_grad_reduce", "silu_gate",    "smallm_splitk",   "lora_transpose",
-                                      "adapter_merge", "fp4_codec",     "adamw_step"};
+                                      "adapter_merge", "fp4_codec",     "adamw_step",      "nvfp4_gemm"};
 }  // namespace
 
 const char* trace_name(int kind) { return (kind >= 0 && kind < TK_COUNT) ? kNames[kind] : "unknown"; }

@@ -26,6 +26,7 @@ enum TraceKind : int {
   TK_MERGE,
   TK_FP4,
   TK_ADAMW,
+  TK_FP4GEMM,
   TK_COUNT
 };
 

@@ -311,6 +311,38 @@ ql_status nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const float
 ql_status mxfp4_dequant(const uint8_t* codes, const uint8_t* scales, int64_t n, float* out, void* stream);
 
 /*
+ * NVFP4 x NVFP4 GEMM on the block-scaled tensor cores ([P1] "Lesson 4 of the
+ * Finetuning Sessions", "From Turing to Blackwell": the 5th-generation tensor
+ * cores execute the 4-bit block formats natively; "From FP32 to the 4-Bit
+ * Horizon": E2M1 elements, one E4M3 scale per 16, one fp32 tensor scale):
+ *   Y[m, n] = s_a s_b sum_k (E2M1(a[m, k]) S_a[m, k/16]) (E2M1(b[n, k]) S_b[n, k/16])
+ * for A [M, K] and B [N, K] row-major, each quantized by nvfp4_quantize as one
+ * tensor of rows x K elements (so each block of 16 runs along K).  This is
+ * W4A4: both operands are 4-bit, not the QLoRA linear's bf16 activations.
+ *
+ * nvfp4_scale_atoms: scales device uint8 [rows * K/16] (row-major, as
+ *   nvfp4_quantize writes them) -> atoms device out uint8
+ *   [nvfp4_scale_atoms_bytes(rows, K)]: per 128-row tile and 64-element K
+ *   block, 512 bytes with row m = m0 + 32 m1 (m0 < 32, m1 < 4) and scale kb < 4
+ *   at byte 16 m0 + 4 m1 + kb (the tensor cores' scale layout); rows past
+ *   `rows` in the last tile are 0.
+ * nvfp4_gemm: a_codes / b_codes device uint8 [M * K/2] / [N * K/2]; a_atoms /
+ *   b_atoms from nvfp4_scale_atoms with rows = M / N; a_tensor_scale /
+ *   b_tensor_scale device fp32 [1]; Y device out fp32 [M, N] row-major.  The
+ *   products are exact and accumulate in fp32 on the tensor cores (order
+ *   unspecified); then Y = fl32(acc fl32(s_a s_b)).
+ * Constraints: K a multiple of 256; M, N, K < 2^31.  Errors:
+ * QL_ERR_INVALID_ARG (M, N or K < 1, a NULL or misaligned pointer),
+ * QL_ERR_UNSUPPORTED (K % 256 != 0, sizes of 2^31 or more), QL_ERR_CUDA.
+ * A bounded wait that runs out sets QL_ERR_TIMEOUT in the status word.
+ */
+size_t nvfp4_scale_atoms_bytes(int64_t rows, int64_t K);
+ql_status nvfp4_scale_atoms(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, void* stream);
+ql_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_tensor_scale,
+                     const uint8_t* b_codes, const uint8_t* b_atoms, const float* b_tensor_scale, int64_t M,
+                     int64_t N, int64_t K, float* Y, void* stream);
+
+/*
  * qlora_adamw_step — one AdamW update of adapter parameters with fp32 states
  * (the paged optimizer: [P2] §2.3 and [P3] "Paged optimizers: surviving the
  * spikes" keep the states in unified memory, paged to host RAM under memory

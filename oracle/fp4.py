@@ -129,6 +129,21 @@ def nvfp4_dequant(codes, S, s_t: float, n: int) -> np.ndarray:
     return fl32(v * scale[np.arange(n) // NV_BLOCK])
 
 
+def nvfp4_gemm(a_codes, a_S, a_st: float, b_codes, b_S, b_st: float, M: int, N: int, K: int) -> np.ndarray:
+    """Y = A_hat B_hat^T in float64, A [M, K] and B [N, K] row-major NVFP4
+    tensors dequantized by nvfp4_dequant.
+
+    [P1] "Lesson 4 of the Finetuning Sessions", "From Turing to Blackwell": the
+    5th-generation tensor cores multiply the 4-bit block formats natively, each
+    element times its block scale (and the tensor scale), accumulating the
+    products.  Reading: the exact value of that product is the product of the
+    dequantized tensors; the kernel's fp32 accumulation order is unspecified, so
+    parity is within a tolerance."""
+    A = nvfp4_dequant(a_codes, a_S, a_st, M * K).reshape(M, K)
+    B = nvfp4_dequant(b_codes, b_S, b_st, N * K).reshape(N, K)
+    return A @ B.T
+
+
 def storage_bits_per_element(fmt: str) -> float:
     """Bits per element including the block scales (MX: 8 per 32; NV: 8 per 16;
     the single NVFP4 tensor scale is not counted)."""

@@ -107,6 +107,15 @@ def test_argument_errors_return_before_launch(lib):
     assert adam(16, 1, 0.9, -0.5, 1e-8) == lib.QL_ERR_INVALID_ARG
     assert adam(16, 1, 0.9, 0.999, -1.0) == lib.QL_ERR_INVALID_ARG
     assert adam(16, 1, 0.9, 0.999, 1e-8, g=fake + 4) == lib.QL_ERR_INVALID_ARG
+    g = lambda M, N, K, a=fake, y=fake: L.nvfp4_gemm(a, fake, fake, fake, fake, fake, M, N, K, y, s0)
+    assert g(0, 128, 256) == lib.QL_ERR_INVALID_ARG
+    assert g(128, 128, 256, a=None) == lib.QL_ERR_INVALID_ARG
+    assert g(128, 128, 256, y=fake + 4) == lib.QL_ERR_INVALID_ARG
+    assert g(128, 128, 320) == lib.QL_ERR_UNSUPPORTED                                       # K % 256
+    assert g(1 << 31, 128, 256) == lib.QL_ERR_UNSUPPORTED
+    assert L.nvfp4_scale_atoms(fake, 0, 256, fake, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.nvfp4_scale_atoms(fake, 128, 192, fake, s0) == lib.QL_ERR_UNSUPPORTED
+    assert L.nvfp4_scale_atoms(fake + 8, 128, 256, fake, s0) == lib.QL_ERR_INVALID_ARG
     assert L.qlora_paged_prefetch(None, 64, lib.QL_PAGE_HOST, s0) == lib.QL_ERR_INVALID_ARG
     assert L.qlora_paged_prefetch(fake, 0, lib.QL_PAGE_HOST, s0) == lib.QL_ERR_INVALID_ARG
     assert L.qlora_paged_prefetch(fake, 64, 5, s0) == lib.QL_ERR_INVALID_ARG
@@ -150,3 +159,11 @@ def test_workspace_sizes_follow_the_documented_layout(lib, M, N, K, r):
     want = a256(r * N * 2) + a256(r * Mp * 2) + a256(M * r * 2) + a256(r * Mp * 2)
     assert lib.qlora_workspace_size(lib.QL_OP_BWD, M, N, K, r) == want
     assert lib.qlora_workspace_size(lib.QL_OP_BWD, M, N, K, 0) == 0
+
+
+def test_nvfp4_scale_atom_sizes(lib):
+    """One 512-byte atom per 128-row tile and 64-element block of K."""
+    assert lib.nvfp4_scale_atoms_bytes(128, 256) == 4 * 512
+    assert lib.nvfp4_scale_atoms_bytes(129, 256) == 2 * 4 * 512       # a partial tile is padded
+    assert lib.nvfp4_scale_atoms_bytes(28672, 8192) == 224 * 128 * 512
+    assert lib.nvfp4_scale_atoms_bytes(0, 256) == 0

@@ -121,3 +121,41 @@ def test_nvfp4_tensor_scale_power_of_two_invariance():
 def test_storage_bits():
     assert fp4.storage_bits_per_element("mxfp4") == 4.25
     assert fp4.storage_bits_per_element("nvfp4") == 4.5
+
+
+def test_nvfp4_gemm_closed_form():
+    """Every element one E2M1 value under one scale: Y = K (v_a S_a s_a)(v_b S_b s_b) exactly."""
+    M, N, K = 3, 5, 64
+    code_one = fp4.e2m1_encode(np.array([1.5]))[0]        # +1.5
+    code_neg = fp4.e2m1_encode(np.array([-3.0]))[0]       # -3
+    a = np.full(M * K, code_one, dtype=np.uint8)
+    b = np.full(N * K, code_neg, dtype=np.uint8)
+    Sa = np.full(M * K // 16, 2.0)
+    Sb = np.full(N * K // 16, 0.5)
+    Y = fp4.nvfp4_gemm(a, Sa, 0.25, b, Sb, 4.0, M, N, K)
+    assert Y.shape == (M, N)
+    assert np.all(Y == K * (1.5 * 2.0 * 0.25) * (-3.0 * 0.5 * 4.0))
+
+
+def test_nvfp4_gemm_exact_rational_bruteforce():
+    """A small random case against a sum of exact rationals, element by element:
+    the dequantized values are fp32 numbers, so their products and sums are
+    exact as fractions; float64 with K = 32 terms is within a few ulp."""
+    from fractions import Fraction
+    rng = np.random.default_rng(7)
+    M, N, K = 4, 3, 32
+    xa = rng.standard_normal((M, K))
+    xb = rng.standard_normal((N, K)) * 0.02
+    ca, Sa, sta = fp4.nvfp4_quantize(xa.reshape(-1))
+    cb, Sb, stb = fp4.nvfp4_quantize(xb.reshape(-1))
+    Y = fp4.nvfp4_gemm(ca, Sa, sta, cb, Sb, stb, M, N, K)
+    A = fp4.nvfp4_dequant(ca, Sa, sta, M * K).reshape(M, K)
+    B = fp4.nvfp4_dequant(cb, Sb, stb, N * K).reshape(N, K)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(A[m, k])) * Fraction(float(B[n, k])) for k in range(K))
+            assert abs(Fraction(float(Y[m, n])) - exact) <= abs(exact) * Fraction(1, 2 ** 48) + Fraction(1, 2 ** 80)
+    # and the dequantized values are the codes times the block scale times the tensor scale
+    v = fp4.e2m1_decode(ca).reshape(M, K)
+    scale = np.repeat(np.asarray(Sa, dtype=np.float64), 16).reshape(M, K) * sta
+    assert np.allclose(A, v * scale, rtol=2 ** -22, atol=0)
