@@ -520,6 +520,7 @@ def secondary_legs(q, dev, hbm_peak, bf16_peak, peak_src, layer_set):
                               "gemm_traffic": rf["traffic"]}
     del proj
     torch.cuda.empty_cache()
+    out.update(fp4_gemm_leg(q, dev, flush, bf16_peak, layer_set))
     out.update(mlp_leg(q, dev, flush))
     out.update(small_m_and_codec(q, dev, hbm_peak, flush))
     out.update(adamw_leg(q, dev, hbm_peak, layer_set, flush))
@@ -547,6 +548,50 @@ def dense_context_leg(layer_set, flush, t_nf4):
         "ms": round(t * 1e3, 3), "TFLOPs": round(flop / t / 1e12, 1),
         "what": "Y = X W^T and dX = dY W per linear, bf16 dense weights, torch.matmul (context only)",
         "nf4_fwd_bwd_over_dense": round(t_nf4 / t, 3)}}
+
+
+def fp4_gemm_leg(q, dev, flush, bf16_peak, layer_set):
+    """The next row's native 4-bit product: the gate linear's shape (2048
+    tokens x 28672 x 8192) as an NVFP4 x NVFP4 GEMM on the block-scaled tensor
+    cores (both operands quantized by nvfp4_quantize from the layer's bf16
+    tensors), beside the NF4 path's forward GEMM on the same shape (no
+    adapter).  The FP4 peak is the measured bf16 peak times the nominal 4x."""
+    import torch
+    it = layer_set.items[4]
+    M, N, K = layer_set.M, it["N"], it["K"]
+
+    def operand(x, rows):
+        n = x.numel()
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        sc = torch.empty(n // 16, dtype=torch.uint8, device=dev)
+        ts = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(max(256, q.qlora_workspace_size(q.QL_OP_NVFP4, n)), dtype=torch.uint8, device=dev)
+        q.nvfp4_quantize(x, codes, sc, ts, ws)
+        atoms = torch.empty(q.nvfp4_scale_atoms_bytes(rows, K), dtype=torch.uint8, device=dev)
+        q.nvfp4_scale_atoms(sc, rows, K, atoms)
+        return codes, atoms, ts
+
+    a, b = operand(it["X"], M), operand(it["W"], N)
+    Y = torch.empty(M, N, dtype=torch.float32, device=dev)
+    t = _time_calls(lambda: q.nvfp4_gemm(a[0], a[1], a[2], b[0], b[1], b[2], M, N, K, Y), flush, n_warm=3, n=10)
+    flop = 2.0 * M * N * K
+    Yb = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(16, q.qlora_workspace_size(q.QL_OP_FWD, M, N, K, 0)), dtype=torch.uint8, device=dev)
+    A0 = torch.empty(0, K, dtype=torch.bfloat16, device=dev)
+    B0 = torch.empty(N, 0, dtype=torch.bfloat16, device=dev)
+    t_nf4 = _time_calls(lambda: q.qlora_linear_fwd(it["wq"], it["X"], A0, B0, 0, 1.0, Yb, ws=ws), flush, n_warm=3, n=10)
+    st = q.qlora_get_status()
+    if st != q.QL_OK:
+        raise RuntimeError(f"device status: {q.status_string(st)}")
+    peak = 4 * bf16_peak
+    res = {"nvfp4_gemm_gate_shape": {"us": round(t * 1e6, 2), "TFLOPs": round(flop / t / 1e12, 1),
+                                     "frac_fp4_peak": round(flop / t / 1e12 / peak, 3),
+                                     "fp4_peak_TFLOPs": round(peak, 1), "shape": [M, N, K],
+                                     "nf4_fwd_same_shape_us": round(t_nf4 * 1e6, 2),
+                                     "speedup_over_nf4_fwd": round(t_nf4 / t, 2)}}
+    del a, b, Y, Yb
+    torch.cuda.empty_cache()
+    return res
 
 
 def mlp_leg(q, dev, flush):

@@ -329,7 +329,7 @@ ql_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const float
   if (!aligned16(a_codes) || !aligned16(a_atoms) || !aligned16(b_codes) || !aligned16(b_atoms) ||
       !aligned16(Y) || !a_tensor_scale || !b_tensor_scale)
     return QL_ERR_INVALID_ARG;
-  if (K % 256 != 0 || M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31))
+  if (K % 256 != 0 || M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 23) || K >= ((int64_t)1 << 31))
     return QL_ERR_UNSUPPORTED;
   return ql::launch_nvfp4_gemm(a_codes, a_atoms, a_tensor_scale, b_codes, b_atoms, b_tensor_scale, M, N, K, Y,
                                as_stream(stream));

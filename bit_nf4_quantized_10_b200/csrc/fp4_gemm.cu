@@ -8,17 +8,19 @@
 // operands quantized by nvfp4_quantize as row-major [rows, K] tensors (so a
 // block of 16 runs along K).
 //
-// One CTA per 128 x 128 output tile, cta_group::1:
+// One CTA per 128 x 128 output tile, cta_group::1, the token (M) tiles
+// fastest so that the CTAs resident at once share a few weight (N) tiles in L2:
 //   * warp 0, one thread: TMA of the A and B code tiles (128 rows x 256
 //     elements = 128 bytes per row, 128-byte swizzle) and a 1-D bulk copy of
-//     each operand's scale atoms for the stage, into a 4-stage ring;
+//     each operand's scale atoms for the stage, into a 3-stage ring (two CTAs
+//     fit on an SM, so one's drain overlaps the other's main loop);
 //   * warp 1, one thread: per 64-element K block, tcgen05.cp of the A and B
 //     scale atoms into TMEM (32 lanes x 128 bits, broadcast to the four lane
 //     quarters), then tcgen05.mma kind::mxf4nvf4 with 16-element scale blocks,
 //     accumulating in TMEM; a thread's tcgen05.cp and tcgen05.mma execute in
 //     issue order, so the same TMEM scale columns serve every stage;
 //   * warps 2-5: the 128 x 128 fp32 accumulator out of TMEM, times s_a s_b,
-//     into Y.
+//     staged in shared memory and written to Y a row per store instruction.
 // Scale atoms: the tensor cores take a 128-row block's scales for one
 // 64-element K block as 512 bytes, row m = m0 + 32 m1 (m0 < 32, m1 < 4) and
 // scale index kb < 4 at byte 16 m0 + 4 m1 + kb; nvfp4_scale_atoms writes the
@@ -45,7 +47,7 @@ namespace fp4g {
 constexpr int BM = 128, BN = 128;
 constexpr int KS = 256;                                   // K elements per stage: 128 code bytes per row
 constexpr int KBLK = 64;                                  // K elements per MMA
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;                                 // 109 KB: two CTAs per SM
 constexpr int A_BYTES = BM * KS / 2;                      // 16 KB
 constexpr int B_BYTES = BN * KS / 2;                      // 16 KB
 constexpr int SF_BYTES = (KS / KBLK) * 512;               // 2 KB of scale atoms per operand
@@ -109,7 +111,7 @@ __device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_addr = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<int*>(tmem_addr + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;   // token tiles fastest: resident CTAs share B tiles in L2
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -146,8 +148,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       prefetch_tmap(&tmap_a);
       prefetch_tmap(&tmap_b);
-      const uint8_t* sfa = p.sfa + (int64_t)blockIdx.y * p.sf_tile_bytes;
-      const uint8_t* sfb = p.sfb + (int64_t)blockIdx.x * p.sf_tile_bytes;
+      const uint8_t* sfa = p.sfa + (int64_t)blockIdx.x * p.sf_tile_bytes;
+      const uint8_t* sfb = p.sfb + (int64_t)blockIdx.y * p.sf_tile_bytes;
       int issued = 0;
       for (int i = 0; i < p.ksteps; ++i) {
         const int s = i % STAGES, use = i / STAGES;
@@ -190,33 +192,43 @@ __global__ void __launch_bounds__(THREADS, 1)
       mma_commit(acc_full);
     }
   } else {
-    // drain (warps 2-5): warp w reads TMEM lanes 32 (w % 4) .. +31, one output
-    // row per thread, 16 columns per load
+    // drain (warps 2-5): warp w reads TMEM lanes 32 (w % 4) .. +31 (one output
+    // row per thread, 16 columns per load), scales them and stages its
+    // 32 x 128 block in the idle stage buffers (row pitch 132 floats keeps the
+    // 16-byte writes conflict-free), then writes it a row at a time: 32 lanes x
+    // 16 bytes, one contiguous 512-byte row per store instruction.
     const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.wait_limit) && !*abort_flag);
     const int quad = warp & 3;
-    const int row = m0 + quad * 32 + lane;
     const float scale = __fmul_rn(*p.sa, *p.sb);
+    constexpr int PITCH = BN + 4;
+    float* stage_out = reinterpret_cast<float*>(base) + quad * 32 * PITCH;
     if (ok) {
       tc_fence_after();
       for (int c16 = 0; c16 < BN / 16; ++c16) {
         uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(c16 * 16), v);
         tmem_ld_wait();
-        if (row < p.M) {
-          float* y = p.Y + (size_t)row * p.N + n0 + c16 * 16;
-          const int left = p.N - (n0 + c16 * 16);
-          if (left >= 16 && (p.N & 3) == 0) {
+        float4* dst = reinterpret_cast<float4*>(stage_out + lane * PITCH + c16 * 16);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              reinterpret_cast<float4*>(y)[q] =
-                  make_float4(__fmul_rn(__uint_as_float(v[4 * q]), scale), __fmul_rn(__uint_as_float(v[4 * q + 1]), scale),
-                              __fmul_rn(__uint_as_float(v[4 * q + 2]), scale),
-                              __fmul_rn(__uint_as_float(v[4 * q + 3]), scale));
-          } else {
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_float4(__fmul_rn(__uint_as_float(v[4 * q]), scale), __fmul_rn(__uint_as_float(v[4 * q + 1]), scale),
+                               __fmul_rn(__uint_as_float(v[4 * q + 2]), scale),
+                               __fmul_rn(__uint_as_float(v[4 * q + 3]), scale));
+      }
+      __syncwarp();
+      const int col = n0 + 4 * lane;
+      for (int rr = 0; rr < 32; ++rr) {
+        const int row = m0 + quad * 32 + rr;
+        if (row >= p.M) break;
+        const float4 val = *reinterpret_cast<const float4*>(stage_out + rr * PITCH + 4 * lane);
+        float* y = p.Y + (size_t)row * p.N + col;
+        if ((p.N & 3) == 0 && col + 4 <= p.N) {
+          *reinterpret_cast<float4*>(y) = val;
+        } else {
+          const float e[4] = {val.x, val.y, val.z, val.w};
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-              if (q < left) y[q] = __fmul_rn(__uint_as_float(v[q]), scale);
-          }
+          for (int q = 0; q < 4; ++q)
+            if (col + q < p.N) y[q] = e[q];
         }
       }
     }
@@ -268,7 +280,9 @@ ql_status launch_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, cons
   using namespace fp4g;
   if (per_device(reinterpret_cast<const void*>(nvfp4_gemm_kernel), 0, [] {
         if (cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
-            cudaSuccess) {
+                cudaSuccess ||
+            cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+                cudaSuccess) {
           cudaGetLastError();
           return -1;
         }
@@ -293,7 +307,7 @@ ql_status launch_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, cons
   p.sb = b_ts;
   p.Y = Y;
   p.wait_limit = 1u << 22;
-  const dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  const dim3 grid((unsigned)((M + BM - 1) / BM), (unsigned)((N + BN - 1) / BN));
   TraceScope ts(TK_FP4GEMM, st);
   QL_CUDA_TRY(launch(nvfp4_gemm_kernel, grid, dim3(THREADS), SMEM_BYTES, st, 1, 1, map_a, map_b, p));
   QL_LAUNCH_CHECK();

@@ -331,9 +331,9 @@ ql_status mxfp4_dequant(const uint8_t* codes, const uint8_t* scales, int64_t n, 
  *   b_tensor_scale device fp32 [1]; Y device out fp32 [M, N] row-major.  The
  *   products are exact and accumulate in fp32 on the tensor cores (order
  *   unspecified); then Y = fl32(acc fl32(s_a s_b)).
- * Constraints: K a multiple of 256; M, N, K < 2^31.  Errors:
+ * Constraints: K a multiple of 256; M, K < 2^31; N < 2^23.  Errors:
  * QL_ERR_INVALID_ARG (M, N or K < 1, a NULL or misaligned pointer),
- * QL_ERR_UNSUPPORTED (K % 256 != 0, sizes of 2^31 or more), QL_ERR_CUDA.
+ * QL_ERR_UNSUPPORTED (K % 256 != 0, sizes past the constraints), QL_ERR_CUDA.
  * A bounded wait that runs out sets QL_ERR_TIMEOUT in the status word.
  */
 size_t nvfp4_scale_atoms_bytes(int64_t rows, int64_t K);

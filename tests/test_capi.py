@@ -113,6 +113,7 @@ def test_argument_errors_return_before_launch(lib):
     assert g(128, 128, 256, y=fake + 4) == lib.QL_ERR_INVALID_ARG
     assert g(128, 128, 320) == lib.QL_ERR_UNSUPPORTED                                       # K % 256
     assert g(1 << 31, 128, 256) == lib.QL_ERR_UNSUPPORTED
+    assert g(128, 1 << 23, 256) == lib.QL_ERR_UNSUPPORTED
     assert L.nvfp4_scale_atoms(fake, 0, 256, fake, s0) == lib.QL_ERR_INVALID_ARG
     assert L.nvfp4_scale_atoms(fake, 128, 192, fake, s0) == lib.QL_ERR_UNSUPPORTED
     assert L.nvfp4_scale_atoms(fake + 8, 128, 256, fake, s0) == lib.QL_ERR_INVALID_ARG
