@@ -46,7 +46,7 @@ def parse():
     p.add_argument("--no-secondary", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
-    p.add_argument("--leg", choices=["layer", "projection", "smallm", "codec", "merge"], default="layer",
+    p.add_argument("--leg", choices=["layer", "projection", "smallm", "codec", "merge", "fp4gemm"], default="layer",
                    help="with --profile: which workload to run")
     p.add_argument("--profile", action="store_true",
                    help="fixed launch sequence for profilers: exactly --warmup then --steps steps of --leg, "
@@ -752,7 +752,8 @@ def profile_leg(args, q, dev):
     measured step (one stream); projection = the 4096^2 step; smallm = the
     16-token forward on the 28672 x 8192 weight; merge = the adapter merge of
     that weight (bf16 output and re-quantized codes); codec = quantize + double
-    quant of 256 Mi bf16 elements.  Prints per-call device times."""
+    quant of 256 Mi bf16 elements; fp4gemm = the NVFP4 x NVFP4 GEMM at
+    2048 x 4096 x 8192.  Prints per-call device times."""
     import torch
     from synthetic import inputs as S
     w5 = S.WORKLOADS["c5"]
@@ -772,6 +773,23 @@ def profile_leg(args, q, dev):
         codes_out = torch.empty(N * K // 2, dtype=torch.uint8, device=dev)
         absmax_out = torch.empty(N * K // 64, dtype=torch.float32, device=dev)
         call = lambda: q.qlora_merge(wq, A, B, r, w5.s, W_out=W_out, codes_out=codes_out, absmax_out=absmax_out)
+    elif args.leg == "fp4gemm":
+        # NVFP4 x NVFP4 on the block-scaled tensor cores, 2048 x 4096 x 8192
+        M, N, K = 2048, 4096, 8192
+        fp = []
+        for rows, std, seed in ((M, 1.0, 950), (N, 0.015, 951)):
+            x = S.normal((rows, K), std, seed, device=dev, dtype=torch.bfloat16)
+            codes = torch.empty(rows * K // 2, dtype=torch.uint8, device=dev)
+            sc = torch.empty(rows * K // 16, dtype=torch.uint8, device=dev)
+            ts = torch.empty(1, dtype=torch.float32, device=dev)
+            ws = torch.empty(max(256, q.qlora_workspace_size(q.QL_OP_NVFP4, rows * K)), dtype=torch.uint8, device=dev)
+            q.nvfp4_quantize(x, codes, sc, ts, ws)
+            atoms = torch.empty(q.nvfp4_scale_atoms_bytes(rows, K), dtype=torch.uint8, device=dev)
+            q.nvfp4_scale_atoms(sc, rows, K, atoms)
+            fp.append((codes, atoms, ts))
+        Yf = torch.empty(M, N, dtype=torch.float32, device=dev)
+        (ac, aa, at), (bc, ba, bt) = fp
+        call = lambda: q.nvfp4_gemm(ac, aa, at, bc, ba, bt, M, N, K, Yf)
     elif args.leg == "smallm":
         lin = w5.linears[0]
         N, K, r, s, M = lin.N, lin.K, w5.r, w5.s, 16
