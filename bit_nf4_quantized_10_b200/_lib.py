@@ -26,7 +26,7 @@ EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_double_quant_noalloc", "nf4_
            "nf4_codebook", "qlora_get_status", "qlora_status_string", "qlora_selftest_wait_timeout",
            "qlora_merge", "nf4_double_quant_level1", "nf4_double_quant_finish", "nvfp4_quantize", "mxfp4_quantize",
            "nvfp4_dequant", "mxfp4_dequant", "qlora_adamw_step", "qlora_paged_prefetch", "nvfp4_scale_atoms_bytes",
-           "nvfp4_scale_atoms", "nvfp4_gemm")
+           "nvfp4_scale_atoms", "nvfp4_gemm", "mxfp4_scale_atoms_bytes", "mxfp4_scale_atoms", "mxfp4_gemm")
 
 
 class QLoraError(RuntimeError):
@@ -74,6 +74,9 @@ def _load() -> ctypes.CDLL:
         "nvfp4_scale_atoms_bytes": (sz, [i64, i64]),
         "nvfp4_scale_atoms": (i32, [vp, i64, i64, vp, vp]),
         "nvfp4_gemm": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]),
+        "mxfp4_scale_atoms_bytes": (sz, [i64, i64]),
+        "mxfp4_scale_atoms": (i32, [vp, i64, i64, vp, vp]),
+        "mxfp4_gemm": (i32, [vp, vp, vp, vp, i64, i64, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -195,6 +198,20 @@ def nvfp4_gemm(a_codes: torch.Tensor, a_atoms: torch.Tensor, a_tensor_scale: tor
                stream=None) -> None:
     _check(LIB.nvfp4_gemm(_ptr(a_codes), _ptr(a_atoms), _ptr(a_tensor_scale), _ptr(b_codes), _ptr(b_atoms),
                           _ptr(b_tensor_scale), int(M), int(N), int(K), _ptr(Y), _stream(stream)), "nvfp4_gemm")
+
+
+def mxfp4_scale_atoms_bytes(rows: int, K: int) -> int:
+    return int(LIB.mxfp4_scale_atoms_bytes(int(rows), int(K)))
+
+
+def mxfp4_scale_atoms(scales: torch.Tensor, rows: int, K: int, atoms: torch.Tensor, stream=None) -> None:
+    _check(LIB.mxfp4_scale_atoms(_ptr(scales), int(rows), int(K), _ptr(atoms), _stream(stream)), "mxfp4_scale_atoms")
+
+
+def mxfp4_gemm(a_codes: torch.Tensor, a_atoms: torch.Tensor, b_codes: torch.Tensor, b_atoms: torch.Tensor, M: int,
+               N: int, K: int, Y: torch.Tensor, stream=None) -> None:
+    _check(LIB.mxfp4_gemm(_ptr(a_codes), _ptr(a_atoms), _ptr(b_codes), _ptr(b_atoms), int(M), int(N), int(K),
+                          _ptr(Y), _stream(stream)), "mxfp4_gemm")
 
 
 def mxfp4_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None) -> None:

@@ -54,11 +54,11 @@ ql_status launch_fp4_dequant(const uint8_t* codes, const uint8_t* scales, const 
                              float* out, cudaStream_t st);
 unsigned status_word_fp4(cudaStream_t st);
 unsigned status_word_fp4g(cudaStream_t st);
-size_t nvfp4_atoms_bytes(int64_t rows, int64_t K);
-ql_status launch_nvfp4_atoms(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, cudaStream_t st);
-ql_status launch_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts, const uint8_t* b_codes,
-                            const uint8_t* b_atoms, const float* b_ts, int64_t M, int64_t N, int64_t K, float* Y,
-                            cudaStream_t st);
+size_t fp4_atoms_bytes(int64_t rows, int64_t K, int vs);
+ql_status launch_fp4_atoms(const uint8_t* scales, int64_t rows, int64_t K, int vs, uint8_t* atoms, cudaStream_t st);
+ql_status launch_fp4_gemm(int vs, const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts,
+                          const uint8_t* b_codes, const uint8_t* b_atoms, const float* b_ts, int64_t M, int64_t N,
+                          int64_t K, float* Y, cudaStream_t st);
 // adamw.cu
 ql_status launch_adamw(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int64_t t, float lr,
                        float b1, float b2, float eps, float wd, cudaStream_t st);
@@ -311,28 +311,53 @@ ql_status mxfp4_dequant(const uint8_t* codes, const uint8_t* scales, int64_t n, 
 
 size_t nvfp4_scale_atoms_bytes(int64_t rows, int64_t K) {
   if (rows < 1 || K < 64) return 0;
-  return ql::nvfp4_atoms_bytes(rows, K);
+  return ql::fp4_atoms_bytes(rows, K, 16);
+}
+
+size_t mxfp4_scale_atoms_bytes(int64_t rows, int64_t K) {
+  if (rows < 1 || K < 128) return 0;
+  return ql::fp4_atoms_bytes(rows, K, 32);
+}
+
+static ql_status fp4_scale_atoms(const uint8_t* scales, int64_t rows, int64_t K, int vs, uint8_t* atoms, void* stream) {
+  if (rows < 1 || K < 1 || !aligned16(scales) || !aligned16(atoms)) return QL_ERR_INVALID_ARG;
+  if (K % 256 != 0 || rows >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31)) return QL_ERR_UNSUPPORTED;
+  return ql::launch_fp4_atoms(scales, rows, K, vs, atoms, as_stream(stream));
 }
 
 ql_status nvfp4_scale_atoms(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, void* stream) {
   NvtxRange nvtx_range("qlora_nf4/nvfp4_scale_atoms");
-  if (rows < 1 || K < 1 || !aligned16(scales) || !aligned16(atoms)) return QL_ERR_INVALID_ARG;
-  if (K % 256 != 0 || rows >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31)) return QL_ERR_UNSUPPORTED;
-  return ql::launch_nvfp4_atoms(scales, rows, K, atoms, as_stream(stream));
+  return fp4_scale_atoms(scales, rows, K, 16, atoms, stream);
+}
+
+ql_status mxfp4_scale_atoms(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/mxfp4_scale_atoms");
+  return fp4_scale_atoms(scales, rows, K, 32, atoms, stream);
+}
+
+static ql_status fp4_gemm_checked(int vs, const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_ts,
+                                  const uint8_t* b_codes, const uint8_t* b_atoms, const float* b_ts, int64_t M,
+                                  int64_t N, int64_t K, float* Y, void* stream) {
+  if (M < 1 || N < 1 || K < 1) return QL_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_atoms) || !aligned16(b_codes) || !aligned16(b_atoms) || !aligned16(Y))
+    return QL_ERR_INVALID_ARG;
+  if (vs == 16 && (!a_ts || !b_ts)) return QL_ERR_INVALID_ARG;
+  if (K % 256 != 0 || M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 23) || K >= ((int64_t)1 << 31))
+    return QL_ERR_UNSUPPORTED;
+  return ql::launch_fp4_gemm(vs, a_codes, a_atoms, a_ts, b_codes, b_atoms, b_ts, M, N, K, Y, as_stream(stream));
 }
 
 ql_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const float* a_tensor_scale,
                      const uint8_t* b_codes, const uint8_t* b_atoms, const float* b_tensor_scale, int64_t M,
                      int64_t N, int64_t K, float* Y, void* stream) {
   NvtxRange nvtx_range("qlora_nf4/nvfp4_gemm");
-  if (M < 1 || N < 1 || K < 1) return QL_ERR_INVALID_ARG;
-  if (!aligned16(a_codes) || !aligned16(a_atoms) || !aligned16(b_codes) || !aligned16(b_atoms) ||
-      !aligned16(Y) || !a_tensor_scale || !b_tensor_scale)
-    return QL_ERR_INVALID_ARG;
-  if (K % 256 != 0 || M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 23) || K >= ((int64_t)1 << 31))
-    return QL_ERR_UNSUPPORTED;
-  return ql::launch_nvfp4_gemm(a_codes, a_atoms, a_tensor_scale, b_codes, b_atoms, b_tensor_scale, M, N, K, Y,
-                               as_stream(stream));
+  return fp4_gemm_checked(16, a_codes, a_atoms, a_tensor_scale, b_codes, b_atoms, b_tensor_scale, M, N, K, Y, stream);
+}
+
+ql_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_t* b_codes, const uint8_t* b_atoms,
+                     int64_t M, int64_t N, int64_t K, float* Y, void* stream) {
+  NvtxRange nvtx_range("qlora_nf4/mxfp4_gemm");
+  return fp4_gemm_checked(32, a_codes, a_atoms, nullptr, b_codes, b_atoms, nullptr, M, N, K, Y, stream);
 }
 
 ql_status qlora_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int64_t t, float lr,

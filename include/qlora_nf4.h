@@ -343,6 +343,31 @@ ql_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const float
                      int64_t N, int64_t K, float* Y, void* stream);
 
 /*
+ * MXFP4 x MXFP4 GEMM on the same tensor-core path ("From FP32 to the 4-Bit
+ * Horizon": MXFP4 is E2M1 elements with one power-of-two E8M0 scale per 32 and
+ * no tensor scale):
+ *   Y[m, n] = sum_k (E2M1(a[m, k]) 2^{k_a[m, k/32]}) (E2M1(b[n, k]) 2^{k_b[n, k/32]})
+ * for A [M, K] and B [N, K] row-major, each quantized by mxfp4_quantize as one
+ * tensor of rows x K elements.
+ *
+ * mxfp4_scale_atoms: scales device uint8 [rows * K/32] (the E8M0 bytes
+ *   mxfp4_quantize writes, row-major) -> atoms device out uint8
+ *   [mxfp4_scale_atoms_bytes(rows, K)]: per 128-row tile and 128-element K
+ *   block, 512 bytes in the layout nvfp4_scale_atoms uses (scale kb < 4 of the
+ *   block now covering elements 32 kb .. 32 kb + 31); rows past `rows` are 0.
+ *   mxfp4_scale_atoms_bytes returns 0 for rows < 1 or K < 128.
+ * mxfp4_gemm: a_codes / b_codes device uint8 [M * K/2] / [N * K/2]; a_atoms /
+ *   b_atoms from mxfp4_scale_atoms with rows = M / N; Y device out fp32 [M, N]
+ *   row-major.  Products are exact and accumulate in fp32 on the tensor cores
+ *   (order unspecified); no scaling after the accumulation.
+ * Constraints and errors as for nvfp4_gemm.
+ */
+size_t mxfp4_scale_atoms_bytes(int64_t rows, int64_t K);
+ql_status mxfp4_scale_atoms(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* atoms, void* stream);
+ql_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_atoms, const uint8_t* b_codes, const uint8_t* b_atoms,
+                     int64_t M, int64_t N, int64_t K, float* Y, void* stream);
+
+/*
  * qlora_adamw_step — one AdamW update of adapter parameters with fp32 states
  * (the paged optimizer: [P2] §2.3 and [P3] "Paged optimizers: surviving the
  * spikes" keep the states in unified memory, paged to host RAM under memory

@@ -144,6 +144,19 @@ def nvfp4_gemm(a_codes, a_S, a_st: float, b_codes, b_S, b_st: float, M: int, N: 
     return A @ B.T
 
 
+def mxfp4_gemm(a_codes, a_k, b_codes, b_k, M: int, N: int, K: int) -> np.ndarray:
+    """Y = A_hat B_hat^T in float64, A [M, K] and B [N, K] row-major MXFP4
+    tensors dequantized by mxfp4_dequant (block scale exponents a_k, b_k).
+
+    [P1] "Lesson 4 of the Finetuning Sessions", "From Turing to Blackwell", as
+    for nvfp4_gemm; "From FP32 to the 4-Bit Horizon": an MXFP4 block scale is a
+    power of two and there is no tensor scale, so every product is exact in
+    float64 and the result is the product of the dequantized tensors."""
+    A = mxfp4_dequant(a_codes, a_k, M * K).reshape(M, K)
+    B = mxfp4_dequant(b_codes, b_k, N * K).reshape(N, K)
+    return A @ B.T
+
+
 def storage_bits_per_element(fmt: str) -> float:
     """Bits per element including the block scales (MX: 8 per 32; NV: 8 per 16;
     the single NVFP4 tensor scale is not counted)."""

@@ -117,6 +117,14 @@ def test_argument_errors_return_before_launch(lib):
     assert L.nvfp4_scale_atoms(fake, 0, 256, fake, s0) == lib.QL_ERR_INVALID_ARG
     assert L.nvfp4_scale_atoms(fake, 128, 192, fake, s0) == lib.QL_ERR_UNSUPPORTED
     assert L.nvfp4_scale_atoms(fake + 8, 128, 256, fake, s0) == lib.QL_ERR_INVALID_ARG
+    mg = lambda M, N, K, a=fake, y=fake: L.mxfp4_gemm(a, fake, fake, fake, M, N, K, y, s0)
+    assert mg(128, 0, 256) == lib.QL_ERR_INVALID_ARG
+    assert mg(128, 128, 256, a=fake + 2) == lib.QL_ERR_INVALID_ARG
+    assert mg(128, 128, 256, y=None) == lib.QL_ERR_INVALID_ARG
+    assert mg(128, 128, 384) == lib.QL_ERR_UNSUPPORTED                                      # K % 256
+    assert mg(128, 1 << 23, 256) == lib.QL_ERR_UNSUPPORTED
+    assert L.mxfp4_scale_atoms(fake, 128, 0, fake, s0) == lib.QL_ERR_INVALID_ARG
+    assert L.mxfp4_scale_atoms(fake, 128, 128, fake, s0) == lib.QL_ERR_UNSUPPORTED
     assert L.qlora_paged_prefetch(None, 64, lib.QL_PAGE_HOST, s0) == lib.QL_ERR_INVALID_ARG
     assert L.qlora_paged_prefetch(fake, 0, lib.QL_PAGE_HOST, s0) == lib.QL_ERR_INVALID_ARG
     assert L.qlora_paged_prefetch(fake, 64, 5, s0) == lib.QL_ERR_INVALID_ARG
@@ -168,3 +176,11 @@ def test_nvfp4_scale_atom_sizes(lib):
     assert lib.nvfp4_scale_atoms_bytes(129, 256) == 2 * 4 * 512       # a partial tile is padded
     assert lib.nvfp4_scale_atoms_bytes(28672, 8192) == 224 * 128 * 512
     assert lib.nvfp4_scale_atoms_bytes(0, 256) == 0
+
+
+def test_mxfp4_scale_atom_sizes(lib):
+    """One 512-byte atom per 128-row tile and 128-element block of K."""
+    assert lib.mxfp4_scale_atoms_bytes(128, 256) == 2 * 512
+    assert lib.mxfp4_scale_atoms_bytes(300, 512) == 3 * 4 * 512
+    assert lib.mxfp4_scale_atoms_bytes(28672, 8192) == 224 * 64 * 512
+    assert lib.mxfp4_scale_atoms_bytes(128, 64) == 0

@@ -159,3 +159,42 @@ def test_nvfp4_gemm_exact_rational_bruteforce():
     v = fp4.e2m1_decode(ca).reshape(M, K)
     scale = np.repeat(np.asarray(Sa, dtype=np.float64), 16).reshape(M, K) * sta
     assert np.allclose(A, v * scale, rtol=2 ** -22, atol=0)
+
+
+def test_mxfp4_gemm_closed_form_per_block_scales():
+    """One E2M1 value per operand, a different power-of-two scale on every
+    32-element block: Y = sum_b 32 v_a v_b 2^(k_a[b] + k_b[b]) exactly, which
+    fails if a block covered 16 elements or the scales of A and B were swapped
+    between rows."""
+    M, N, K = 2, 3, 128
+    va, vb = 1.5, -3.0
+    a = np.full(M * K, fp4.e2m1_encode(np.array([va]))[0], dtype=np.uint8)
+    b = np.full(N * K, fp4.e2m1_encode(np.array([vb]))[0], dtype=np.uint8)
+    ka = np.array([[0, 1, -2, 3], [5, -1, 0, 2]])            # [M, K/32]
+    kb = np.array([[1, 0, 0, -3], [2, 2, -4, 0], [0, -1, 1, 1]])
+    Y = fp4.mxfp4_gemm(a, ka.reshape(-1), b, kb.reshape(-1), M, N, K)
+    for m in range(M):
+        for n in range(N):
+            want = sum(32 * va * vb * 2.0 ** (ka[m, j] + kb[n, j]) for j in range(K // 32))
+            assert Y[m, n] == want
+
+
+def test_mxfp4_gemm_exact_rational_bruteforce():
+    """A small random MXFP4 case against a sum of exact rationals; every
+    dequantized value is a dyadic rational, so the bound is a few ulp of
+    float64."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    M, N, K = 3, 4, 64
+    xa = rng.standard_normal((M, K))
+    xb = rng.standard_normal((N, K)) * 0.03
+    ca, ka = fp4.mxfp4_quantize(xa.reshape(-1))
+    cb, kb = fp4.mxfp4_quantize(xb.reshape(-1))
+    Y = fp4.mxfp4_gemm(ca, ka, cb, kb, M, N, K)
+    v_a = fp4.e2m1_decode(ca).reshape(M, K)
+    v_b = fp4.e2m1_decode(cb).reshape(N, K)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(v_a[m, k])) * Fraction(2) ** int(ka[m * K // 32 + k // 32]) *
+                        Fraction(float(v_b[n, k])) * Fraction(2) ** int(kb[n * K // 32 + k // 32]) for k in range(K))
+            assert abs(Fraction(float(Y[m, n])) - exact) <= abs(exact) * Fraction(1, 2 ** 48) + Fraction(1, 2 ** 100)
