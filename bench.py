@@ -46,7 +46,7 @@ def parse():
     p.add_argument("--no-secondary", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
-    p.add_argument("--leg", choices=["layer", "projection", "smallm", "codec", "merge", "fp4gemm"], default="layer",
+    p.add_argument("--leg", choices=["layer", "projection", "smallm", "codec", "merge", "fp4gemm", "mxfp4gemm"], default="layer",
                    help="with --profile: which workload to run")
     p.add_argument("--profile", action="store_true",
                    help="fixed launch sequence for profilers: exactly --warmup then --steps steps of --leg, "
@@ -552,10 +552,10 @@ def dense_context_leg(layer_set, flush, t_nf4):
 
 def fp4_gemm_leg(q, dev, flush, bf16_peak, layer_set):
     """The next row's native 4-bit product: the gate linear's shape (2048
-    tokens x 28672 x 8192) as an NVFP4 x NVFP4 GEMM on the block-scaled tensor
-    cores (both operands quantized by nvfp4_quantize from the layer's bf16
-    tensors), beside the NF4 path's forward GEMM on the same shape (no
-    adapter).  The FP4 peak is the measured bf16 peak times the nominal 4x."""
+    tokens x 28672 x 8192) as NVFP4 x NVFP4 and MXFP4 x MXFP4 GEMMs on the
+    block-scaled tensor cores (both operands quantized on the GPU from the
+    layer's bf16 tensors), beside the NF4 path's forward GEMM on the same shape
+    (no adapter).  The FP4 peak is the measured bf16 peak times the nominal 4x."""
     import torch
     it = layer_set.items[4]
     M, N, K = layer_set.M, it["N"], it["K"]
@@ -571,9 +571,22 @@ def fp4_gemm_leg(q, dev, flush, bf16_peak, layer_set):
         q.nvfp4_scale_atoms(sc, rows, K, atoms)
         return codes, atoms, ts
 
+    def mx_operand(x, rows):
+        n = x.numel()
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        sc = torch.empty(n // 32, dtype=torch.uint8, device=dev)
+        q.mxfp4_quantize(x, codes, sc)
+        atoms = torch.empty(q.mxfp4_scale_atoms_bytes(rows, K), dtype=torch.uint8, device=dev)
+        q.mxfp4_scale_atoms(sc, rows, K, atoms)
+        return codes, atoms
+
     a, b = operand(it["X"], M), operand(it["W"], N)
     Y = torch.empty(M, N, dtype=torch.float32, device=dev)
     t = _time_calls(lambda: q.nvfp4_gemm(a[0], a[1], a[2], b[0], b[1], b[2], M, N, K, Y), flush, n_warm=3, n=10)
+    del a, b
+    am, bm = mx_operand(it["X"], M), mx_operand(it["W"], N)
+    t_mx = _time_calls(lambda: q.mxfp4_gemm(am[0], am[1], bm[0], bm[1], M, N, K, Y), flush, n_warm=3, n=10)
+    del am, bm
     flop = 2.0 * M * N * K
     Yb = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     ws = torch.empty(max(16, q.qlora_workspace_size(q.QL_OP_FWD, M, N, K, 0)), dtype=torch.uint8, device=dev)
@@ -588,8 +601,11 @@ def fp4_gemm_leg(q, dev, flush, bf16_peak, layer_set):
                                      "frac_fp4_peak": round(flop / t / 1e12 / peak, 3),
                                      "fp4_peak_TFLOPs": round(peak, 1), "shape": [M, N, K],
                                      "nf4_fwd_same_shape_us": round(t_nf4 * 1e6, 2),
-                                     "speedup_over_nf4_fwd": round(t_nf4 / t, 2)}}
-    del a, b, Y, Yb
+                                     "speedup_over_nf4_fwd": round(t_nf4 / t, 2)},
+           "mxfp4_gemm_gate_shape": {"us": round(t_mx * 1e6, 2), "TFLOPs": round(flop / t_mx / 1e12, 1),
+                                     "frac_fp4_peak": round(flop / t_mx / 1e12 / peak, 3), "shape": [M, N, K],
+                                     "speedup_over_nf4_fwd": round(t_nf4 / t_mx, 2)}}
+    del Y, Yb
     torch.cuda.empty_cache()
     return res
 
@@ -752,8 +768,8 @@ def profile_leg(args, q, dev):
     measured step (one stream); projection = the 4096^2 step; smallm = the
     16-token forward on the 28672 x 8192 weight; merge = the adapter merge of
     that weight (bf16 output and re-quantized codes); codec = quantize + double
-    quant of 256 Mi bf16 elements; fp4gemm = the NVFP4 x NVFP4 GEMM at
-    2048 x 4096 x 8192.  Prints per-call device times."""
+    quant of 256 Mi bf16 elements; fp4gemm / mxfp4gemm = the NVFP4 x NVFP4 /
+    MXFP4 x MXFP4 GEMM at 2048 x 4096 x 8192.  Prints per-call device times."""
     import torch
     from synthetic import inputs as S
     w5 = S.WORKLOADS["c5"]
@@ -790,6 +806,21 @@ def profile_leg(args, q, dev):
         Yf = torch.empty(M, N, dtype=torch.float32, device=dev)
         (ac, aa, at), (bc, ba, bt) = fp
         call = lambda: q.nvfp4_gemm(ac, aa, at, bc, ba, bt, M, N, K, Yf)
+    elif args.leg == "mxfp4gemm":
+        # MXFP4 x MXFP4 on the block-scaled tensor cores, 2048 x 4096 x 8192
+        M, N, K = 2048, 4096, 8192
+        fp = []
+        for rows, std, seed in ((M, 1.0, 950), (N, 0.015, 951)):
+            x = S.normal((rows, K), std, seed, device=dev, dtype=torch.bfloat16)
+            codes = torch.empty(rows * K // 2, dtype=torch.uint8, device=dev)
+            sc = torch.empty(rows * K // 32, dtype=torch.uint8, device=dev)
+            q.mxfp4_quantize(x, codes, sc)
+            atoms = torch.empty(q.mxfp4_scale_atoms_bytes(rows, K), dtype=torch.uint8, device=dev)
+            q.mxfp4_scale_atoms(sc, rows, K, atoms)
+            fp.append((codes, atoms))
+        Ym = torch.empty(M, N, dtype=torch.float32, device=dev)
+        (ac, aa), (bc, ba) = fp
+        call = lambda: q.mxfp4_gemm(ac, aa, bc, ba, M, N, K, Ym)
     elif args.leg == "smallm":
         lin = w5.linears[0]
         N, K, r, s, M = lin.N, lin.K, w5.r, w5.s, 16
