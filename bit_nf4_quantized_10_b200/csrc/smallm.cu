@@ -54,6 +54,7 @@ constexpr int MAX_R = 64;
 struct Params {
   int M, N, K, r;
   int kb;            // K / 64 (blocks per weight row)
+  int cw_two;        // a warp's E4M3 constants of a row can span two words or two groups (K / 64 % 4 != 0)
   int parts;         // CTAs' K parts
   int part_k;        // reduction elements per part (WARPS * KV)
   int row_blocks;    // ceil(N / (16 T))
@@ -97,14 +98,16 @@ __device__ __forceinline__ uint32_t expand_pair(uint32_t e4, uint32_t o4, uint32
 }
 
 // Ring stages per warp, and the bytes of one stage: 16 T rows of KV / 2 code
-// bytes, then per (row, block) the 4-byte word holding the block constant (the
-// aligned word around an E4M3 byte, or a plain fp32 constant) and the group
-// scale s_2, as [block][row] words.
+// bytes, then the block constants of those rows: four words per row for E4M3
+// constants (two code words, two group scales), KV / 64 words per row for
+// plain fp32 constants (layouts at issue_codes).
 constexpr int STAGES = 4;
 template <int KV, int T>
 __host__ __device__ constexpr int code_bytes() { return 16 * T * (KV / 2); }
 template <int KV, int T>
-__host__ __device__ constexpr int stage_bytes() { return code_bytes<KV, T>() + 2 * 4 * 16 * T * (KV / 64); }
+__host__ __device__ constexpr int stage_bytes() {
+  return code_bytes<KV, T>() + 4 * 16 * T * (KV / 64 > 4 ? KV / 64 : 4);
+}
 
 // In a stage, row `row`'s 32-byte segment of block j sits at segment
 // j ^ seg_swizzle(row): the 8 rows g a warp's 64-bit fragment read touches
@@ -137,25 +140,52 @@ __device__ __forceinline__ void issue_codes(const Params& p, uint32_t stage, int
     const uint8_t* src = live ? p.codes + (size_t)grow * (p.K / 2) + (size_t)kb0 * 32 + cc * 16 : p.codes;
     cp_async16(stage + row * (KV / 2) + ((((j ^ seg_swizzle<KV>(row)) << 1) | (cc & 1)) << 4), src, live ? 16u : 0u);
   }
-  // constants: one (row, block) pair per lane and round.  An E4M3 byte comes
-  // in the aligned 4-byte word that holds it (a word never straddles a page,
-  // so the bytes around it are safe to read); its byte is picked at decode.
-  constexpr int PAIRS = 16 * T * (KV / 64);
-  const uint32_t cw = stage + code_bytes<KV, T>(), sw = cw + 4 * PAIRS;
+  // Block constants.  Plain fp32 constants: one (row, block) pair per lane and
+  // round, as [block][row] words.  E4M3 constants: the warp's NB = KV / 64
+  // bytes of a row are consecutive, so per row the aligned word holding the
+  // first of them (and the next word if they run past it), and the group scale
+  // s_2 of the first block (and of the last block if it lies in the next group
+  // of 256): [w0 | s0 | w1 | s1] x 16 T rows.  The second pair is only needed
+  // when K / 64 is not a multiple of 4 (p.cw_two).  An aligned word around a
+  // live byte never straddles a page, so the bytes beside it are safe to read.
+  constexpr int ROWS = 16 * T;
+  const uint32_t cw = stage + code_bytes<KV, T>();
+  if (p.wc.absmax) {
+    constexpr int PAIRS = ROWS * (KV / 64);
 #pragma unroll
-  for (int i = 0; i < (PAIRS + 31) / 32; ++i) {
-    const int idx = lane + 32 * i;
-    if (idx < PAIRS) {
-      const int row = idx % (16 * T), j = idx / (16 * T);
-      const int grow = rb * 16 * T + row;
-      const bool live = grow < p.N && j < nbw;
-      const int64_t b = live ? (int64_t)grow * p.kb + kb0 + j : 0;
-      if (p.wc.absmax) {
+    for (int i = 0; i < (PAIRS + 31) / 32; ++i) {
+      const int idx = lane + 32 * i;
+      if (idx < PAIRS) {
+        const int row = idx % ROWS, j = idx / ROWS;
+        const int grow = rb * ROWS + row;
+        const bool live = grow < p.N && j < nbw;
+        const int64_t b = live ? (int64_t)grow * p.kb + kb0 + j : 0;
         cp_async4(cw + 4 * idx, p.wc.absmax + b, live ? 4u : 0u);
-        cp_async4(sw + 4 * idx, p.wc.absmax + b, 0u);
-      } else {
-        cp_async4(cw + 4 * idx, p.wc.absmax_q + (b & ~(int64_t)3), live ? 4u : 0u);
-        cp_async4(sw + 4 * idx, p.wc.scale2 + (b >> 8), live ? 4u : 0u);
+      }
+    }
+  } else {
+    const int rounds = p.cw_two ? 4 : 2;           // word kinds: w0, s0 (, w1, s1)
+#pragma unroll
+    for (int i = 0; i < (4 * ROWS + 31) / 32; ++i) {
+      const int idx = lane + 32 * i, kind = idx / ROWS, row = idx % ROWS;
+      if (kind < rounds) {
+        const int grow = rb * ROWS + row;
+        const bool live = grow < p.N && nbw > 0;
+        const int64_t b0 = live ? (int64_t)grow * p.kb + kb0 : 0, bl = b0 + (nbw > 0 ? nbw - 1 : 0);
+        const void* src = p.wc.absmax_q;
+        bool need = live;
+        if (kind == 0) {
+          src = p.wc.absmax_q + (b0 & ~(int64_t)3);
+        } else if (kind == 1) {
+          src = p.wc.scale2 + (b0 >> 8);
+        } else if (kind == 2) {
+          need = live && (b0 >> 2) != (bl >> 2);
+          src = need ? p.wc.absmax_q + (bl & ~(int64_t)3) : p.wc.absmax_q;
+        } else {
+          need = live && (b0 >> 8) != (bl >> 8);
+          src = need ? p.wc.scale2 + (bl >> 8) : p.wc.scale2;
+        }
+        cp_async4(cw + 4 * idx, src, need ? 4u : 0u);
       }
     }
   }
@@ -190,9 +220,8 @@ __device__ __forceinline__ void compute_frag(const Params& p, const uint8_t* sta
       for (int i = 0; i < 4; ++i) acc[t][n][i] = 0.0f;
   // this thread's decoded constants (its quad index's block, rows g and g+8):
   // each is decoded once per quad and handed to the other three by shuffles
-  constexpr int NB = KV / 64;
+  constexpr int NB = KV / 64, ROWS = 16 * T;
   const uint32_t* cw = reinterpret_cast<const uint32_t*>(stage + code_bytes<KV, T>());
-  const float* sw = reinterpret_cast<const float*>(cw + 16 * T * NB);
   float cmine[T][2];
 #pragma unroll
   for (int t = 0; t < T; ++t)
@@ -200,13 +229,17 @@ __device__ __forceinline__ void compute_frag(const Params& p, const uint8_t* sta
     for (int h = 0; h < 2; ++h) {
       const int row = 16 * t + g + 8 * h;
       const int jq = tq < NB ? tq : 0;
-      const uint32_t word = cw[jq * 16 * T + row];
-      uint32_t q = word;
-      if (!p.wc.absmax) {
-        const int64_t b = (int64_t)(rb * 16 * T + row) * p.kb + kb0 + jq;
-        q = (word >> (8 * (int)(b & 3))) & 0xFFu;
+      if (p.wc.absmax) {
+        cmine[t][h] = __uint_as_float(cw[jq * ROWS + row]);
+      } else {
+        // byte jq of the row's window starting at block b0 (words w0, w1), and
+        // the scale of its group (s0, or s1 past a group boundary)
+        const int64_t b0 = (int64_t)(rb * ROWS + row) * p.kb + kb0, b = b0 + jq;
+        const uint32_t word = (b >> 2) == (b0 >> 2) ? cw[row] : cw[2 * ROWS + row];
+        const uint32_t q = (word >> (8 * (int)(b & 3))) & 0xFFu;
+        const float s2 = __uint_as_float((b >> 8) == (b0 >> 8) ? cw[ROWS + row] : cw[3 * ROWS + row]);
+        cmine[t][h] = decode_const(p.wc, q, s2, mu);
       }
-      cmine[t][h] = decode_const(p.wc, q, sw[jq * 16 * T + row], mu);
     }
 #pragma unroll
   for (int j = 0; j < KV / 64; ++j) {
@@ -460,6 +493,7 @@ ql_status launch_smallm_fwd(const ql_nf4_weight* w, const void* X, int64_t M, co
   p.K = K;
   p.r = r;
   p.kb = K / 64;
+  p.cw_two = (p.kb % 4) != 0;
   p.parts = parts;
   p.part_k = WARPS * sh.kv;
   p.row_blocks = (N + 16 * sh.t - 1) / (16 * sh.t);
